@@ -184,8 +184,9 @@ def quantize_weights_per_channel(W: np.ndarray):
         z32 = np.where(s32 == 0, F32(0), rne(-wlo / s32))
         r = W32 / s32[:, None]
     q = np.where(s32[:, None] == 0, F32(0), np.clip(rne(r) + z32[:, None], 0, U4_MAX))
-    z = z32.astype(np.float16)
-    assert np.all(z.astype(F32) == z32), "zero point not exact in FP16"
+    zi = z32.astype(np.int64)                 # the zero point is an integer (no signed zero)
+    z = zi.astype(np.float16)
+    assert np.all(z.astype(np.int64) == zi), "zero point not exact in FP16"
     return dict(q=q.astype(np.uint8), s=s, z=z)
 
 

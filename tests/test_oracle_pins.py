@@ -289,6 +289,7 @@ def test_per_channel_closed_forms():
     d = oracle.quantize_weights_per_channel(W)
     assert d["s"][0] == np.float16(np.float32(0.5) / np.float32(15))
     assert d["z"][0] == 0 and np.all(d["q"][0] == 15)
+    assert d["z"].view(np.uint16)[0] == 0          # integer zero point: +0, never -0
     assert d["z"][1] == 15 and np.all(d["q"][1] == 0)
 
 
