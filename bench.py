@@ -1,0 +1,464 @@
+"""Benchmark of the QoQ W4A8 hot path on B200: per-token activation
+quantisation + W4A8 GEMM with the fused FP16 epilogue.
+
+One step = every GEMM of the workload once, each preceded by the per-token
+quantisation of its activations:
+  decode  (default): Llama-3-8B linear shapes (K->N) 4096->6144 (qkv),
+                     4096->4096 (o), 4096->28672 (gate+up), 14336->4096 (down)
+                     x M in {1, 4, 16, 64, 256}: 20 GEMMs, HBM-bound regime
+  prefill:           the same shapes x M in {2048, 8192, 16384}, per-token
+                     scales spanning 1e-3..1e1: INT8-tensor-bound regime
+Weights are packed once (offline step, not timed); every GEMM of a step reads
+its own copy of the packed weights, so the weights a step streams (about
+550 MB for decode) exceed the 126 MB L2 and every launch reads from HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode|prefill]
+    python bench.py --impl reference ...   (the CPU oracle, timed on host cores)
+
+Prints one JSON line. Multi-GPU (torchrun): every rank runs the same step on
+its own GPU (independent problems, no collective on the data path; weak
+scaling); the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from w4a8_quantized_gemm_qoq_b200 import inputs  # noqa: E402
+
+METRIC = "W4A8 GEMM TOPS and % of roofline vs M on Llama-3-8B linear shapes (1 B200)"
+GROUP = 128
+SHAPES = [(K, N) for (K, N, _) in inputs.LLAMA3_8B]
+NAMES = [name for (_, _, name) in inputs.LLAMA3_8B]
+WORKLOADS = {
+    "decode": dict(M=inputs.DECODE_M, span=None,
+                   desc="Llama-3-8B decode GEMMs (qkv 4096->6144, o 4096->4096, gate_up 4096->28672, "
+                        "down 14336->4096) x M in {1,4,16,64,256}, g128, act-quant + GEMM"),
+    "prefill": dict(M=inputs.PREFILL_M, span=(-3, 1),
+                    desc="Llama-3-8B prefill GEMMs (same four shapes) x M in {2048,8192,16384}, g128, "
+                         "per-token scales 1e-3..1e1, act-quant + GEMM"),
+}
+
+
+def gemm_bytes(M, N, K):
+    """Algorithmic HBM bytes of one W4A8 GEMM: 4-bit weights, (s, z*s) per
+    group, s_w, X8, s_x and the FP16 output."""
+    return 0.5 * N * K + 2 * N * (K // GROUP) + 2 * N + M * K + 2 * M + 2 * M * N
+
+
+def gemm_ops(M, N, K):
+    return 2.0 * M * N * K
+
+
+def act_bytes(M, K):
+    return 2 * M * K + M * K + 2 * M + 4 * M
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm=float(p["hbm_gbs"]), bf16=float(p["bf16_tflops"]),
+                    bf16_sus=float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), src="measured")
+    except Exception:
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+def roof_us(M, N, K, peaks):
+    """Roofline time: the slower of HBM bytes and INT8 tensor work (INT8 peak =
+    2 x the measured dense bf16 peak, the nominal 4.5/2.25 PFLOP/s ratio)."""
+    t_mem = gemm_bytes(M, N, K) / (peaks["hbm"] * 1e9)
+    t_tc = gemm_ops(M, N, K) / (2.0 * peaks["bf16"] * 1e12)
+    return max(t_mem, t_tc) * 1e6, ("hbm" if t_mem >= t_tc else "tensor")
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Read-only NVML polling (about every 2 ms) of SM clock and clock-event
+    reasons while the timed region runs."""
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, uuid: str | None, period_s: float = 0.002):
+        self.uuid, self.period = uuid, period_s
+        self.samples = []
+        self.max_mhz = None
+        self._stop = None
+        self._th = None
+
+    def __enter__(self):
+        import threading
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByUUID(self.uuid) if self.uuid else pynvml.nvmlDeviceGetHandleByIndex(0)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            get_reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+        except Exception:
+            return self
+        self._stop = threading.Event()
+
+        def poll():
+            while not self._stop.is_set():
+                try:
+                    self.samples.append((pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM), int(get_reasons(h)),
+                                         pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0))
+                except Exception:
+                    pass
+                self._stop.wait(self.period)
+        self._th = threading.Thread(target=poll, daemon=True)
+        self._th.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._th is not None:
+            self._stop.set()
+            self._th.join(timeout=2)
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"], "samples": 0}
+        mhz = sorted(s[0] for s in self.samples)
+        reasons = set()
+        for _, r, _ in self.samples:
+            for bit, nm in self.REASONS.items():
+                if r & bit:
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons),
+                "samples": len(self.samples), "power_w_max": round(max(s[2] for s in self.samples), 1)}
+
+
+# ------------------------------------------------------------- ranks
+
+def max_over_ranks(x: float, device=None) -> float:
+    """Max of a per-rank scalar over the process group (NCCL needs the tensor
+    on this rank's GPU; gloo takes a CPU tensor)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64,
+                     device=device if dist.get_backend() == "nccl" else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, device=None) -> float:
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64,
+                     device=device if dist.get_backend() == "nccl" else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ------------------------------------------------------------- GPU arm
+
+class Problem:
+    def __init__(self, K, N, M, blob, X, span, device):
+        import torch
+        from w4a8_quantized_gemm_qoq_b200 import qoq
+        self.K, self.N, self.M = K, N, M
+        self.blob = blob
+        self.X = X
+        self.X8 = torch.empty((M, K), dtype=torch.int8, device=device)
+        self.s_x = torch.empty((M,), dtype=torch.float16, device=device)
+        self.rowsum = torch.empty((M,), dtype=torch.int32, device=device)
+        self.Y = torch.empty((M, N), dtype=torch.float16, device=device)
+        self.ws = qoq.Workspace.for_shape(M, N, K, GROUP, device)
+
+    def run(self, qoq, ev=None):
+        if ev is not None:
+            ev[0].record()
+        qoq.quantize_act_per_token(self.X, self.X8, self.s_x, self.rowsum)
+        if ev is not None:
+            ev[1].record()
+        qoq.gemm_fp16_out(self.X8, self.s_x, self.blob, self.N, self.K, GROUP, rowsum=self.rowsum, ws=self.ws,
+                          Y=self.Y)
+        if ev is not None:
+            ev[2].record()
+
+
+def build_problems(workload, device, seed):
+    import torch
+    from w4a8_quantized_gemm_qoq_b200 import qoq
+    wl = WORKLOADS[workload]
+    probs = []
+    for si, (K, N) in enumerate(SHAPES):
+        W = torch.from_numpy(inputs.make_weights(N, K, seed=seed + si)).to(device)
+        blob0 = qoq.quantize_weights(W, GROUP)
+        del W
+        for mi, M in enumerate(wl["M"]):
+            blob = blob0 if mi == 0 else blob0.clone()        # one copy per GEMM: no L2 reuse in a step
+            X = torch.from_numpy(inputs.make_activations(M, K, seed=seed + 100 * si + mi,
+                                                         token_scale_span=wl["span"])).to(device)
+            probs.append(Problem(K, N, M, blob, X, wl["span"], device))
+    torch.cuda.synchronize()
+    return probs
+
+
+def run_gpu(args, rank, world, local_rank):
+    import torch
+    from w4a8_quantized_gemm_qoq_b200 import build as qbuild, qoq
+    qbuild.build()
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    peaks = load_peaks()
+    wl = WORKLOADS[args.workload]
+    probs = build_problems(args.workload, device, seed=rank * 1000)
+    stream = torch.cuda.Stream(device)
+    nP = len(probs)
+
+    # One CUDA graph per step shape: a plain one, and EV_GRAPHS copies that
+    # also record per-launch events (external event nodes) for the last steps
+    # of the timed region.
+    EV_GRAPHS = 4
+    with torch.cuda.stream(stream):
+        for p in probs:                      # eager warm-up: library load, attributes, first launch
+            p.run(qoq)
+    stream.synchronize()
+    ev = [[[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for _ in range(nP)]
+          for _ in range(EV_GRAPHS)]
+    plain = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(plain, stream=stream):
+        for p in probs:
+            p.run(qoq)
+    ev_graphs = []
+    for g in range(EV_GRAPHS):
+        cg = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(cg, stream=stream):
+            for p, e in zip(probs, ev[g]):
+                p.run(qoq, e)
+        ev_graphs.append(cg)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            plain.replay()
+    stream.synchronize()
+    for p in probs:
+        assert p.ws.status() == 0, "device status %d" % p.ws.status()
+
+    K = args.steps
+    n_ev = min(EV_GRAPHS, K)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(local_rank).uuid)
+    except Exception:
+        pass
+    with ClockSampler(uuid) as clk:
+        with torch.cuda.stream(stream):
+            t0.record()
+            for k in range(K):
+                j = k - (K - n_ev)
+                (ev_graphs[j] if j >= 0 else plain).replay()
+            t1.record()
+        stream.synchronize()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    step_ms = max_over_ranks(t0.elapsed_time(t1) / K, device) if world > 1 else t0.elapsed_time(t1) / K
+    gemm_ms = [sum(ev[g][i][1].elapsed_time(ev[g][i][2]) for g in range(n_ev)) / n_ev for i in range(nP)]
+    act_ms = [sum(ev[g][i][0].elapsed_time(ev[g][i][1]) for g in range(n_ev)) / n_ev for i in range(nP)]
+    for p in probs:
+        assert p.ws.status() == 0, "device status %d" % p.ws.status()
+
+    ops_step = sum(gemm_ops(p.M, p.N, p.K) for p in probs)
+    per = []
+    tot_bytes = tot_gemm_us = 0.0
+    for i, p in enumerate(probs):
+        us = 1000.0 * gemm_ms[i]
+        b = gemm_bytes(p.M, p.N, p.K)
+        r_us, bound = roof_us(p.M, p.N, p.K, peaks)
+        per.append({"shape": NAMES[SHAPES.index((p.K, p.N))], "K": p.K, "N": p.N, "M": p.M,
+                    "gemm_us": round(us, 3), "act_quant_us": round(1000.0 * act_ms[i], 3),
+                    "TOPS": round(gemm_ops(p.M, p.N, p.K) / us / 1e6, 2), "GBps": round(b / us / 1e3, 1),
+                    "roof_us": round(r_us, 3), "bound": bound, "frac_of_roofline": round(r_us / us, 3)})
+        tot_bytes += b
+        tot_gemm_us += us
+    if args.workload == "decode":
+        achieved = tot_bytes / tot_gemm_us / 1e3
+        roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm"], "unit": "GB/s",
+                    "frac": round(achieved / peaks["hbm"], 4), "traffic": None,
+                    "peak_source": peaks["src"], "kernel": "qoq_gemm_kernel",
+                    "frac_of_time_roofline": round(sum(x["roof_us"] for x in per) / tot_gemm_us, 4)}
+    else:
+        achieved = ops_step / tot_gemm_us / 1e6
+        pk = 2.0 * peaks["bf16"]
+        roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": pk, "unit": "TOPS",
+                    "frac": round(achieved / pk, 4), "traffic": None, "peak_source": peaks["src"] +
+                    " (INT8 = 2 x measured bf16 burst, nominal ratio)", "kernel": "qoq_gemm_kernel",
+                    "frac_of_time_roofline": round(sum(x["roof_us"] for x in per) / tot_gemm_us, 4)}
+
+    e2e = run_e2e(args, probs, qoq, stream) if rank == 0 else None
+    res = {
+        "metric": METRIC, "value": round(world * ops_step / (step_ms * 1e-3) / 1e12, 3), "unit": "TOPS",
+        "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup),
+        "ms_per_step": round(step_ms, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int8", "data": "synthetic",
+        "config": {"workload": wl["desc"], "M": wl["M"], "shapes_K_N": SHAPES, "group_size": GROUP,
+                   "l2": "inputs larger than L2: each GEMM of a step reads its own packed-weight copy "
+                         "(%.0f MB per step)" % (sum(0.5 * p.N * p.K + p.N * p.K / 64 for p in probs) / 1e6),
+                   "launch": "CUDA graph replay of the step; per-launch events from the last %d steps" % n_ev,
+                   "parallelism": "replicas (one independent step per GPU)" if world > 1 else "single GPU"},
+        "roofline": roofline,
+        "gpu_launches": 2 * nP * args.steps,
+        "clocks": clk.summary(),
+        "e2e": e2e,
+        "per_gemm": per,
+    }
+    return res
+
+
+def run_e2e(args, probs, qoq, stream):
+    """Same metric through the public API with host buffers: every step copies
+    each problem's FP16 activations host->device (pinned), runs the two calls,
+    and reads the FP16 output back device->host."""
+    import torch
+    hx = [p.X.cpu().pin_memory() for p in probs]
+    hy = [torch.empty(p.Y.shape, dtype=torch.float16).pin_memory() for p in probs]
+    dx = [torch.empty_like(p.X) for p in probs]
+    h2d = sum(x.numel() * 2 for x in hx)
+    d2h = sum(y.numel() * 2 for y in hy)
+
+    def once():
+        for p, a, b, c in zip(probs, hx, dx, hy):
+            b.copy_(a, non_blocking=True)
+            X8, s_x, rs = qoq.quantize_act_per_token(b, p.X8, p.s_x, p.rowsum)
+            qoq.gemm_fp16_out(X8, s_x, p.blob, p.N, p.K, GROUP, rowsum=rs, ws=p.ws, Y=p.Y)
+            c.copy_(p.Y, non_blocking=True)
+
+    steps = max(1, args.steps)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            once()
+        stream.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            once()
+        e1.record()
+    stream.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    ops = sum(gemm_ops(p.M, p.N, p.K) for p in probs)
+    return {"value": round(ops / (ms * 1e-3) / 1e12, 3), "unit": "TOPS", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 4),
+            "launch": "eager calls through the C ABI, pinned host buffers"}
+
+
+# ------------------------------------------------------------- CPU oracle
+
+def oracle_sample(workload, seed=0):
+    """A bounded sample of the workload for the CPU oracle: the o-projection
+    GEMM (K=N=4096) at M=16 (decode) or M=64 (prefill), weights quantised
+    beforehand (offline), act-quant + int64 GEMM + FP16 epilogue timed."""
+    import oracle
+    K, N = 4096, 4096
+    M = 16 if workload == "decode" else 64
+    W = inputs.make_weights(N, K, seed=seed)
+    X = inputs.make_activations(M, K, seed=seed, token_scale_span=WORKLOADS[workload]["span"])
+    d = oracle.quantize_weights_group(W)
+
+    def once():
+        X8, s_x, rowsum = oracle.quantize_act_per_token(X)
+        acc = oracle.gemm_int(X8, d["Wint"])
+        oracle.epilogue_fp16(acc, s_x, d["s_w"])
+    desc = "o-proj GEMM K=N=4096, M=%d: act quant + int64 triple-loop GEMM + FP16 epilogue " \
+           "(weights pre-quantised)" % M
+    return once, gemm_ops(M, N, K), desc
+
+
+def time_oracle(workload, budget_s=10.0, min_runs=1):
+    once, ops, desc = oracle_sample(workload)
+    once()   # compile/load the C part outside the timing
+    n, t0 = 0, time.perf_counter()
+    while True:
+        once()
+        n += 1
+        el = time.perf_counter() - t0
+        if n >= min_runs and el >= budget_s:
+            break
+    return {"value": round(ops * n / el / 1e12, 6), "unit": "TOPS", "cores": 1, "kind": "oracle",
+            "sample": "%s; %d runs in %.1f s" % (desc, n, el)}
+
+
+def run_reference(args):
+    """--impl reference: the CPU oracle, as it stands, on the host cores."""
+    cb_steps = []
+    once, ops, desc = oracle_sample(args.workload)
+    once()
+    for _ in range(max(0, args.warmup)):
+        once()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        s = time.perf_counter()
+        once()
+        cb_steps.append(time.perf_counter() - s)
+    el = time.perf_counter() - t0
+    val = ops * args.steps / el / 1e12
+    return {"impl": "reference", "metric": METRIC, "value": round(val, 6), "unit": "TOPS", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1000 * el / args.steps, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64",
+            "data": "synthetic",
+            "config": {"workload": WORKLOADS[args.workload]["desc"], "sample": desc},
+            "cpu_baseline": {"value": round(val, 6), "unit": "TOPS", "cores": 1, "kind": "oracle",
+                             "sample": "%s; one sample GEMM per step" % desc},
+            "e2e": {"value": round(val, 6), "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode")
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)))
+        return
+
+    if world > 1:
+        import datetime
+        import torch
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        cpu = time_oracle(args.workload, budget_s=args.cpu_budget)
+    res = run_gpu(args, rank, world, local_rank)
+    if rank == 0:
+        res["cpu_baseline"] = cpu
+        print(json.dumps(res))
+    if world > 1:
+        import torch
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,154 @@
+/*
+ * qoq.h -- C ABI of libqoq.so, the QoQ W4A8 GEMM for NVIDIA B200 (sm_100a).
+ *
+ * What it computes (QServe: W4A8KV4 Quantization and System Co-design for
+ * Efficient LLM Serving, arXiv 2405.04532; paperlayer.ai summary sections 4-6,
+ * study.space summary):
+ *
+ *   Y = diag(s_x) . (X8 . Wint^T) . diag(s_w)
+ *
+ * X8 are FP16 activations quantised per token to INT8 with FP16 scale s_x.
+ * Wint are 4-bit weights brought back to INT8 inside the GEMM: progressive
+ * group quantisation first quantises W per output channel to INT8 with an FP16
+ * scale s_w, kept in the protective range [-119, 119], then quantises each
+ * group of 128 INT8 values along K to UINT4 codes q with an integer scale s and
+ * zero z, so Wint = (q - z) * s = q*s - z*s always fits INT8 with no
+ * saturation. The product runs on INT8 tensor cores with exact INT32
+ * accumulation; a fused epilogue applies s_x and s_w in FP32 and stores FP16.
+ * A per-channel variant (group_size 0) has no INT8 level: UINT4 codes per
+ * output channel with an FP16 scale and zero, the zero-point correction
+ * z * sum_k X8 applied in the epilogue.
+ *
+ * Conventions for every call
+ *   - All buffers are DEVICE memory owned by the caller. The library never
+ *     allocates, frees or synchronises; all work is enqueued on `stream`
+ *     (a cudaStream_t; NULL = the legacy default stream).
+ *   - Arguments are validated before anything is launched; a failed check
+ *     returns its status and enqueues nothing.
+ *   - Shapes: N and K are positive multiples of 128, K <= 65536; M >= 0
+ *     (M == 0 is a no-op). Matrices are row-major and dense.
+ *   - Pointers to matrices, the blob and the workspace must be 16-byte
+ *     aligned; scale and rowsum vectors need their natural alignment.
+ *   - Inputs must be finite.
+ *   - QOQ_ERR_CUDA is returned when a launch fails; errors found on the device
+ *     (a blob whose header does not match the arguments, a pipeline wait that
+ *     ran out) are written to the workspace status word (below).
+ */
+#ifndef QOQ_H
+#define QOQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    QOQ_OK = 0,
+    QOQ_ERR_INVALID_ARG = 1,   /* null pointer, negative size, bad group size   */
+    QOQ_ERR_UNSUPPORTED = 2,   /* N or K not a multiple of 128, K too large      */
+    QOQ_ERR_ALIGNMENT = 3,     /* pointer misaligned                             */
+    QOQ_ERR_WORKSPACE = 4,     /* blob or workspace capacity too small           */
+    QOQ_ERR_BAD_BLOB = 5,      /* blob header does not match N, K, group_size    */
+    QOQ_ERR_CUDA = 6,          /* a CUDA runtime call or launch failed           */
+    QOQ_ERR_TIMEOUT = 7        /* a device pipeline wait ran out (status word)   */
+} qoq_status;
+
+/*
+ * Per-token INT8 quantisation of activations.
+ * (paperlayer.ai summary, section 6 "Evaluation": per-token INT8 activations;
+ *  section 5: QServe fuses this into the preceding layer.)
+ *
+ *   s_x[m]    = FP16(max_k |X[m,k]| / 127)           (FP32 divide, one rounding)
+ *   X8[m,k]   = clamp(RNE(X[m,k] / s_x[m]), -127, 127), 0 when s_x[m] == 0
+ *   rowsum[m] = sum_k X8[m,k]
+ *
+ * X_fp16  [M][K] FP16, read.        X8     [M][K] int8, written.
+ * s_x     [M] FP16, written.        rowsum [M] int32, written; may be NULL.
+ */
+qoq_status qoq_quantize_act_per_token(const void *X_fp16, int64_t M, int64_t K,
+                                      int8_t *X8, void *s_x_fp16, int32_t *rowsum,
+                                      void *stream);
+
+/*
+ * Offline weight quantisation and packing into the compute-order blob.
+ * (paperlayer.ai summary, section 4 "Progressive Group Quantization" and
+ *  section 5 "compute-aware weight reordering"; study.space summary.)
+ *
+ * group_size 128: level 1  s_w[n] = FP16(max_k |W[n,k]| / 119),
+ *                          Q8 = clamp(RNE(W / s_w), -119, 119);
+ *                 level 2  per group of 128 along K with vmin/vmax of Q8:
+ *                          s = max(1, RNE((vmax - vmin) / 15)),
+ *                          z = RNE(-vmin / s), q = clamp(RNE(Q8 / s) + z, 0, 15).
+ * group_size 0:   per channel, range [min(0, min W), max(0, max W)]:
+ *                          s = FP16(range / 15), z = RNE(-min / s) (stored FP16),
+ *                          q = clamp(RNE(W / s) + z, 0, 15).
+ *
+ * Blob layout (little-endian): a 256-byte header (magic 'QOQW', version 1,
+ * N, K, group, block bytes, section offsets, total bytes); code blocks, one per
+ * (128-row n-tile, 128-column k-tile), n-tile major; each block holds the codes
+ * as [chunk c = 0..3][row r = 0..127][16 bytes], where word j of a chunk covers
+ * columns k0 = 32c + 8j .. k0 + 7 and its byte b is q[k0+b] | q[k0+b+4] << 4,
+ * followed in group mode by [row][u8 s, s8 z*s]; then FP16 s_w (or s) [N] and,
+ * per-channel, FP16 z [N], each section 256-byte aligned.
+ *
+ * W_fp16 [N][K] FP16, read. blob: device buffer of *blob_bytes bytes, written.
+ * Size query: blob == NULL stores the required size in *blob_bytes and returns
+ * QOQ_OK without launching. A capacity below it returns QOQ_ERR_WORKSPACE.
+ */
+qoq_status qoq_quantize_weights(const void *W_fp16, int64_t N, int64_t K, int group_size,
+                                void *blob, size_t *blob_bytes, void *stream);
+
+/*
+ * W4A8 GEMM, exact INT32 result (the main loop without the FP scaling).
+ * (paperlayer.ai summary, section 4: weights dequantised to INT8 in the main
+ *  loop, four codes per register op; section 5: subtraction after
+ *  multiplication, zero-point correction in the epilogue.)
+ *
+ * group_size 128: acc[m,n] = sum_k X8[m,k] * Wint[n,k]
+ * group_size 0:   acc[m,n] = sum_k X8[m,k] * q[n,k] - z[n] * rowsum[m]
+ *
+ * X8 [M][K] int8; rowsum [M] int32 (required when group_size == 0, else may be
+ * NULL); blob from qoq_quantize_weights with the same N, K, group_size;
+ * acc [M][N] int32, written.
+ *
+ * Workspace: device memory of *workspace_bytes bytes, ZERO-FILLED by the caller
+ * before its first use; every call that completes leaves it zero-filled again,
+ * so one workspace can serve any number of calls on one stream (calls that may
+ * overlap on the device need separate workspaces). Its first 4 bytes are an
+ * int32 status word: 0, or a qoq_status code (QOQ_ERR_BAD_BLOB,
+ * QOQ_ERR_TIMEOUT) written by the device; after such an error, zero-fill the
+ * workspace again. Size query: workspace == NULL stores the required size for
+ * (M, N, K, group_size) in *workspace_bytes and returns QOQ_OK.
+ */
+qoq_status qoq_w4a8_gemm(const int8_t *X8, const int32_t *rowsum, const void *blob,
+                         int64_t M, int64_t N, int64_t K, int group_size,
+                         int32_t *acc, void *workspace, size_t *workspace_bytes,
+                         void *stream);
+
+/*
+ * W4A8 GEMM with the fused FP16 epilogue: the timed hot path.
+ * (paperlayer.ai summary, section 5: INT8 tensor cores, FP16 outputs,
+ *  per-channel scaling fused into the GEMM epilogue.)
+ *
+ * Y[m,n] = FP16( FP32(acc[m,n]) * (FP32(s_x[m]) * FP32(s_w[n])) )
+ * with acc as in qoq_w4a8_gemm and s_w the blob's per-channel FP16 scale
+ * (group_size 0: the per-channel scale s).
+ *
+ * s_x [M] FP16; Y [M][N] FP16, written. Other arguments, the workspace and
+ * its status word as for qoq_w4a8_gemm.
+ */
+qoq_status qoq_gemm_fp16_out(const int8_t *X8, const void *s_x_fp16, const int32_t *rowsum,
+                             const void *blob, int64_t M, int64_t N, int64_t K, int group_size,
+                             void *Y_fp16, void *workspace, size_t *workspace_bytes,
+                             void *stream);
+
+/* Name of a status code (static string, never NULL). */
+const char *qoq_status_string(qoq_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QOQ_H */

@@ -1,0 +1,87 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every function include/qoq.h declares, answers size queries, and rejects bad
+arguments before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from w4a8_quantized_gemm_qoq_b200 import qoq
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names.update(re.findall(r"\b(qoq_[a-z0-9_]+)\s*\(", src))
+    return names
+
+
+@pytest.fixture(scope="module")
+def L():
+    from w4a8_quantized_gemm_qoq_b200 import build
+    build.build()
+    return qoq.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = _declared()
+    assert {"qoq_quantize_weights", "qoq_quantize_act_per_token", "qoq_w4a8_gemm",
+            "qoq_gemm_fp16_out"} <= names
+    for n in sorted(names):
+        assert hasattr(L, n), n
+    assert L.qoq_status_string(4) == b"QOQ_ERR_WORKSPACE"
+
+
+def test_blob_size_query_matches_layout(L):
+    for N, K, g in [(128, 128, 128), (256, 512, 128), (4096, 14336, 128), (12288, 4096, 0), (384, 640, 0)]:
+        assert qoq.blob_bytes(N, K, g) == oracle.blob_layout(N, K, g)["total"]
+
+
+def test_workspace_size_query(L):
+    small = qoq.workspace_bytes(1, 4096, 4096)
+    big = qoq.workspace_bytes(4096, 4096, 4096)
+    assert 0 < small < big
+    assert qoq.workspace_bytes(0, 128, 128) > 0
+
+
+def _sz(v=0):
+    return ctypes.byref(ctypes.c_size_t(v))
+
+
+def test_argument_validation_without_launch(L):
+    dummy = ctypes.c_void_p(16 * 1024)   # never dereferenced: every call below fails validation first
+    # N / K not multiples of 128, or K too large
+    assert L.qoq_quantize_weights(dummy, 100, 128, 128, dummy, _sz(1 << 30), None) == 2
+    assert L.qoq_quantize_weights(dummy, 128, 130, 128, dummy, _sz(1 << 30), None) == 2
+    assert L.qoq_quantize_weights(dummy, 128, 131072, 128, dummy, _sz(1 << 30), None) == 2
+    # bad group size, negative sizes, null size pointer
+    assert L.qoq_quantize_weights(dummy, 128, 128, 64, dummy, _sz(1 << 30), None) == 1
+    assert L.qoq_quantize_weights(dummy, -128, 128, 128, dummy, _sz(1 << 30), None) == 1
+    assert L.qoq_quantize_weights(dummy, 128, 128, 128, dummy, None, None) == 1
+    # capacity too small
+    assert L.qoq_quantize_weights(dummy, 128, 128, 128, dummy, _sz(100), None) == 4
+    # misaligned weights
+    assert L.qoq_quantize_weights(ctypes.c_void_p(16 * 1024 + 2), 128, 128, 128, dummy, _sz(1 << 30), None) == 3
+    # activation quant
+    assert L.qoq_quantize_act_per_token(dummy, -1, 128, dummy, dummy, None, None) == 1
+    assert L.qoq_quantize_act_per_token(dummy, 4, 100, dummy, dummy, None, None) == 2
+    assert L.qoq_quantize_act_per_token(ctypes.c_void_p(8), 4, 128, dummy, dummy, None, None) == 3
+    assert L.qoq_quantize_act_per_token(None, 4, 128, dummy, dummy, None, None) == 1
+    assert L.qoq_quantize_act_per_token(None, 0, 128, None, None, None, None) == 0   # empty: no-op
+    # GEMM
+    ws = _sz(1 << 30)
+    assert L.qoq_gemm_fp16_out(dummy, dummy, None, dummy, 4, 128, 128, 128, dummy, dummy, None, None) == 1
+    assert L.qoq_gemm_fp16_out(dummy, dummy, None, dummy, 4, 127, 128, 128, dummy, dummy, ws, None) == 2
+    assert L.qoq_gemm_fp16_out(dummy, dummy, None, dummy, 4, 128, 128, 128, dummy, dummy, _sz(8), None) == 4
+    assert L.qoq_gemm_fp16_out(dummy, None, None, dummy, 4, 128, 128, 128, dummy, dummy, ws, None) == 1
+    assert L.qoq_w4a8_gemm(dummy, None, dummy, 4, 128, 128, 0, dummy, dummy, ws, None) == 1   # rowsum needed
+    assert L.qoq_w4a8_gemm(ctypes.c_void_p(16 * 1024 + 8), None, dummy, 4, 128, 128, 128, dummy, dummy, ws,
+                           None) == 3
+    assert L.qoq_w4a8_gemm(dummy, None, dummy, 0, 128, 128, 128, dummy, dummy, ws, None) == 0   # M = 0

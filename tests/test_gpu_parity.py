@@ -1,0 +1,146 @@
+"""CUDA path vs CPU oracle, element by element, through the C ABI.
+
+Bar: bit-exact INT8 codes, FP16 scales, row sums, packed blob bytes and INT32
+accumulators; FP16 outputs within 1 ulp of the oracle's FP32 epilogue.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from w4a8_quantized_gemm_qoq_b200 import inputs, qoq
+from gpu_helpers import check_full, check_sampled, dev, host, assert_fp16_close, torch
+
+pytestmark = [pytest.mark.gpu, pytest.mark.filterwarnings("ignore::RuntimeWarning")]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    t = torch()
+    assert t.cuda.is_available(), "GPU tests need a CUDA device"
+    from w4a8_quantized_gemm_qoq_b200 import build
+    build.build()
+    yield
+
+
+# ----------------------------------------------------------- small, full oracle
+
+def test_config_small_g128():
+    """M=16 N=256 K=512, g=128: the small configuration, every intermediate."""
+    X = inputs.make_activations(16, 512, seed=0)
+    W = inputs.make_weights(256, 512, seed=0)
+    check_full(X, W, 128, "C1")
+
+
+@pytest.mark.parametrize("M", [1, 7, 15, 16, 17, 31, 33, 64, 65, 127, 129, 255, 256, 257, 300])
+def test_ragged_tokens_g128(M):
+    X = inputs.make_activations(M, 640, seed=M)
+    W = inputs.make_weights(384, 640, seed=M)
+    check_full(X, W, 128, "M=%d" % M)
+
+
+@pytest.mark.parametrize("M", [1, 16, 100, 256, 513])
+def test_ragged_tokens_per_channel(M):
+    X = inputs.make_activations(M, 384, seed=100 + M)
+    W = inputs.make_weights(640, 384, seed=100 + M)
+    check_full(X, W, 0, "per-channel M=%d" % M)
+
+
+@pytest.mark.parametrize("N,K", [(128, 128), (128, 1152), (1152, 128), (896, 2176)])
+def test_tile_shapes(N, K):
+    X = inputs.make_activations(24, K, seed=N + K)
+    W = inputs.make_weights(N, K, seed=N + K)
+    check_full(X, W, 128, "N=%d K=%d" % (N, K))
+    check_full(X, W, 0, "per-channel N=%d K=%d" % (N, K))
+
+
+def test_prefill_token_scales():
+    X = inputs.make_activations(300, 1024, seed=3, token_scale_span=(-3, 1))
+    W = inputs.make_weights(512, 1024, seed=3)
+    check_full(X, W, 128, "scaled tokens")
+
+
+def test_degenerate_inputs():
+    """Zero rows and columns, constant rows, one-hot tokens."""
+    K, N = 256, 256
+    W = inputs.make_weights(N, K, seed=4)
+    W[3] = 0
+    W[7] = 0.05
+    W[9] = -2.0
+    W[:, 5] = 0
+    X = inputs.make_activations(40, K, seed=4)
+    X[0] = 0
+    X[1] = 0.25
+    X[2] = 0
+    X[2, 77] = -3.0
+    check_full(X, W, 128, "degenerate")
+    check_full(X, W, 0, "degenerate per-channel")
+
+
+def test_identity_reads_back_dequantised_weights():
+    """K one-hot tokens: acc = 127 * Wint^T, i.e. the GEMM returns the whole
+    dequantised weight matrix, which pins the packed layout end to end."""
+    K, N = 384, 256
+    W = inputs.make_weights(N, K, seed=5)
+    X = np.zeros((K, K), dtype=np.float16)
+    X[np.arange(K), np.arange(K)] = 1.0
+    r, g = check_full(X, W, 128, "identity")
+    assert np.array_equal(g["acc"], 127 * r["w"]["Wint"].astype(np.int32).T)
+
+
+def test_workspace_reuse_and_zero_m():
+    X = inputs.make_activations(33, 512, seed=6)
+    W = inputs.make_weights(256, 512, seed=6)
+    Wd, Xd = dev(W), dev(X)
+    blob = qoq.quantize_weights(Wd, 128)
+    X8, s_x, rs = qoq.quantize_act_per_token(Xd)
+    ws = qoq.Workspace.for_shape(33, 256, 512)
+    y1 = host(qoq.gemm_fp16_out(X8, s_x, blob, 256, 512, ws=ws))
+    y2 = host(qoq.gemm_fp16_out(X8, s_x, blob, 256, 512, ws=ws))
+    assert np.array_equal(y1.view(np.uint16), y2.view(np.uint16))
+    assert not ws.buf.any().item()
+    # M = 0 is a no-op that succeeds
+    e = torch().empty((0, 512), dtype=torch().int8, device="cuda")
+    out = qoq.gemm_fp16_out(e, s_x[:0], blob, 256, 512, ws=ws)
+    assert out.shape == (0, 256)
+
+
+def test_bad_blob_header_reported_on_device():
+    """A blob whose header does not match the arguments: the kernel does no
+    work and writes QOQ_ERR_BAD_BLOB to the workspace status word."""
+    W = inputs.make_weights(256, 512, seed=7)
+    blob = qoq.quantize_weights(dev(W), 128)
+    X8 = torch().zeros((16, 512), dtype=torch().int8, device="cuda")
+    s_x = torch().ones((16,), dtype=torch().float16, device="cuda")
+    ws = qoq.Workspace.for_shape(16, 256, 512)
+    Y = torch().full((16, 128), 7.0, dtype=torch().float16, device="cuda")
+    # claim N = 128 for a blob built with N = 256
+    qoq.gemm_fp16_out(X8, s_x, blob, 128, 512, ws=ws, Y=Y)
+    torch().cuda.synchronize()
+    assert ws.status() == 5
+    assert bool((Y == 7.0).all().item())
+
+
+# ------------------------------------------------------- full sizes, sampled oracle
+
+@pytest.mark.parametrize("K,N", [(4096, 6144), (4096, 4096), (4096, 28672), (14336, 4096)])
+@pytest.mark.parametrize("M", [1, 4, 16, 64, 256])
+def test_llama3_8b_decode_shapes(M, K, N):
+    check_sampled(M, N, K, 128, seed=M + N)
+
+
+@pytest.mark.parametrize("K,N", [(4096, 28672), (14336, 4096)])
+@pytest.mark.parametrize("M", [2048, 16384])
+def test_llama3_8b_prefill_shapes(M, K, N):
+    check_sampled(M, N, K, 128, seed=M + K, token_scale_span=(-3, 1), rows=12)
+
+
+@pytest.mark.parametrize("K,N,M", [(8192, 24576, 1), (8192, 8192, 16), (8192, 49152, 128), (24576, 8192, 512),
+                                   (8192, 8192, 4096)])
+def test_qwen15_72b_shapes(M, K, N):
+    check_sampled(M, N, K, 128, seed=N + M, std=0.01, rows=12)
+
+
+@pytest.mark.parametrize("K,N", [(4096, 12288), (4096, 4096), (4096, 22016), (11008, 4096)])
+@pytest.mark.parametrize("M", [1, 8, 64, 1024])
+def test_llama2_7b_per_channel_shapes(M, K, N):
+    check_sampled(M, N, K, 0, seed=K + M, rows=12)

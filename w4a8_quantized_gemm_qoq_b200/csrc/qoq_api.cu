@@ -1,0 +1,126 @@
+// C-ABI entry points of libqoq.so (declared in include/qoq.h): argument
+// validation, size queries and dispatch to the kernels. Nothing here
+// allocates, frees or synchronises; every launch goes to the caller's stream.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "qoq_internal.h"
+
+using namespace qoq;
+
+namespace {
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+qoq_status check_nk(int64_t N, int64_t K) {
+    if (N <= 0 || K <= 0) return QOQ_ERR_INVALID_ARG;
+    if (N % kTileN != 0 || K % kTileK != 0 || K > kMaxK || N > (int64_t)INT32_MAX / 2) return QOQ_ERR_UNSUPPORTED;
+    return QOQ_OK;
+}
+
+qoq_status check_group(int group) {
+    return (group == kGroup || group == 0) ? QOQ_OK : QOQ_ERR_INVALID_ARG;
+}
+
+qoq_status gemm_common(const int8_t *X8, const void *s_x, const int32_t *rowsum, const void *blob, int64_t M,
+                       int64_t N, int64_t K, int group, void *out, bool fp16_out, void *ws, size_t *ws_bytes,
+                       void *stream) {
+    if (ws_bytes == nullptr) return QOQ_ERR_INVALID_ARG;
+    if (M < 0 || M > INT32_MAX) return QOQ_ERR_INVALID_ARG;
+    qoq_status st = check_nk(N, K);
+    if (st != QOQ_OK) return st;
+    if ((st = check_group(group)) != QOQ_OK) return st;
+    if (M * N > (int64_t)1 << 40) return QOQ_ERR_UNSUPPORTED;
+    const size_t need = workspace_bytes_for(M);
+    if (ws == nullptr) {
+        *ws_bytes = need;
+        return QOQ_OK;
+    }
+    if (*ws_bytes < need) return QOQ_ERR_WORKSPACE;
+    if (M == 0) return QOQ_OK;
+    if (X8 == nullptr || blob == nullptr || out == nullptr) return QOQ_ERR_INVALID_ARG;
+    if (fp16_out && s_x == nullptr) return QOQ_ERR_INVALID_ARG;
+    if (group == 0 && rowsum == nullptr) return QOQ_ERR_INVALID_ARG;
+    if (!aligned(X8, 16) || !aligned(blob, 16) || !aligned(out, 16) || !aligned(ws, 16)) return QOQ_ERR_ALIGNMENT;
+    if ((s_x && !aligned(s_x, 2)) || (rowsum && !aligned(rowsum, 4))) return QOQ_ERR_ALIGNMENT;
+    GemmArgs a;
+    a.X8 = X8;
+    a.s_x = s_x;
+    a.rowsum = rowsum;
+    a.blob = blob;
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.group = group;
+    a.out = out;
+    a.fp16_out = fp16_out;
+    a.ws = ws;
+    return launch_gemm(a, static_cast<cudaStream_t>(stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+qoq_status qoq_quantize_act_per_token(const void *X_fp16, int64_t M, int64_t K, int8_t *X8, void *s_x_fp16,
+                                      int32_t *rowsum, void *stream) {
+    if (M < 0 || M > INT32_MAX || K <= 0) return QOQ_ERR_INVALID_ARG;
+    if (K % kTileK != 0 || K > kMaxK) return QOQ_ERR_UNSUPPORTED;
+    if (M == 0) return QOQ_OK;
+    if (X_fp16 == nullptr || X8 == nullptr || s_x_fp16 == nullptr) return QOQ_ERR_INVALID_ARG;
+    if (!aligned(X_fp16, 16) || !aligned(X8, 16) || !aligned(s_x_fp16, 2) || (rowsum && !aligned(rowsum, 4)))
+        return QOQ_ERR_ALIGNMENT;
+    return launch_act_quant(X_fp16, M, K, X8, s_x_fp16, rowsum, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? QOQ_OK
+               : QOQ_ERR_CUDA;
+}
+
+qoq_status qoq_quantize_weights(const void *W_fp16, int64_t N, int64_t K, int group_size, void *blob,
+                                size_t *blob_bytes, void *stream) {
+    if (blob_bytes == nullptr) return QOQ_ERR_INVALID_ARG;
+    qoq_status st = check_nk(N, K);
+    if (st != QOQ_OK) return st;
+    if ((st = check_group(group_size)) != QOQ_OK) return st;
+    const BlobLayout L = blob_layout(N, K, group_size);
+    if (blob == nullptr) {
+        *blob_bytes = (size_t)L.total;
+        return QOQ_OK;
+    }
+    if (*blob_bytes < (size_t)L.total) return QOQ_ERR_WORKSPACE;
+    if (W_fp16 == nullptr) return QOQ_ERR_INVALID_ARG;
+    if (!aligned(W_fp16, 16) || !aligned(blob, 16)) return QOQ_ERR_ALIGNMENT;
+    return launch_weight_quant(W_fp16, N, K, group_size, blob, L, static_cast<cudaStream_t>(stream)) ==
+                   cudaSuccess
+               ? QOQ_OK
+               : QOQ_ERR_CUDA;
+}
+
+qoq_status qoq_w4a8_gemm(const int8_t *X8, const int32_t *rowsum, const void *blob, int64_t M, int64_t N,
+                         int64_t K, int group_size, int32_t *acc, void *workspace, size_t *workspace_bytes,
+                         void *stream) {
+    return gemm_common(X8, nullptr, rowsum, blob, M, N, K, group_size, acc, false, workspace, workspace_bytes,
+                       stream);
+}
+
+qoq_status qoq_gemm_fp16_out(const int8_t *X8, const void *s_x_fp16, const int32_t *rowsum, const void *blob,
+                             int64_t M, int64_t N, int64_t K, int group_size, void *Y_fp16, void *workspace,
+                             size_t *workspace_bytes, void *stream) {
+    return gemm_common(X8, s_x_fp16, rowsum, blob, M, N, K, group_size, Y_fp16, true, workspace,
+                       workspace_bytes, stream);
+}
+
+const char *qoq_status_string(qoq_status status) {
+    switch (status) {
+        case QOQ_OK: return "QOQ_OK";
+        case QOQ_ERR_INVALID_ARG: return "QOQ_ERR_INVALID_ARG";
+        case QOQ_ERR_UNSUPPORTED: return "QOQ_ERR_UNSUPPORTED";
+        case QOQ_ERR_ALIGNMENT: return "QOQ_ERR_ALIGNMENT";
+        case QOQ_ERR_WORKSPACE: return "QOQ_ERR_WORKSPACE";
+        case QOQ_ERR_BAD_BLOB: return "QOQ_ERR_BAD_BLOB";
+        case QOQ_ERR_CUDA: return "QOQ_ERR_CUDA";
+        case QOQ_ERR_TIMEOUT: return "QOQ_ERR_TIMEOUT";
+    }
+    return "QOQ_ERR_UNKNOWN";
+}
+
+}  // extern "C"

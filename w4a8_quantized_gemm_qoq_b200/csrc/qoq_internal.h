@@ -1,0 +1,82 @@
+// Host-side declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/qoq.h"
+
+namespace qoq {
+
+constexpr int kTileN = 128;        // weight rows per tile (TMEM lanes)
+constexpr int kTileK = 128;        // K per tile = one quantisation group
+constexpr int kGroup = 128;
+constexpr int kMaxK = 65536;
+constexpr int kMaxGrid = 256;      // upper bound of the persistent grid (>= SM count)
+constexpr uint32_t kMagic = 0x57514F51u;   // 'Q','O','Q','W'
+constexpr uint32_t kVersion = 1u;
+constexpr int kHeaderBytes = 256;
+
+// Byte layout of a packed weight blob.
+struct BlobLayout {
+    int64_t NT, KT;
+    int64_t block;      // bytes per (n-tile, k-tile) block
+    int64_t off_codes, off_scale, off_zero, total;
+};
+
+inline int64_t align256(int64_t x) { return (x + 255) / 256 * 256; }
+
+inline BlobLayout blob_layout(int64_t N, int64_t K, int group) {
+    BlobLayout L;
+    L.NT = N / kTileN;
+    L.KT = K / kTileK;
+    L.block = 8192 + (group ? 256 : 0);
+    L.off_codes = kHeaderBytes;
+    L.off_scale = L.off_codes + L.NT * L.KT * L.block;
+    if (group) {
+        L.off_zero = 0;
+        L.total = L.off_scale + align256(2 * N);
+    } else {
+        L.off_zero = L.off_scale + align256(2 * N);
+        L.total = L.off_zero + align256(2 * N);
+    }
+    return L;
+}
+
+// Token-tile width (MMA N) chosen for M tokens.
+inline int token_tile_for(int64_t M) {
+    if (M <= 16) return 16;
+    if (M <= 32) return 32;
+    if (M <= 64) return 64;
+    if (M <= 128) return 128;
+    return 256;
+}
+
+// Workspace: [0, 256) status word + reserved; then int32 counters [kMaxGrid];
+// then int32 partial tiles [kMaxGrid][tok][128].
+inline size_t workspace_bytes_for(int64_t M) {
+    const int tok = token_tile_for(M);
+    return 256 + sizeof(int32_t) * kMaxGrid + sizeof(int32_t) * (size_t)kMaxGrid * tok * kTileN;
+}
+
+// Kernel launchers (return cudaSuccess or the launch error).
+cudaError_t launch_act_quant(const void *X, int64_t M, int64_t K, int8_t *X8, void *s_x, int32_t *rowsum,
+                             cudaStream_t stream);
+cudaError_t launch_weight_quant(const void *W, int64_t N, int64_t K, int group, void *blob,
+                                const BlobLayout &L, cudaStream_t stream);
+
+struct GemmArgs {
+    const int8_t *X8;
+    const void *s_x;
+    const int32_t *rowsum;
+    const void *blob;
+    int64_t M, N, K;
+    int group;
+    void *out;          // int32 [M][N] or fp16 [M][N]
+    bool fp16_out;
+    void *ws;
+};
+qoq_status launch_gemm(const GemmArgs &a, cudaStream_t stream);
+
+}  // namespace qoq

@@ -1,0 +1,170 @@
+"""ctypes binding of libqoq.so (the C ABI in include/qoq.h).
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels. PyTorch supplies device memory and the current stream. There is no
+CPU fallback: if the library is missing or no CUDA device is present the calls
+raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libqoq.so")
+
+QOQ_OK = 0
+STATUS = {0: "QOQ_OK", 1: "QOQ_ERR_INVALID_ARG", 2: "QOQ_ERR_UNSUPPORTED", 3: "QOQ_ERR_ALIGNMENT",
+          4: "QOQ_ERR_WORKSPACE", 5: "QOQ_ERR_BAD_BLOB", 6: "QOQ_ERR_CUDA", 7: "QOQ_ERR_TIMEOUT"}
+TILE = 128
+GROUP = 128
+
+_lib = None
+
+
+class QoQError(RuntimeError):
+    def __init__(self, fn, code):
+        super().__init__("%s failed: %s (%d)" % (fn, STATUS.get(code, "?"), code))
+        self.code = code
+
+
+def lib() -> ctypes.CDLL:
+    """Open libqoq.so (built in-tree by w4a8_quantized_gemm_qoq_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError("libqoq.so is not built (%s); run python -m w4a8_quantized_gemm_qoq_b200.build"
+                              % LIB_PATH)
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t)
+        L.qoq_quantize_act_per_token.argtypes = [vp, i64, i64, vp, vp, vp, vp]
+        L.qoq_quantize_weights.argtypes = [vp, i64, i64, i32, vp, sz, vp]
+        L.qoq_w4a8_gemm.argtypes = [vp, vp, vp, i64, i64, i64, i32, vp, vp, sz, vp]
+        L.qoq_gemm_fp16_out.argtypes = [vp, vp, vp, vp, i64, i64, i64, i32, vp, vp, sz, vp]
+        L.qoq_status_string.argtypes = [ctypes.c_int]
+        L.qoq_status_string.restype = ctypes.c_char_p
+        for f in (L.qoq_quantize_act_per_token, L.qoq_quantize_weights, L.qoq_w4a8_gemm, L.qoq_gemm_fp16_out):
+            f.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _check(fn, code):
+    if code != QOQ_OK:
+        raise QoQError(fn, code)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _cuda_tensor(t, dtype, name):
+    import torch
+    if not (isinstance(t, torch.Tensor) and t.is_cuda):
+        raise TypeError("%s must be a CUDA tensor" % name)
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    return t
+
+
+# ------------------------------------------------------------------ sizes
+
+def blob_bytes(N: int, K: int, group_size: int = GROUP) -> int:
+    n = ctypes.c_size_t(0)
+    _check("qoq_quantize_weights", lib().qoq_quantize_weights(None, N, K, group_size, None, ctypes.byref(n), None))
+    return n.value
+
+
+def workspace_bytes(M: int, N: int, K: int, group_size: int = GROUP) -> int:
+    n = ctypes.c_size_t(0)
+    _check("qoq_gemm_fp16_out", lib().qoq_gemm_fp16_out(None, None, None, None, M, N, K, group_size, None, None,
+                                                        ctypes.byref(n), None))
+    return n.value
+
+
+# ------------------------------------------------------------------ calls
+
+def quantize_act_per_token(X, X8=None, s_x=None, rowsum=None, stream=None):
+    """X [M][K] fp16 -> (X8 int8 [M][K], s_x fp16 [M], rowsum int32 [M])."""
+    import torch
+    X = _cuda_tensor(X, torch.float16, "X")
+    M, K = X.shape
+    X8 = torch.empty((M, K), dtype=torch.int8, device=X.device) if X8 is None else X8
+    s_x = torch.empty((M,), dtype=torch.float16, device=X.device) if s_x is None else s_x
+    rowsum = torch.empty((M,), dtype=torch.int32, device=X.device) if rowsum is None else rowsum
+    _check("qoq_quantize_act_per_token",
+           lib().qoq_quantize_act_per_token(_ptr(X), M, K, _ptr(X8), _ptr(s_x), _ptr(rowsum), _stream(stream)))
+    return X8, s_x, rowsum
+
+
+def quantize_weights(W, group_size: int = GROUP, blob=None, stream=None):
+    """W [N][K] fp16 -> packed blob (uint8 tensor) in compute order."""
+    import torch
+    W = _cuda_tensor(W, torch.float16, "W")
+    N, K = W.shape
+    need = blob_bytes(N, K, group_size)
+    blob = torch.empty((need,), dtype=torch.uint8, device=W.device) if blob is None else blob
+    n = ctypes.c_size_t(blob.numel())
+    _check("qoq_quantize_weights",
+           lib().qoq_quantize_weights(_ptr(W), N, K, group_size, _ptr(blob), ctypes.byref(n), _stream(stream)))
+    return blob
+
+
+class Workspace:
+    """Zero-filled device workspace for the GEMM calls (the library leaves it
+    zero-filled after each call; its first int32 is the device status word)."""
+
+    def __init__(self, nbytes: int, device="cuda"):
+        import torch
+        self.buf = torch.zeros((nbytes + 15) // 16 * 16, dtype=torch.uint8, device=device)
+
+    @classmethod
+    def for_shape(cls, M, N, K, group_size=GROUP, device="cuda"):
+        return cls(workspace_bytes(M, N, K, group_size), device)
+
+    def status(self) -> int:
+        return int(self.buf[:4].view(dtype=__import__("torch").int32).item())
+
+    def reset(self):
+        self.buf.zero_()
+
+
+def w4a8_gemm(X8, blob, N, K, group_size=GROUP, rowsum=None, ws=None, acc=None, stream=None):
+    """Exact INT32 GEMM: acc [M][N]."""
+    import torch
+    X8 = _cuda_tensor(X8, torch.int8, "X8")
+    M = X8.shape[0]
+    ws = ws or Workspace.for_shape(M, N, K, group_size, X8.device)
+    acc = torch.empty((M, N), dtype=torch.int32, device=X8.device) if acc is None else acc
+    n = ctypes.c_size_t(ws.buf.numel())
+    _check("qoq_w4a8_gemm", lib().qoq_w4a8_gemm(_ptr(X8), _ptr(rowsum), _ptr(blob), M, N, K, group_size, _ptr(acc),
+                                                _ptr(ws.buf), ctypes.byref(n), _stream(stream)))
+    return acc
+
+
+def gemm_fp16_out(X8, s_x, blob, N, K, group_size=GROUP, rowsum=None, ws=None, Y=None, stream=None):
+    """W4A8 GEMM with fused FP16 epilogue: Y [M][N] fp16."""
+    import torch
+    X8 = _cuda_tensor(X8, torch.int8, "X8")
+    M = X8.shape[0]
+    ws = ws or Workspace.for_shape(M, N, K, group_size, X8.device)
+    Y = torch.empty((M, N), dtype=torch.float16, device=X8.device) if Y is None else Y
+    n = ctypes.c_size_t(ws.buf.numel())
+    _check("qoq_gemm_fp16_out", lib().qoq_gemm_fp16_out(_ptr(X8), _ptr(s_x), _ptr(rowsum), _ptr(blob), M, N, K,
+                                                        group_size, _ptr(Y), _ptr(ws.buf), ctypes.byref(n),
+                                                        _stream(stream)))
+    return Y
+
+
+def linear(X, blob, N, K, group_size=GROUP, ws=None, stream=None):
+    """The whole hot path: per-token quantisation of X then the W4A8 GEMM."""
+    X8, s_x, rowsum = quantize_act_per_token(X, stream=stream)
+    return gemm_fp16_out(X8, s_x, blob, N, K, group_size, rowsum=rowsum, ws=ws, stream=stream)
