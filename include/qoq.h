@@ -44,6 +44,9 @@
 extern "C" {
 #endif
 
+/* Leading workspace bytes that hold control words (status + flags). */
+#define QOQ_WORKSPACE_CONTROL_BYTES 1280
+
 typedef enum {
     QOQ_OK = 0,
     QOQ_ERR_INVALID_ARG = 1,   /* null pointer, negative size, bad group size   */
@@ -114,12 +117,14 @@ qoq_status qoq_quantize_weights(const void *W_fp16, int64_t N, int64_t K, int gr
  * acc [M][N] int32, written.
  *
  * Workspace: device memory of *workspace_bytes bytes, ZERO-FILLED by the caller
- * before its first use; every call that completes leaves it zero-filled again,
- * so one workspace can serve any number of calls on one stream (calls that may
- * overlap on the device need separate workspaces). Its first 4 bytes are an
- * int32 status word: 0, or a qoq_status code (QOQ_ERR_BAD_BLOB,
- * QOQ_ERR_TIMEOUT) written by the device; after such an error, zero-fill the
- * workspace again. Size query: workspace == NULL stores the required size for
+ * before its first use. Its first QOQ_WORKSPACE_CONTROL_BYTES bytes are
+ * control words that every call which completes leaves zero again (an int32
+ * status word at offset 0, then cross-CTA flags); the rest is scratch for the
+ * stream-K partial sums. So one workspace serves any number of calls on one
+ * stream; calls that may overlap on the device need separate workspaces. The
+ * status word is 0, or a qoq_status code (QOQ_ERR_BAD_BLOB, QOQ_ERR_TIMEOUT)
+ * written by the device; after such an error, zero-fill the control bytes
+ * again. Size query: workspace == NULL stores the required size for
  * (M, N, K, group_size) in *workspace_bytes and returns QOQ_OK.
  */
 qoq_status qoq_w4a8_gemm(const int8_t *X8, const int32_t *rowsum, const void *blob,

@@ -55,7 +55,7 @@ def check_full(X, W, group, what=""):
     assert np.array_equal(g["blob"], r["blob"]), what + " blob"
     assert np.array_equal(g["acc"], r["acc"]), what + " acc"
     assert_fp16_close(g["Y"], r["Y"], what + " Y")
-    assert not g["ws"].buf.any().item(), what + " workspace not left zero-filled"
+    assert g["ws"].control_clear(), what + " workspace control words not left zero"
     return r, g
 
 
@@ -112,5 +112,5 @@ def check_sampled(M, N, K, group, seed=0, std=0.02, token_scale_span=None, rows=
         got_y = host(Y[rows_d][:, cols])
         assert np.array_equal(got_acc, ref_acc), "acc tile %d" % nt
         assert_fp16_close(got_y, ref_y, "Y tile %d" % nt)
-    assert not ws.buf.any().item()
+    assert ws.control_clear()
     return ncols

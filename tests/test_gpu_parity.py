@@ -97,7 +97,7 @@ def test_workspace_reuse_and_zero_m():
     y1 = host(qoq.gemm_fp16_out(X8, s_x, blob, 256, 512, ws=ws))
     y2 = host(qoq.gemm_fp16_out(X8, s_x, blob, 256, 512, ws=ws))
     assert np.array_equal(y1.view(np.uint16), y2.view(np.uint16))
-    assert not ws.buf.any().item()
+    assert ws.control_clear()
     # M = 0 is a no-op that succeeds
     e = torch().empty((0, 512), dtype=torch().int8, device="cuda")
     out = qoq.gemm_fp16_out(e, s_x[:0], blob, 256, 512, ws=ws)

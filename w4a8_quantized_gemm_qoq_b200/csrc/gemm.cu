@@ -23,13 +23,18 @@
 //     scalar. 8 nibbles per 32-bit word decode with and/shift, one 32-bit
 //     multiply-add (q*s <= 240 and q*s + 128 - z*s in [7, 249] never carry
 //     between bytes) and one xor that turns excess-128 bytes into int8.
-//   * warp roles: 1 TMA producer, 1 MMA issuer, two dequant warpgroups that
-//     alternate k-tiles, one epilogue warpgroup; mbarrier rings between them.
-//   * persistent stream-K: the (token tile, n-tile, k-tile) blocks are split
-//     evenly over at most one CTA per SM; a tile cut between CTAs is summed
-//     exactly in INT32 in a workspace slot (integer addition is associative,
-//     so the result does not depend on the order), and the last contributor
-//     runs the epilogue and re-zeros the slot.
+//   * warp roles: 1 TMA producer warp, 1 MMA warp, two dequant warpgroups that
+//     alternate pipeline units, one epilogue warpgroup; the role loops are
+//     warp-uniform and lane 0 issues TMA / MMA / commit.
+//   * a pipeline unit is up to KB consecutive k-tiles of one n-tile: one bulk
+//     copy of the packed weights, one TMA per token tile, one TMEM A buffer,
+//     one commit that frees both the shared-memory stage and the TMEM buffer.
+//   * persistent stream-K at k-tile granularity: the (token tile, n-tile,
+//     k-tile) blocks are split evenly over at most one CTA per SM. A tile cut
+//     between CTAs is finished by its owner -- the CTA holding the tile's
+//     first k-tile, which it reaches last -- after the other contributors
+//     (which reach their share of the tile first) have stored their INT32
+//     partial sums and raised a flag. The sum is exact in any order.
 #include <algorithm>
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -48,31 +53,35 @@ constexpr int kWarpDequant0 = 4;         // warps 4..11: two dequant warpgroups
 constexpr int kWarpEpilogue = 12;        // warps 12..15
 constexpr uint64_t kDrainNs = 100ull * 1000ull * 1000ull;   // 100 ms
 
-__device__ __forceinline__ long long lmin(long long a, long long b) { return a < b ? a : b; }
-
-__host__ __device__ constexpr int pow2_at_least(int x) {
-    int p = 32;
-    while (p < x) p <<= 1;
-    return p;
-}
-
 template <int TOK, int MODE>
 struct GemmCfg {
-    static constexpr int kXBytes = TOK * 128;                   // token tile, 128 k
-    static constexpr int kWBytes = MODE == 0 ? 8448 : 8192;     // codes (+ s, z*s)
+    // KB = k-tiles per pipeline unit: two for decode-sized token tiles (halves
+    // the barrier and issue work per weight byte), one for wide token tiles
+    // (their MMA work per k-tile already hides it, and shared memory holds
+    // fewer wide stages).
+    static constexpr int kKB = TOK <= 64 ? 2 : 1;
+    static constexpr int kXTile = TOK * 128;                    // token tile, 128 k
+    static constexpr int kWTile = MODE == 0 ? 8448 : 8192;      // codes (+ s, z*s) per k-tile
+    static constexpr int kXBytes = kKB * kXTile;
+    static constexpr int kWBytes = kKB * kWTile;
     static constexpr int kStageBytes = (kXBytes + kWBytes + 1023) / 1024 * 1024;
     static constexpr int kSmemLimit = 232448;                   // 227 KB per CTA
     static constexpr int kReserve = 2048;                       // alignment slack + barriers
-    static constexpr int kStagesFit = (kSmemLimit - kReserve) / kStageBytes;
-    static constexpr int kStages = kStagesFit > 16 ? 16 : kStagesFit;
-    static constexpr int kAStages = 4;                          // TMEM A buffers (32 cols each)
     static constexpr int kAccBufs = TOK <= 128 ? 2 : 1;
     static constexpr int kACol0 = kAccBufs * TOK;
-    static constexpr int kTmemCols = pow2_at_least(kACol0 + kAStages * 32);
+    // One CTA per SM (shared memory use guarantees it), so the CTA takes all
+    // 512 TMEM columns: accumulators first, then one A buffer per stage
+    // (32 columns per dequantised 128x128 k-tile).
+    static constexpr int kTmemCols = 512;
+    static constexpr int kStagesSmem = (kSmemLimit - kReserve) / kStageBytes;
+    static constexpr int kStagesTmem = (kTmemCols - kACol0) / (kKB * 32);
+    static constexpr int kStagesMin = kStagesSmem < kStagesTmem ? kStagesSmem : kStagesTmem;
+    static constexpr int kStages = kStagesMin > 16 ? 16 : kStagesMin;
     static constexpr int kSmemBytes = kStages * kStageBytes + kReserve;
     static_assert(kStages >= 3, "pipeline too shallow");
-    static_assert(kTmemCols <= 512, "TMEM over-subscribed");
-    static_assert(kXBytes % 1024 == 0, "token tile must keep the swizzle atom aligned");
+    static_assert(kACol0 + kStages * kKB * 32 <= kTmemCols, "TMEM over-subscribed");
+    static_assert(kSmemBytes > 232448 / 2, "two CTAs per SM would contend for TMEM");
+    static_assert(kXTile % 1024 == 0, "token tile must keep the swizzle atom aligned");
 };
 
 struct GemmParams {
@@ -81,24 +90,77 @@ struct GemmParams {
     const int32_t *rowsum;
     void *out;
     int32_t *status;
-    int32_t *counters;
-    int32_t *partials;
+    int32_t *flags;         // [grid]: contributor c has stored its partial tile
+    int32_t *partials;      // [grid][TOK][128]: contributor c's partial sums
     int M, N, K, group;
     int NT, KT, MT;
     int grid;
-    long long total_blocks;
+    uint32_t total_blocks;  // MT * NT * KT (k-tile blocks)
     long long off_codes, off_scale, off_zero;
     int fp16_out;
 };
 
 struct SharedCtl {
-    uint64_t full[16], empty[16];
-    uint64_t a_full[4], a_empty[4];
+    uint64_t full[16], freed[16], a_full[16];
     uint64_t acc_full[2], acc_empty[2];
     uint64_t final_bar;
     uint32_t tmem_base;
     int abort_flag;
-    int last_flag;
+};
+
+// First k-tile block of CTA c (the stream-K split), and the CTA holding block b.
+__device__ __forceinline__ uint32_t cta_begin(uint32_t c, uint32_t B, uint32_t G) {
+    return (uint32_t)(((unsigned long long)c * B) / G);
+}
+__device__ __forceinline__ uint32_t cta_of(uint32_t b, uint32_t B, uint32_t G) {
+    return (uint32_t)((((unsigned long long)b + 1) * G + B - 1) / B) - 1;
+}
+
+// Walks this CTA's k-tile blocks as pipeline units: up to KB consecutive
+// k-tiles of one tile, never crossing a tile boundary. No division per step.
+template <int KB>
+struct UnitCursor {
+    uint32_t b, b1, seg_end;
+    int KT, NT;
+    int kt, nk, nt, mt;
+    __device__ __forceinline__ void init(uint32_t b0, uint32_t b1_, int KT_, int NT_) {
+        b = b0;
+        b1 = b1_;
+        KT = KT_;
+        NT = NT_;
+        const uint32_t t = b0 / (uint32_t)KT;
+        kt = (int)(b0 - t * (uint32_t)KT);
+        mt = (int)(t / (uint32_t)NT);
+        nt = (int)(t - (uint32_t)mt * (uint32_t)NT);
+        set_segment();
+    }
+    __device__ __forceinline__ void set_segment() {
+        const uint32_t tile_end = b - (uint32_t)kt + (uint32_t)KT;
+        seg_end = tile_end < b1 ? tile_end : b1;
+        set_nk();
+    }
+    __device__ __forceinline__ void set_nk() {
+        const uint32_t left = seg_end - b;
+        nk = left < (uint32_t)KB ? (int)left : KB;
+    }
+    __device__ __forceinline__ bool done() const { return b >= b1; }
+    // Advance one unit; returns true when the current segment (tile) ends.
+    __device__ __forceinline__ bool advance() {
+        b += (uint32_t)nk;
+        kt += nk;
+        if (b < seg_end) {
+            set_nk();
+            return false;
+        }
+        if (b >= b1) return true;
+        kt = 0;
+        if (++nt == NT) {
+            nt = 0;
+            ++mt;
+        }
+        set_segment();
+        return true;
+    }
 };
 
 // Epilogue for CH consecutive tokens (m_first ..) of weight row n.
@@ -139,9 +201,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     qoq_gemm_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ CUtensorMap tmap_x) {
     using C = GemmCfg<TOK, MODE>;
     constexpr int CH = TOK < 32 ? TOK : 32;
+    constexpr int S = C::kStages;
+    constexpr int KB = C::kKB;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    SharedCtl *ctl = reinterpret_cast<SharedCtl *>(smem + C::kStages * C::kStageBytes);
+    SharedCtl *ctl = reinterpret_cast<SharedCtl *>(smem + S * C::kStageBytes);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const Watchdog wd{&ctl->abort_flag, p.status};
@@ -149,14 +213,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ set-up
     if (threadIdx.x == 0) {
         ctl->abort_flag = 0;
-        ctl->last_flag = 0;
-        for (int s = 0; s < C::kStages; ++s) {
+        for (int s = 0; s < S; ++s) {
             mbar_init(&ctl->full[s], 1);
-            mbar_init(&ctl->empty[s], 1);
-        }
-        for (int a = 0; a < C::kAStages; ++a) {
-            mbar_init(&ctl->a_full[a], 4);
-            mbar_init(&ctl->a_empty[a], 1);
+            mbar_init(&ctl->freed[s], 1);
+            mbar_init(&ctl->a_full[s], 4);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&ctl->acc_full[b], 1);
@@ -164,9 +224,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_init(&ctl->final_bar, 1);
         mbar_fence_init();
-        const uint32_t *h = reinterpret_cast<const uint32_t *>(p.blob);
-        if (h[0] != kMagic || h[1] != kVersion || h[2] != (uint32_t)p.N || h[3] != (uint32_t)p.K ||
-            h[4] != (uint32_t)p.group)
+        const int32_t *h = reinterpret_cast<const int32_t *>(p.blob);
+        if ((uint32_t)ld_cg_s32(h) != kMagic || (uint32_t)ld_cg_s32(h + 1) != kVersion ||
+            ld_cg_s32(h + 2) != p.N || ld_cg_s32(h + 3) != p.K || ld_cg_s32(h + 4) != p.group)
             wd.fail(QOQ_ERR_BAD_BLOB);
     }
     if (warp == kWarpProducer && lane == 0) prefetch_tensormap(&tmap_x);
@@ -178,135 +238,167 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = ctl->tmem_base;
+    const bool bad_blob = wd.aborted();
 
-    // Stream-K share of this CTA: blocks [b0, b1) of the (tile, k-tile) order.
-    const long long B = p.total_blocks;
-    const long long b0 = (long long)blockIdx.x * B / p.grid;
-    const long long b1 = (long long)(blockIdx.x + 1) * B / p.grid;
-    const int nblk = (int)(b1 - b0);
+    // Stream-K share of this CTA: k-tile blocks [b0, b1) in (token tile,
+    // n-tile, k-tile) order, k-tile fastest.
+    const uint32_t B = p.total_blocks, G = (uint32_t)p.grid;
+    const uint32_t b0 = cta_begin(blockIdx.x, B, G);
+    const uint32_t b1 = cta_begin(blockIdx.x + 1, B, G);
     const int KT = p.KT;
 
     auto stage_x = [&](int s) { return smem + s * C::kStageBytes; };
     auto stage_w = [&](int s) { return smem + s * C::kStageBytes + C::kXBytes; };
 
-    if (!wd.aborted()) {
+    if (!bad_blob) {
         if (warp == kWarpProducer) {
             // ------------------------------------------------ TMA producer
-            if (lane == 0) {
-                const uint64_t pol_w = policy_evict_first();   // weights: streamed once
-                const uint64_t pol_x = policy_evict_last();    // activations: reused by every n-tile
-                int issued = 0;
-                for (int i = 0; i < nblk; ++i) {
-                    const long long b = b0 + i;
-                    const long long t = b / KT;
-                    const int kt = (int)(b - t * KT);
-                    const int mt = (int)(t / p.NT);
-                    const int nt = (int)(t - (long long)mt * p.NT);
-                    const int s = i % C::kStages;
-                    const uint32_t ph = (uint32_t)(i / C::kStages) & 1u;
-                    if (!wait_bounded(&ctl->empty[s], ph ^ 1u, wd)) break;
-                    mbar_arrive_expect_tx(&ctl->full[s], C::kXBytes + C::kWBytes);
-                    const uint8_t *wsrc = p.blob + p.off_codes + ((long long)nt * KT + kt) * C::kWBytes;
-                    bulk_load(stage_w(s), wsrc, C::kWBytes, &ctl->full[s], pol_w);
-                    tma_load_2d(stage_x(s), &tmap_x, &ctl->full[s], kt * kTileK, mt * TOK, pol_x);
-                    issued = i + 1;
+            const uint64_t pol_w = policy_evict_first();   // weights: streamed once
+            const uint64_t pol_x = policy_evict_last();    // activations: reused by every n-tile
+            UnitCursor<KB> cur;
+            cur.init(b0, b1, KT, p.NT);
+            auto issue_w = [&](int s, const UnitCursor<KB> &c) {
+                mbar_arrive_expect_tx(&ctl->full[s], (uint32_t)(c.nk * (C::kWTile + C::kXTile)));
+                const uint8_t *wsrc = p.blob + p.off_codes + ((long long)c.nt * KT + c.kt) * C::kWTile;
+                bulk_load(stage_w(s), wsrc, (uint32_t)(c.nk * C::kWTile), &ctl->full[s], pol_w);
+            };
+            auto issue_x = [&](int s, const UnitCursor<KB> &c) {
+                for (int j = 0; j < c.nk; ++j)
+                    tma_load_2d(stage_x(s) + j * C::kXTile, &tmap_x, &ctl->full[s], (c.kt + j) * kTileK,
+                                c.mt * TOK, pol_x);
+            };
+            int issued = 0;
+            int s = 0;
+            uint32_t ph = 0;
+            for (int i = 0; !cur.done(); ++i) {
+                const bool ok = __all_sync(0xffffffffu, wait_bounded(&ctl->freed[s], ph ^ 1u, wd));
+                if (!ok) break;
+                if (lane == 0) {
+                    issue_w(s, cur);
+                    issue_x(s, cur);
                 }
-                // Let every copy that was issued land before the CTA can exit.
-                for (int i = issued > C::kStages ? issued - C::kStages : 0; i < issued; ++i)
-                    wait_drain(&ctl->full[i % C::kStages], (uint32_t)(i / C::kStages) & 1u, kDrainNs);
+                __syncwarp();
+                issued = i + 1;
+                cur.advance();
+                if (++s == S) {
+                    s = 0;
+                    ph ^= 1u;
+                }
             }
+            // Let every copy that was issued land before the CTA can exit.
+            if (lane == 0)
+                for (int i = issued > S ? issued - S : 0; i < issued; ++i)
+                    wait_drain(&ctl->full[i % S], (uint32_t)(i / S) & 1u, kDrainNs);
+            __syncwarp();
         } else if (warp == kWarpMma) {
             // ------------------------------------------------ MMA issuer
-            if (lane == 0) {
-                constexpr uint32_t idesc = idesc_i8(128, TOK, true, true);
-                int i = 0, seg = 0;
-                bool ok = true;
-                long long b = b0;
-                while (ok && b < b1) {
-                    const long long t = b / KT;
-                    const long long e = lmin(b1, (t + 1) * KT);
-                    const int buf = seg % C::kAccBufs;
-                    const uint32_t aph = (uint32_t)(seg / C::kAccBufs) & 1u;
-                    if (!wait_bounded(&ctl->acc_empty[buf], aph ^ 1u, wd)) break;
-                    tc_fence_after();
-                    const uint32_t d_tmem = tmem_base + (uint32_t)(buf * TOK);
-                    for (long long bb = b; bb < e; ++bb, ++i) {
-                        const int s = i % C::kStages;
-                        const uint32_t ph = (uint32_t)(i / C::kStages) & 1u;
-                        const int a = i % C::kAStages;
-                        const uint32_t ap = (uint32_t)(i / C::kAStages) & 1u;
-                        if (!wait_bounded(&ctl->full[s], ph, wd) || !wait_bounded(&ctl->a_full[a], ap, wd)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        const uint64_t bdesc = smem_desc_k_sw128(smem_u32(stage_x(s)));
-                        const uint32_t a_tmem = tmem_base + (uint32_t)(C::kACol0 + a * 32);
-#pragma unroll
-                        for (int j = 0; j < 4; ++j)   // 4 x K=32 per 128-wide k-tile
-                            mma_i8_ts(d_tmem, a_tmem + (uint32_t)(j * 8), bdesc + (uint64_t)(j * 2), idesc,
-                                      (bb > b || j > 0) ? 1u : 0u);
-                        tc_commit(&ctl->empty[s]);
-                        tc_commit(&ctl->a_empty[a]);
-                    }
+            constexpr uint32_t idesc = idesc_i8(128, TOK, true, true);
+            UnitCursor<KB> cur;
+            cur.init(b0, b1, KT, p.NT);
+            int s = 0, seg = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            while (ok && !cur.done()) {
+                const int buf = seg % C::kAccBufs;
+                const uint32_t aph = (uint32_t)(seg / C::kAccBufs) & 1u;
+                ok = __all_sync(0xffffffffu, wait_bounded(&ctl->acc_empty[buf], aph ^ 1u, wd));
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(buf * TOK);
+                bool first = true, seg_done = false;
+                while (!seg_done) {
+                    // The token tile (shared memory) and the dequantised weights
+                    // (TMEM) of this unit.
+                    ok = __all_sync(0xffffffffu,
+                                    wait_bounded(&ctl->full[s], ph, wd) && wait_bounded(&ctl->a_full[s], ph, wd));
                     if (!ok) break;
-                    tc_commit(&ctl->acc_full[buf]);
-                    ++seg;
-                    b = e;
+                    tc_fence_after();
+                    if (lane == 0) {
+                        const uint32_t a_tmem = tmem_base + (uint32_t)(C::kACol0 + s * KB * 32);
+                        const uint32_t xaddr = smem_u32(stage_x(s));
+                        for (int j = 0; j < cur.nk; ++j) {
+                            const uint64_t bdesc = smem_desc_k_sw128(xaddr + j * C::kXTile);
+#pragma unroll
+                            for (int q = 0; q < 4; ++q)   // 4 x K=32 per 128-wide k-tile
+                                mma_i8_ts(d_tmem, a_tmem + (uint32_t)(j * 32 + q * 8), bdesc + (uint64_t)(q * 2),
+                                          idesc, (first && j == 0 && q == 0) ? 0u : 1u);
+                        }
+                        tc_commit(&ctl->freed[s]);
+                    }
+                    __syncwarp();
+                    first = false;
+                    if (++s == S) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                    seg_done = cur.advance();
                 }
-                // Every MMA must have completed before tensor memory is freed.
+                if (!ok) break;
+                if (lane == 0) tc_commit(&ctl->acc_full[buf]);
+                __syncwarp();
+                ++seg;
+            }
+            // Every MMA must have completed before tensor memory is freed.
+            if (lane == 0) {
                 tc_commit(&ctl->final_bar);
                 wait_drain(&ctl->final_bar, 0, kDrainNs);
             }
             __syncwarp();
         } else if (warp >= kWarpDequant0 && warp < kWarpEpilogue) {
             // ------------------------------------------------ dequant
-            const int g = (warp - kWarpDequant0) >> 2;     // warpgroup 0 / 1
+            const int g = (warp - kWarpDequant0) >> 2;     // warpgroup 0 / 1: even / odd units
             const int quarter = warp & 3;                    // TMEM lanes 32q .. 32q+31
             const int r = quarter * 32 + lane;               // weight row in the tile
             const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-            for (int i = g; i < nblk; i += 2) {
-                const int s = i % C::kStages;
-                const uint32_t ph = (uint32_t)(i / C::kStages) & 1u;
-                const int a = i % C::kAStages;
-                const uint32_t ap = (uint32_t)(i / C::kAStages) & 1u;
-                bool ok = wait_bounded(&ctl->full[s], ph, wd) && wait_bounded(&ctl->a_empty[a], ap ^ 1u, wd);
-                if (!__all_sync(0xffffffffu, ok)) break;
-                const uint32_t wbase = smem_u32(stage_w(s));
-                uint32_t outw[32];
-                if (MODE == 0) {
-                    const uint32_t sz = lds16(wbase + 8192 + 2 * r);
-                    const uint32_t sc = sz & 0xFFu;
-                    const int zs = (int)(int8_t)(sz >> 8);
-                    const uint32_t c4 = (uint32_t)(128 - zs) * 0x01010101u;
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const uint4 v = lds128(wbase + c * 2048 + r * 16);
-                        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const uint32_t lo = w[j] & 0x0F0F0F0Fu;
-                            const uint32_t hi = (w[j] >> 4) & 0x0F0F0F0Fu;
-                            outw[8 * c + 2 * j] = (lo * sc + c4) ^ 0x80808080u;
-                            outw[8 * c + 2 * j + 1] = (hi * sc + c4) ^ 0x80808080u;
-                        }
-                    }
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const uint4 v = lds128(wbase + c * 2048 + r * 16);
-                        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            outw[8 * c + 2 * j] = w[j] & 0x0F0F0F0Fu;
-                            outw[8 * c + 2 * j + 1] = (w[j] >> 4) & 0x0F0F0F0Fu;
-                        }
-                    }
+            UnitCursor<KB> cur;
+            cur.init(b0, b1, KT, p.NT);
+            int s = 0;
+            uint32_t ph = 0;
+            for (int i = 0; !cur.done(); ++i, cur.advance()) {
+                const int unit_s = s;
+                const uint32_t unit_ph = ph;
+                if (++s == S) {
+                    s = 0;
+                    ph ^= 1u;
                 }
-                tmem_st32_wait(tmem_base + lane_addr + (uint32_t)(C::kACol0 + a * 32), outw);
+                if ((i & 1) != g) continue;
+                // full[s] for this unit implies the producer saw freed[s] for
+                // the unit S earlier, i.e. TMEM A buffer s is no longer read.
+                const bool ok = __all_sync(0xffffffffu, wait_bounded(&ctl->full[unit_s], unit_ph, wd));
+                if (!ok) break;
+                const uint32_t a_col = tmem_base + lane_addr + (uint32_t)(C::kACol0 + unit_s * KB * 32);
+                for (int j = 0; j < cur.nk; ++j) {
+                    const uint32_t wbase = smem_u32(stage_w(unit_s) + j * C::kWTile);
+                    uint32_t sc = 0u, c4 = 0u;
+                    if (MODE == 0) {
+                        const uint32_t sz = lds16(wbase + 8192 + 2 * r);
+                        sc = sz & 0xFFu;
+                        c4 = (uint32_t)(128 - (int)(int8_t)(sz >> 8)) * 0x01010101u;
+                    }
+                    uint32_t o[32];
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const uint4 v = lds128(wbase + c * 2048 + r * 16);
+                        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const uint32_t lo = w[q] & 0x0F0F0F0Fu;
+                            const uint32_t hi = (w[q] >> 4) & 0x0F0F0F0Fu;
+                            if (MODE == 0) {
+                                o[8 * c + 2 * q] = (lo * sc + c4) ^ 0x80808080u;
+                                o[8 * c + 2 * q + 1] = (hi * sc + c4) ^ 0x80808080u;
+                            } else {
+                                o[8 * c + 2 * q] = lo;
+                                o[8 * c + 2 * q + 1] = hi;
+                            }
+                        }
+                    }
+                    tmem_st32_wait(a_col + (uint32_t)(j * 32), o);
+                }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&ctl->a_full[a]);
+                if (lane == 0) mbar_arrive(&ctl->a_full[unit_s]);
+                __syncwarp();
             }
         } else if (warp >= kWarpEpilogue) {
             // ------------------------------------------------ epilogue
@@ -314,31 +406,63 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int r = quarter * 32 + lane;
             const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
             const bool leader = (threadIdx.x == kWarpEpilogue * 32);
+            UnitCursor<KB> cur;
+            cur.init(b0, b1, KT, p.NT);
             int seg = 0;
-            long long b = b0;
-            while (b < b1) {
-                const long long t = b / KT;
-                const long long e = lmin(b1, (t + 1) * KT);
-                const int kt_lo = (int)(b - t * KT), kt_hi = (int)(e - t * KT);
-                const int mt = (int)(t / p.NT);
-                const int nt = (int)(t - (long long)mt * p.NT);
+            while (!cur.done()) {
+                const uint32_t seg_b = cur.b, seg_e = cur.seg_end;
+                const int kt_lo = cur.kt, kt_hi = cur.kt + (int)(seg_e - seg_b);
+                const int mt = cur.mt, nt = cur.nt;
+                const uint32_t tile_b = seg_b - (uint32_t)kt_lo;
+                while (!cur.advance()) {
+                }
                 const int buf = seg % C::kAccBufs;
                 const uint32_t aph = (uint32_t)(seg / C::kAccBufs) & 1u;
-                const bool ok = wait_bounded(&ctl->acc_full[buf], aph, wd);
-                // All four epilogue warps leave together: the partial-tile path
-                // below meets at named barriers.
+                // Every lane spins on its own; the vote reconverges the warp
+                // before the named barrier, and all four epilogue warps leave
+                // together (the shared-tile paths below meet at named barriers).
+                const bool ok = __all_sync(0xffffffffu, wait_bounded(&ctl->acc_full[buf], aph, wd));
                 if (named_bar_any(1, 128, !ok)) break;
                 tc_fence_after();
                 const int n = nt * kTileN + r;
                 const int64_t m0 = (int64_t)mt * TOK;
-                float col_scale = 0.0f;
+                const float col_scale = __half2float(reinterpret_cast<const __half *>(p.blob + p.off_scale)[n]);
                 int col_zero = 0;
-                col_scale = __half2float(reinterpret_cast<const __half *>(p.blob + p.off_scale)[n]);
                 if (MODE == 1)
                     col_zero = __half2int_rn(reinterpret_cast<const __half *>(p.blob + p.off_zero)[n]);
                 const uint32_t acc_addr = tmem_base + lane_addr + (uint32_t)(buf * TOK);
-                if (kt_lo == 0 && kt_hi == KT) {
-                    // Whole tile computed here: straight from TMEM.
+                if (kt_lo > 0) {
+                    // Contributor: this tile's first k-tile belongs to an earlier
+                    // CTA. Store the partial sums in this CTA's slot, raise its flag.
+                    int32_t *part = p.partials + (long long)blockIdx.x * TOK * kTileN;
+#pragma unroll 1
+                    for (int c0 = 0; c0 < TOK; c0 += CH) {
+                        uint32_t v[CH];
+                        tmem_load<CH>(acc_addr + (uint32_t)c0, v);
+#pragma unroll
+                        for (int j = 0; j < CH; ++j) part[(c0 + j) * kTileN + r] = (int32_t)v[j];
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&ctl->acc_empty[buf]);
+                    __threadfence();
+                    named_bar_sync(1, 128);
+                    if (leader) st_release_gpu(p.flags + blockIdx.x, 1);
+                    __syncwarp();
+                } else {
+                    // Owner (or sole computer) of the tile: add the contributors'
+                    // partial sums, run the epilogue, clear their flags.
+                    const uint32_t c_first = blockIdx.x + 1;
+                    const uint32_t c_last = (kt_hi == KT) ? blockIdx.x : cta_of(tile_b + (uint32_t)KT - 1, B, G);
+                    if (c_last >= c_first) {
+                        bool got = true;
+                        if (leader)
+                            for (uint32_t c = c_first; c <= c_last && got; ++c)
+                                got = wait_flag_bounded(p.flags + c, wd);
+                        __syncwarp();
+                        if (named_bar_any(1, 128, !got)) break;
+                        __threadfence();
+                    }
 #pragma unroll 1
                     for (int c0 = 0; c0 < TOK; c0 += CH) {
                         uint32_t v[CH];
@@ -348,54 +472,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                             __syncwarp();
                             if (lane == 0) mbar_arrive(&ctl->acc_empty[buf]);
                         }
+                        for (uint32_t c = c_first; c <= c_last; ++c) {
+                            const int32_t *part = p.partials + (long long)c * TOK * kTileN;
+#pragma unroll
+                            for (int j = 0; j < CH; ++j)
+                                v[j] = (uint32_t)((int32_t)v[j] + ld_cg_s32(part + (c0 + j) * kTileN + r));
+                        }
                         store_outputs<CH, MODE>(p, v, m0 + c0, n, col_scale, col_zero);
                     }
-                } else {
-                    // Tile shared with other CTAs: add into its slot, count the
-                    // k-tiles that have arrived; the last contributor finishes.
-                    const long long slot =
-                        ((t * KT + 1) * (long long)p.grid + B - 1) / B - 1;   // first CTA boundary inside t
-                    int32_t *part = p.partials + slot * (long long)TOK * kTileN;
-#pragma unroll 1
-                    for (int c0 = 0; c0 < TOK; c0 += CH) {
-                        uint32_t v[CH];
-                        tmem_load<CH>(acc_addr + (uint32_t)c0, v);
-#pragma unroll
-                        for (int j = 0; j < CH; ++j) red_add_s32(part + (c0 + j) * kTileN + r, (int32_t)v[j]);
-                    }
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&ctl->acc_empty[buf]);
-                    __threadfence();
-                    named_bar_sync(1, 128);
-                    if (leader) {
-                        const int old = atomicAdd(p.counters + slot, kt_hi - kt_lo);
-                        ctl->last_flag = (old + (kt_hi - kt_lo) == KT) ? 1 : 0;
-                    }
-                    named_bar_sync(1, 128);
-                    if (ctl->last_flag) {
-                        __threadfence();
-#pragma unroll 1
-                        for (int c0 = 0; c0 < TOK; c0 += CH) {
-                            uint32_t v[CH];
-#pragma unroll
-                            for (int j = 0; j < CH; ++j) {
-                                int32_t *q = part + (c0 + j) * kTileN + r;
-                                v[j] = (uint32_t)ld_cg_s32(q);
-                                *q = 0;
-                            }
-                            store_outputs<CH, MODE>(p, v, m0 + c0, n, col_scale, col_zero);
-                        }
-                        if (leader) p.counters[slot] = 0;
+                    if (c_last >= c_first) {
+                        named_bar_sync(1, 128);
+                        if (leader)
+                            for (uint32_t c = c_first; c <= c_last; ++c) p.flags[c] = 0;
+                        __syncwarp();
                     }
                 }
                 ++seg;
-                b = e;
             }
         }
     }
 
     // ------------------------------------------------------------ teardown
+    __syncwarp();
     tc_fence_before();
     __syncthreads();
     if (warp == kWarpMma) {
@@ -420,48 +518,47 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
     return fn;
 }
 
-struct DeviceInfo {
-    int sm_count = 0;
-};
-
-static DeviceInfo device_info(int dev) {
-    static DeviceInfo info[64];
+static int sm_count_of(int dev) {
+    static int count[64];
     static std::mutex mu;
+    if (dev < 0 || dev >= 64) return 0;
     std::lock_guard<std::mutex> lock(mu);
-    if (dev < 0 || dev >= 64) return DeviceInfo{};
-    if (info[dev].sm_count == 0) cudaDeviceGetAttribute(&info[dev].sm_count, cudaDevAttrMultiProcessorCount, dev);
-    return info[dev];
+    if (count[dev] == 0) cudaDeviceGetAttribute(&count[dev], cudaDevAttrMultiProcessorCount, dev);
+    return count[dev];
+}
+
+// X8 [M][K] int8, boxes of 128 k x TOK tokens, 128-byte swizzle.
+static bool encode_x_map(CUtensorMap *map, const int8_t *X8, int64_t M, int64_t K, int tok) {
+    auto encode = get_encode_fn();
+    if (!encode) return false;
+    const cuuint64_t gdim[2] = {(cuuint64_t)K, (cuuint64_t)M};
+    const cuuint64_t gstride[1] = {(cuuint64_t)K};
+    const cuuint32_t box[2] = {(cuuint32_t)kTileK, (cuuint32_t)tok};
+    const cuuint32_t estride[2] = {1, 1};
+    return encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t *>(X8), gdim, gstride, box, estride,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int TOK, int MODE>
 static qoq_status launch_gemm_t(const GemmArgs &a, cudaStream_t stream) {
     using C = GemmCfg<TOK, MODE>;
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return QOQ_ERR_CUDA;
-    const DeviceInfo info = device_info(dev);
-    if (info.sm_count <= 0) return QOQ_ERR_CUDA;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return QOQ_ERR_CUDA;
+    const int sms = sm_count_of(dev);
+    if (sms <= 0) return QOQ_ERR_CUDA;
 
     // Opt in to the large dynamic shared memory once per device.
     static std::once_flag attr_once[64];
     static cudaError_t attr_err[64];
-    if (dev >= 64) return QOQ_ERR_CUDA;
     std::call_once(attr_once[dev], [&] {
         attr_err[dev] = cudaFuncSetAttribute(qoq_gemm_kernel<TOK, MODE>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     });
     if (attr_err[dev] != cudaSuccess) return QOQ_ERR_CUDA;
 
-    auto encode = get_encode_fn();
-    if (!encode) return QOQ_ERR_CUDA;
     CUtensorMap tmap;
-    const cuuint64_t gdim[2] = {(cuuint64_t)a.K, (cuuint64_t)a.M};
-    const cuuint64_t gstride[1] = {(cuuint64_t)a.K};
-    const cuuint32_t box[2] = {(cuuint32_t)kTileK, (cuuint32_t)TOK};
-    const cuuint32_t estride[2] = {1, 1};
-    CUresult cr = encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t *>(a.X8), gdim, gstride, box,
-                         estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (cr != CUDA_SUCCESS) return QOQ_ERR_CUDA;
+    if (!encode_x_map(&tmap, a.X8, a.M, a.K, TOK)) return QOQ_ERR_CUDA;
 
     const BlobLayout L = blob_layout(a.N, a.K, a.group);
     GemmParams p;
@@ -471,7 +568,7 @@ static qoq_status launch_gemm_t(const GemmArgs &a, cudaStream_t stream) {
     p.out = a.out;
     uint8_t *ws = static_cast<uint8_t *>(a.ws);
     p.status = reinterpret_cast<int32_t *>(ws);
-    p.counters = reinterpret_cast<int32_t *>(ws + 256);
+    p.flags = reinterpret_cast<int32_t *>(ws + 256);
     p.partials = reinterpret_cast<int32_t *>(ws + 256 + sizeof(int32_t) * kMaxGrid);
     p.M = (int)a.M;
     p.N = (int)a.N;
@@ -480,15 +577,22 @@ static qoq_status launch_gemm_t(const GemmArgs &a, cudaStream_t stream) {
     p.NT = (int)(a.N / kTileN);
     p.KT = (int)(a.K / kTileK);
     p.MT = (int)((a.M + TOK - 1) / TOK);
-    p.total_blocks = (long long)p.MT * p.NT * p.KT;
-    p.grid = (int)std::min<long long>(std::min(info.sm_count, kMaxGrid), p.total_blocks);
+    const long long blocks = (long long)p.MT * p.NT * p.KT;
+    if (blocks >= (1ll << 31)) return QOQ_ERR_UNSUPPORTED;
+    p.total_blocks = (uint32_t)blocks;
+    p.grid = (int)std::min<long long>(std::min(sms, kMaxGrid), blocks);
     p.off_codes = L.off_codes;
     p.off_scale = L.off_scale;
     p.off_zero = L.off_zero;
     p.fp16_out = a.fp16_out ? 1 : 0;
 
-    qoq_gemm_kernel<TOK, MODE><<<p.grid, kThreads, C::kSmemBytes, stream>>>(p, tmap);
-    return cudaGetLastError() == cudaSuccess ? QOQ_OK : QOQ_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)p.grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = stream;
+    cfg.numAttrs = 0;
+    return cudaLaunchKernelEx(&cfg, qoq_gemm_kernel<TOK, MODE>, p, tmap) == cudaSuccess ? QOQ_OK : QOQ_ERR_CUDA;
 }
 
 template <int MODE>

@@ -220,9 +220,32 @@ __device__ __forceinline__ void tmem_st32_wait(uint32_t taddr, const uint32_t (&
         : "memory");
 }
 
+// 32 lanes x 8 columns store; the source registers are read at issue. A later
+// tmem_st_wait() makes all prior stores of this thread visible to the MMA.
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3,
+                                         uint32_t r4, uint32_t r5, uint32_t r6, uint32_t r7) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+                 "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(r4), "r"(r5), "r"(r6), "r"(r7)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// One lane of the (fully active) warp gets true.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b32 r;\n\t"
+        "elect.sync r|p, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
+}
+
 // Load + wait in one asm block so no use of the destination registers can be
 // scheduled before the data has arrived.
 __device__ __forceinline__ void tmem_ld32_wait(uint32_t taddr, uint32_t (&r)[32]) {
+    __syncwarp();   // warp-collective (.sync.aligned)
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
         "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
@@ -237,6 +260,7 @@ __device__ __forceinline__ void tmem_ld32_wait(uint32_t taddr, uint32_t (&r)[32]
 }
 
 __device__ __forceinline__ void tmem_ld16_wait(uint32_t taddr, uint32_t (&r)[16]) {
+    __syncwarp();   // warp-collective (.sync.aligned)
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
         "%14, %15}, [%16];\n\t"
@@ -248,15 +272,58 @@ __device__ __forceinline__ void tmem_ld16_wait(uint32_t taddr, uint32_t (&r)[16]
         : "memory");
 }
 
+// ------------------------------------------- programmatic dependent launch
+
+// Block until the grids this one depends on have completed and their memory
+// is visible (returns at once when launched without a programmatic edge).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Allow the next grid in the stream to start launching.
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ------------------------------------------------- cross-CTA flags (gpu scope)
+
+__device__ __forceinline__ void st_release_gpu(int32_t *p, int32_t v) {
+    asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ int32_t ld_acquire_gpu(const int32_t *p) {
+    int32_t v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Spin until *flag != 0, bounded like the pipeline waits.
+__device__ __forceinline__ bool wait_flag_bounded(const int32_t *flag, const Watchdog &wd,
+                                                  uint64_t limit_ns = kWaitLimitNs) {
+    if (ld_acquire_gpu(flag) != 0) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        __nanosleep(64);
+        if (ld_acquire_gpu(flag) != 0) return true;
+        if ((it & 15u) == 0) {
+            if (wd.aborted()) return false;
+            if (globaltimer_ns() - t0 > limit_ns) {
+                wd.fail(QOQ_ERR_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+
 // -------------------------------------------------------------- misc device
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+    __syncwarp();   // bar.sync is the .aligned form: the warp must arrive converged
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // Named barrier over `nthreads` threads that also returns whether `pred` was
 // true in any of them (every participating thread gets the same answer).
 __device__ __forceinline__ bool named_bar_any(int id, int nthreads, bool pred) {
+    __syncwarp();   // bar.red is the .aligned form: the warp must arrive converged
     uint32_t r;
     asm volatile(
         "{\n\t.reg .pred p, q;\n\t"

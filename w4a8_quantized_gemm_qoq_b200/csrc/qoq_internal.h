@@ -53,8 +53,11 @@ inline int token_tile_for(int64_t M) {
     return 256;
 }
 
-// Workspace: [0, 256) status word + reserved; then int32 counters [kMaxGrid];
-// then int32 partial tiles [kMaxGrid][tok][128].
+// Workspace: [0, 256) status word + reserved; then int32 flags [kMaxGrid]
+// (together QOQ_WORKSPACE_CONTROL_BYTES, left zero by every call); then int32
+// partial tiles [kMaxGrid][tok][128] (scratch).
+static_assert(256 + 4 * kMaxGrid == QOQ_WORKSPACE_CONTROL_BYTES, "workspace control layout");
+
 inline size_t workspace_bytes_for(int64_t M) {
     const int tok = token_tile_for(M);
     return 256 + sizeof(int32_t) * kMaxGrid + sizeof(int32_t) * (size_t)kMaxGrid * tok * kTileN;

@@ -41,7 +41,10 @@ __device__ __forceinline__ int quant_code(float x, float s, int lim) {
 }
 
 // One CTA per token row: absmax (warp shuffles, then across warps), FP16
-// scale, then round-half-even codes and their row sum.
+// scale, then round-half-even codes and their row sum. NCH > 0 keeps the row
+// in registers (NCH 16-byte chunks per thread, one pass over HBM); NCH == 0
+// reads the row twice (any K).
+template <int NCH>
 __global__ void __launch_bounds__(kActThreads) act_quant_kernel(const __half *__restrict__ X, int K,
                                                                  int8_t *__restrict__ X8,
                                                                  __half *__restrict__ s_x,
@@ -49,19 +52,37 @@ __global__ void __launch_bounds__(kActThreads) act_quant_kernel(const __half *__
     __shared__ float red_f[kActThreads / 32];
     __shared__ int red_i[kActThreads / 32];
     __shared__ float s_shared;
+    // X may come from the previous kernel in the stream; release the next one
+    // (the GEMM) so its set-up and weight copies overlap this kernel.
+    griddep_wait();
+    griddep_launch_dependents();
     const int64_t m = blockIdx.x;
     const __half *row = X + m * K;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr int NR = NCH > 0 ? NCH : 1;
 
+    uint4 v[NR];
     float amax = 0.0f;
-    for (int k = threadIdx.x * 8; k < K; k += kActThreads * 8) {
-        uint4 v = *reinterpret_cast<const uint4 *>(row + k);
-        const __half2 *h = reinterpret_cast<const __half2 *>(&v);
+    auto absmax8 = [&](const uint4 &u) {
+        const __half2 *h = reinterpret_cast<const __half2 *>(&u);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             float2 f = __half22float2(h[i]);
             amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
         }
+    };
+    if (NCH > 0) {
+#pragma unroll
+        for (int i = 0; i < NR; ++i) {
+            const int k = (i * kActThreads + threadIdx.x) * 8;
+            // The load address is clamped into the row, so no form of the
+            // guard can read past the end of X; out-of-row chunks become 0.
+            const uint4 u = *reinterpret_cast<const uint4 *>(row + (k < K ? k : K - 8));
+            v[i] = k < K ? u : make_uint4(0u, 0u, 0u, 0u);
+            absmax8(v[i]);
+        }
+    } else {
+        for (int k = threadIdx.x * 8; k < K; k += kActThreads * 8) absmax8(*reinterpret_cast<const uint4 *>(row + k));
     }
     amax = warp_max(amax);
     if (lane == 0) red_f[warp] = amax;
@@ -78,9 +99,8 @@ __global__ void __launch_bounds__(kActThreads) act_quant_kernel(const __half *__
 
     int sum = 0;
     int8_t *out = X8 + m * K;
-    for (int k = threadIdx.x * 8; k < K; k += kActThreads * 8) {
-        uint4 v = *reinterpret_cast<const uint4 *>(row + k);
-        const __half2 *h = reinterpret_cast<const __half2 *>(&v);
+    auto quant8 = [&](const uint4 &u, int k) {
+        const __half2 *h = reinterpret_cast<const __half2 *>(&u);
         uint32_t packed[2] = {0u, 0u};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -90,6 +110,15 @@ __global__ void __launch_bounds__(kActThreads) act_quant_kernel(const __half *__
             packed[i >> 1] |= ((uint32_t)(q0 & 0xFF) << (16 * (i & 1))) | ((uint32_t)(q1 & 0xFF) << (16 * (i & 1) + 8));
         }
         *reinterpret_cast<uint2 *>(out + k) = make_uint2(packed[0], packed[1]);
+    };
+    if (NCH > 0) {
+#pragma unroll
+        for (int i = 0; i < NR; ++i) {
+            const int k = (i * kActThreads + threadIdx.x) * 8;
+            if (k < K) quant8(v[i], k);
+        }
+    } else {
+        for (int k = threadIdx.x * 8; k < K; k += kActThreads * 8) quant8(*reinterpret_cast<const uint4 *>(row + k), k);
     }
     if (rowsum != nullptr) {
         sum = warp_sum(sum);
@@ -103,11 +132,32 @@ __global__ void __launch_bounds__(kActThreads) act_quant_kernel(const __half *__
     }
 }
 
+template <int NCH>
+static cudaError_t launch_act_quant_t(const void *X, int64_t M, int64_t K, int8_t *X8, void *s_x,
+                                      int32_t *rowsum, cudaStream_t stream) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)M);
+    cfg.blockDim = dim3(kActThreads);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, act_quant_kernel<NCH>, static_cast<const __half *>(X), (int)K, X8,
+                              static_cast<__half *>(s_x), rowsum);
+}
+
 cudaError_t launch_act_quant(const void *X, int64_t M, int64_t K, int8_t *X8, void *s_x, int32_t *rowsum,
                              cudaStream_t stream) {
-    act_quant_kernel<<<(unsigned)M, kActThreads, 0, stream>>>(static_cast<const __half *>(X), (int)K, X8,
-                                                              static_cast<__half *>(s_x), rowsum);
-    return cudaGetLastError();
+    const int64_t per_pass = (int64_t)kActThreads * 8;   // halves one pass of the CTA covers
+    const int64_t nch = (K + per_pass - 1) / per_pass;
+    if (nch <= 1) return launch_act_quant_t<1>(X, M, K, X8, s_x, rowsum, stream);
+    if (nch <= 2) return launch_act_quant_t<2>(X, M, K, X8, s_x, rowsum, stream);
+    if (nch <= 4) return launch_act_quant_t<4>(X, M, K, X8, s_x, rowsum, stream);
+    if (nch <= 8) return launch_act_quant_t<8>(X, M, K, X8, s_x, rowsum, stream);
+    if (nch <= 12) return launch_act_quant_t<12>(X, M, K, X8, s_x, rowsum, stream);
+    return launch_act_quant_t<0>(X, M, K, X8, s_x, rowsum, stream);
 }
 
 // ---------------------------------------------------------------- weights

@@ -18,6 +18,7 @@ STATUS = {0: "QOQ_OK", 1: "QOQ_ERR_INVALID_ARG", 2: "QOQ_ERR_UNSUPPORTED", 3: "Q
           4: "QOQ_ERR_WORKSPACE", 5: "QOQ_ERR_BAD_BLOB", 6: "QOQ_ERR_CUDA", 7: "QOQ_ERR_TIMEOUT"}
 TILE = 128
 GROUP = 128
+WORKSPACE_CONTROL_BYTES = 1280   # status word + cross-CTA flags (include/qoq.h)
 
 _lib = None
 
@@ -119,8 +120,9 @@ def quantize_weights(W, group_size: int = GROUP, blob=None, stream=None):
 
 
 class Workspace:
-    """Zero-filled device workspace for the GEMM calls (the library leaves it
-    zero-filled after each call; its first int32 is the device status word)."""
+    """Zero-filled device workspace for the GEMM calls. Its leading control
+    bytes (the device status word, then cross-CTA flags) are left zero by
+    every call that completes; the rest is scratch."""
 
     def __init__(self, nbytes: int, device="cuda"):
         import torch
@@ -132,6 +134,9 @@ class Workspace:
 
     def status(self) -> int:
         return int(self.buf[:4].view(dtype=__import__("torch").int32).item())
+
+    def control_clear(self) -> bool:
+        return not bool(self.buf[:WORKSPACE_CONTROL_BYTES].any().item())
 
     def reset(self):
         self.buf.zero_()
