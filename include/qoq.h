@@ -149,6 +149,37 @@ qoq_status qoq_gemm_fp16_out(const int8_t *X8, const void *s_x_fp16, const int32
                              void *Y_fp16, void *workspace, size_t *workspace_bytes,
                              void *stream);
 
+/*
+ * W4A8 GEMM with the fused FP16 epilogue, for callers that cannot allocate
+ * device memory (a pre-planned memory arena, a thread that must not touch the
+ * device allocator while other work owns it, a runtime that forbids cudaMalloc
+ * after start-up). The QServe pages have no counterpart: it exists only so the
+ * workspace of qoq_gemm_fp16_out need not be allocated by the caller.
+ *
+ * Same computation and arguments as qoq_gemm_fp16_out, except that the
+ * stream-K scratch lives in one fixed 8 MiB device array inside the library,
+ * which every GPU that loads the library keeps until the process exits. That
+ * bounds the problem: it needs 1280 + (SM count) * T * 512 bytes, T being the
+ * token tile (16, 32, 64, ... for M <= 16, 32, 64, ...), so M <= 64 on a
+ * 148-SM B200; larger problems return QOQ_ERR_WORKSPACE and launch nothing.
+ *
+ * status: optional device int32; when non-NULL the call copies the device
+ * status word of this call (0, QOQ_ERR_BAD_BLOB or QOQ_ERR_TIMEOUT) into it
+ * on the same stream.
+ *
+ * The library neither allocates nor frees anything in this call: it clears the
+ * array's control words (cudaMemsetAsync), launches the GEMM and, if asked,
+ * copies the status word. The first call on each device looks up the array's
+ * device address (cudaGetSymbolAddress) with that device current, so make the
+ * first call on a device before any stream capture. All calls share the one
+ * array, which keeps the last call's contents: calls that may overlap on the
+ * device (different streams, or different host threads) race on it and must
+ * be serialised by the caller.
+ */
+qoq_status qoq_gemm_fp16_out_static_ws(const int8_t *X8, const void *s_x_fp16, const int32_t *rowsum,
+                                       const void *blob, int64_t M, int64_t N, int64_t K, int group_size,
+                                       void *Y_fp16, int32_t *status, void *stream);
+
 /* Name of a status code (static string, never NULL). */
 const char *qoq_status_string(qoq_status status);
 
