@@ -228,6 +228,8 @@ def run_gpu(args, rank, world, local_rank):
         for p in probs:                      # eager warm-up: library load, attributes, first launch
             p.run(qoq)
     stream.synchronize()
+    bad = [(p.K, p.N, p.M, p.ws.status(), p.ws.timeout_site()) for p in probs if p.ws.status() != 0]
+    assert not bad, "device status after the eager pass (K, N, M, code, (site, block, detail)): %s" % bad
     ev = [[[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for _ in range(nP)]
           for _ in range(EV_GRAPHS)]
     plain = torch.cuda.CUDAGraph()
@@ -246,8 +248,8 @@ def run_gpu(args, rank, world, local_rank):
         for _ in range(max(3, args.warmup)):
             plain.replay()
     stream.synchronize()
-    for p in probs:
-        assert p.ws.status() == 0, "device status %d" % p.ws.status()
+    bad = [(p.K, p.N, p.M, p.ws.status(), p.ws.timeout_site()) for p in probs if p.ws.status() != 0]
+    assert not bad, "device status (K, N, M, code, (site, block, detail)): %s" % bad
 
     K = args.steps
     n_ev = min(EV_GRAPHS, K)
@@ -275,8 +277,8 @@ def run_gpu(args, rank, world, local_rank):
     step_ms = max_over_ranks(t0.elapsed_time(t1) / K, device) if world > 1 else t0.elapsed_time(t1) / K
     gemm_ms = [sum(ev[g][i][1].elapsed_time(ev[g][i][2]) for g in range(n_ev)) / n_ev for i in range(nP)]
     act_ms = [sum(ev[g][i][0].elapsed_time(ev[g][i][1]) for g in range(n_ev)) / n_ev for i in range(nP)]
-    for p in probs:
-        assert p.ws.status() == 0, "device status %d" % p.ws.status()
+    bad = [(p.K, p.N, p.M, p.ws.status(), p.ws.timeout_site()) for p in probs if p.ws.status() != 0]
+    assert not bad, "device status (K, N, M, code, (site, block, detail)): %s" % bad
 
     ops_step = sum(gemm_ops(p.M, p.N, p.K) for p in probs)
     per = []

@@ -160,8 +160,9 @@ qoq_status qoq_gemm_fp16_out(const int8_t *X8, const void *s_x_fp16, const int32
  * stream-K scratch lives in one fixed 8 MiB device array inside the library,
  * which every GPU that loads the library keeps until the process exits. That
  * bounds the problem: it needs 1280 + (SM count) * T * 512 bytes, T being the
- * token tile (16, 32, 64, ... for M <= 16, 32, 64, ...), so M <= 64 on a
- * 148-SM B200; larger problems return QOQ_ERR_WORKSPACE and launch nothing.
+ * token tile the library picks for (M, N, K) (16 for M <= 16, 32 for M <= 32,
+ * 32 or 64 for M <= 64), so M <= 64 on a 148-SM B200; larger problems return
+ * QOQ_ERR_WORKSPACE and launch nothing.
  *
  * status: optional device int32; when non-NULL the call copies the device
  * status word of this call (0, QOQ_ERR_BAD_BLOB or QOQ_ERR_TIMEOUT) into it

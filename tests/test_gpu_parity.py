@@ -8,7 +8,7 @@ import pytest
 
 import oracle
 from w4a8_quantized_gemm_qoq_b200 import inputs, qoq
-from gpu_helpers import check_full, check_sampled, dev, host, assert_fp16_close, torch
+from gpu_helpers import check_full, check_sampled, dev, host, assert_fp16_close, sample_tiles, torch
 
 pytestmark = [pytest.mark.gpu, pytest.mark.filterwarnings("ignore::RuntimeWarning")]
 
@@ -144,3 +144,60 @@ def test_qwen15_72b_shapes(M, K, N):
 @pytest.mark.parametrize("M", [1, 8, 64, 1024])
 def test_llama2_7b_per_channel_shapes(M, K, N):
     check_sampled(M, N, K, 0, seed=K + M, rows=12)
+
+
+# ------------------------------------------ back-to-back graph replays
+
+def test_graph_replays_are_bit_identical():
+    """Act quant + GEMM for several shapes captured in one CUDA graph and
+    replayed back to back: every replay reproduces the eager outputs bit for
+    bit with a clean status word. The shapes cover token tiles whose pipeline
+    has an odd stage count (16, 32, 256 tokens) and long per-CTA k ranges,
+    where a stage barrier is waited on many times per launch; sampled rows of
+    the eager result are checked against the oracle."""
+    t = torch()
+    cases = [(1, 4096, 28672), (32, 14336, 4096), (8192, 14336, 4096), (2048, 4096, 4096)]
+    probs = []
+    for i, (M, K, N) in enumerate(cases):
+        X = inputs.make_activations(M, K, seed=700 + i, token_scale_span=(-3, 1) if M > 256 else None)
+        W = inputs.make_weights(N, K, seed=700 + i)
+        Xd = dev(X)
+        blob = qoq.quantize_weights(dev(W), 128)
+        X8 = t.empty((M, K), dtype=t.int8, device="cuda")
+        s_x = t.empty((M,), dtype=t.float16, device="cuda")
+        rs = t.empty((M,), dtype=t.int32, device="cuda")
+        Y = t.empty((M, N), dtype=t.float16, device="cuda")
+        ws = qoq.Workspace.for_shape(M, N, K, 128)
+        probs.append(dict(M=M, N=N, K=K, X=X, W=W, Xd=Xd, blob=blob, X8=X8, s_x=s_x, rs=rs, Y=Y, ws=ws))
+
+    def step():
+        for p in probs:
+            qoq.quantize_act_per_token(p["Xd"], p["X8"], p["s_x"], p["rs"])
+            qoq.gemm_fp16_out(p["X8"], p["s_x"], p["blob"], p["N"], p["K"], 128, rowsum=p["rs"], ws=p["ws"], Y=p["Y"])
+
+    stream = t.cuda.Stream()
+    with t.cuda.stream(stream):
+        step()
+    stream.synchronize()
+    ref = [p["Y"].clone() for p in probs]
+    for p in probs:
+        assert p["ws"].status() == 0
+    g = t.cuda.CUDAGraph()
+    with t.cuda.graph(g, stream=stream):
+        step()
+    for r in range(30):
+        with t.cuda.stream(stream):
+            g.replay()
+        stream.synchronize()
+        for i, p in enumerate(probs):
+            assert p["ws"].status() == 0, "replay %d case %d: status %d %s" % (r, i, p["ws"].status(),
+                                                                             p["ws"].timeout_site())
+            assert t.equal(p["Y"], ref[i]), "replay %d case %d: output differs from the eager run" % (r, i)
+    for i, p in enumerate(probs):
+        rows = inputs.sample_rows(p["M"], 6, seed=i)
+        X8s, s_xs, _ = oracle.quantize_act_per_token(p["X"][rows])
+        Yh = host(ref[i])[rows]
+        for nt in sample_tiles(p["N"] // 128, seed=i)[:3]:
+            _, d = oracle.quantize_weights(p["W"][nt * 128:(nt + 1) * 128], 128)
+            want = oracle.epilogue_fp16(oracle.gemm_int(X8s, d["Wint"]), s_xs, d["s_w"])
+            assert_fp16_close(Yh[:, nt * 128:(nt + 1) * 128], want, "graph case %d tile %d" % (i, nt))

@@ -18,17 +18,21 @@
 //     MMA's N dimension (16..256), staged by TMA in shared memory with the
 //     128-byte swizzle. Dequantised weights go registers -> TMEM and never
 //     touch shared memory, leaving shared-memory bandwidth to the copies.
-//   * one dequant thread owns one weight row for one 128-wide k-tile, which is
-//     exactly one quantisation group, so the group's (s, z*s) is a per-thread
-//     scalar. 8 nibbles per 32-bit word decode with and/shift, one 32-bit
+//   * one dequant thread owns half of one weight row of a 128-wide k-tile,
+//     which lies in exactly one quantisation group, so the group's (s, z*s)
+//     is a per-thread scalar. 8 nibbles per 32-bit word decode with and/shift, one 32-bit
 //     multiply-add (q*s <= 240 and q*s + 128 - z*s in [7, 249] never carry
 //     between bytes) and one xor that turns excess-128 bytes into int8.
 //   * warp roles: 1 TMA producer warp, 1 MMA warp, two dequant warpgroups that
-//     alternate pipeline units, one epilogue warpgroup; the role loops are
-//     warp-uniform and lane 0 issues TMA / MMA / commit.
+//     split every pipeline unit by columns, one epilogue warpgroup; the role
+//     loops are warp-uniform and lane 0 issues TMA / MMA / commit.
 //   * a pipeline unit is up to KB consecutive k-tiles of one n-tile: one bulk
 //     copy of the packed weights, one TMA per token tile, one TMEM A buffer,
 //     one commit that frees both the shared-memory stage and the TMEM buffer.
+//   * ready for programmatic dependent launch: everything the previous kernel
+//     may write (activations, scales, outputs, workspace) is touched only
+//     after griddepcontrol.wait, and the first weight copies are issued
+//     before it (the launch attribute is off; see kProgrammaticLaunch).
 //   * persistent stream-K at k-tile granularity: the (token tile, n-tile,
 //     k-tile) blocks are split evenly over at most one CTA per SM. A tile cut
 //     between CTAs is finished by its owner -- the CTA holding the tile's
@@ -216,7 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < S; ++s) {
             mbar_init(&ctl->full[s], 1);
             mbar_init(&ctl->freed[s], 1);
-            mbar_init(&ctl->a_full[s], 4);
+            mbar_init(&ctl->a_full[s], 8);   // the eight dequant warps
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&ctl->acc_full[b], 1);
@@ -224,10 +228,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_init(&ctl->final_bar, 1);
         mbar_fence_init();
+        // No kernel that releases its dependents early (this GEMM, the
+        // activation quantiser) writes a blob, so the blob may be read before
+        // griddepcontrol.wait; read at L2, as the TMA weight copies are.
         const int32_t *h = reinterpret_cast<const int32_t *>(p.blob);
         if ((uint32_t)ld_cg_s32(h) != kMagic || (uint32_t)ld_cg_s32(h + 1) != kVersion ||
             ld_cg_s32(h + 2) != p.N || ld_cg_s32(h + 3) != p.K || ld_cg_s32(h + 4) != p.group)
-            wd.fail(QOQ_ERR_BAD_BLOB);
+            ctl->abort_flag = 1;   // reported on the status word after griddepcontrol.wait
     }
     if (warp == kWarpProducer && lane == 0) prefetch_tensormap(&tmap_x);
     if (warp == kWarpMma) {
@@ -238,7 +245,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = ctl->tmem_base;
+    griddep_launch_dependents();   // the next kernel may start its own set-up
     const bool bad_blob = wd.aborted();
+    if (bad_blob && threadIdx.x == 0) {
+        griddep_wait();
+        atomicCAS(p.status, 0, QOQ_ERR_BAD_BLOB);
+    }
 
     // Stream-K share of this CTA: k-tile blocks [b0, b1) in (token tile,
     // n-tile, k-tile) order, k-tile fastest.
@@ -267,11 +279,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tma_load_2d(stage_x(s) + j * C::kXTile, &tmap_x, &ctl->full[s], (c.kt + j) * kTileK,
                                 c.mt * TOK, pol_x);
             };
-            int issued = 0;
-            int s = 0;
-            uint32_t ph = 0;
-            for (int i = 0; !cur.done(); ++i) {
-                const bool ok = __all_sync(0xffffffffu, wait_bounded(&ctl->freed[s], ph ^ 1u, wd));
+            // The first S units need no free stage: start their weight copies
+            // before waiting for the previous kernel, then their token tiles.
+            int npre = 0;
+            {
+                UnitCursor<KB> c1 = cur;
+                for (; npre < S && !c1.done(); ++npre) {
+                    if (lane == 0) issue_w(npre, c1);
+                    c1.advance();
+                }
+            }
+            __syncwarp();
+            griddep_wait();
+            if (lane == 0) {
+                UnitCursor<KB> c2 = cur;
+                for (int i = 0; i < npre; ++i) {
+                    issue_x(i, c2);
+                    c2.advance();
+                }
+            }
+            __syncwarp();
+            for (int i = 0; i < npre; ++i) cur.advance();
+            int issued = npre;
+            int s = npre % S;
+            uint32_t ph = (uint32_t)(npre / S) & 1u;
+            for (int i = npre; !cur.done(); ++i) {
+                const bool ok = __all_sync(0xffffffffu, wait_bounded(&ctl->freed[s], ph ^ 1u, wd, kSiteProducerFreed, i));
                 if (!ok) break;
                 if (lane == 0) {
                     issue_w(s, cur);
@@ -295,13 +328,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr uint32_t idesc = idesc_i8(128, TOK, true, true);
             UnitCursor<KB> cur;
             cur.init(b0, b1, KT, p.NT);
-            int s = 0, seg = 0;
+            int s = 0, seg = 0, unit = 0;
             uint32_t ph = 0;
             bool ok = true;
             while (ok && !cur.done()) {
                 const int buf = seg % C::kAccBufs;
                 const uint32_t aph = (uint32_t)(seg / C::kAccBufs) & 1u;
-                ok = __all_sync(0xffffffffu, wait_bounded(&ctl->acc_empty[buf], aph ^ 1u, wd));
+                ok = __all_sync(0xffffffffu, wait_bounded(&ctl->acc_empty[buf], aph ^ 1u, wd, kSiteMmaAccEmpty, seg));
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(buf * TOK);
@@ -310,7 +343,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // The token tile (shared memory) and the dequantised weights
                     // (TMEM) of this unit.
                     ok = __all_sync(0xffffffffu,
-                                    wait_bounded(&ctl->full[s], ph, wd) && wait_bounded(&ctl->a_full[s], ph, wd));
+                                    wait_bounded(&ctl->full[s], ph, wd, kSiteMmaOperands, 2 * unit) &&
+                                        wait_bounded(&ctl->a_full[s], ph, wd, kSiteMmaOperands, 2 * unit + 1));
                     if (!ok) break;
                     tc_fence_after();
                     if (lane == 0) {
@@ -327,6 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     __syncwarp();
                     first = false;
+                    ++unit;
                     if (++s == S) {
                         s = 0;
                         ph ^= 1u;
@@ -346,7 +381,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
         } else if (warp >= kWarpDequant0 && warp < kWarpEpilogue) {
             // ------------------------------------------------ dequant
-            const int g = (warp - kWarpDequant0) >> 2;     // warpgroup 0 / 1: even / odd units
+            // Both warpgroups work on every unit: warpgroup h decodes code
+            // chunks 2h, 2h+1 of each row (k 64h .. 64h+63 of the k-tile, TMEM
+            // columns 16h .. 16h+15). Every waiter thus sees every phase of
+            // every stage barrier, so parity waits cannot alias for any stage
+            // count.
+            const int h = (warp - kWarpDequant0) >> 2;
             const int quarter = warp & 3;                    // TMEM lanes 32q .. 32q+31
             const int r = quarter * 32 + lane;               // weight row in the tile
             const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
@@ -355,30 +395,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             int s = 0;
             uint32_t ph = 0;
             for (int i = 0; !cur.done(); ++i, cur.advance()) {
-                const int unit_s = s;
-                const uint32_t unit_ph = ph;
-                if (++s == S) {
-                    s = 0;
-                    ph ^= 1u;
-                }
-                if ((i & 1) != g) continue;
                 // full[s] for this unit implies the producer saw freed[s] for
                 // the unit S earlier, i.e. TMEM A buffer s is no longer read.
-                const bool ok = __all_sync(0xffffffffu, wait_bounded(&ctl->full[unit_s], unit_ph, wd));
+                const bool ok = __all_sync(0xffffffffu, wait_bounded(&ctl->full[s], ph, wd, kSiteDequantFull, i));
                 if (!ok) break;
-                const uint32_t a_col = tmem_base + lane_addr + (uint32_t)(C::kACol0 + unit_s * KB * 32);
+                tc_fence_after();   // the TMEM writes below come after the wait (and the MMA reads it implies)
+                const uint32_t a_col = tmem_base + lane_addr + (uint32_t)(C::kACol0 + s * KB * 32 + 16 * h);
                 for (int j = 0; j < cur.nk; ++j) {
-                    const uint32_t wbase = smem_u32(stage_w(unit_s) + j * C::kWTile);
+                    const uint32_t wbase = smem_u32(stage_w(s) + j * C::kWTile);
                     uint32_t sc = 0u, c4 = 0u;
                     if (MODE == 0) {
                         const uint32_t sz = lds16(wbase + 8192 + 2 * r);
                         sc = sz & 0xFFu;
                         c4 = (uint32_t)(128 - (int)(int8_t)(sz >> 8)) * 0x01010101u;
                     }
-                    uint32_t o[32];
+                    uint32_t o[16];
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const uint4 v = lds128(wbase + c * 2048 + r * 16);
+                    for (int c = 0; c < 2; ++c) {
+                        const uint4 v = lds128(wbase + (2 * h + c) * 2048 + r * 16);
                         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
@@ -393,12 +427,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                             }
                         }
                     }
-                    tmem_st32_wait(a_col + (uint32_t)(j * 32), o);
+                    tmem_st16_wait(a_col + (uint32_t)(j * 32), o);
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&ctl->a_full[unit_s]);
+                if (lane == 0) mbar_arrive(&ctl->a_full[s]);
                 __syncwarp();
+                if (++s == S) {
+                    s = 0;
+                    ph ^= 1u;
+                }
             }
         } else if (warp >= kWarpEpilogue) {
             // ------------------------------------------------ epilogue
@@ -406,6 +444,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int r = quarter * 32 + lane;
             const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
             const bool leader = (threadIdx.x == kWarpEpilogue * 32);
+            griddep_wait();   // outputs, scales, row sums and workspace belong to the previous kernel until now
             UnitCursor<KB> cur;
             cur.init(b0, b1, KT, p.NT);
             int seg = 0;
@@ -421,7 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // Every lane spins on its own; the vote reconverges the warp
                 // before the named barrier, and all four epilogue warps leave
                 // together (the shared-tile paths below meet at named barriers).
-                const bool ok = __all_sync(0xffffffffu, wait_bounded(&ctl->acc_full[buf], aph, wd));
+                const bool ok = __all_sync(0xffffffffu, wait_bounded(&ctl->acc_full[buf], aph, wd, kSiteEpilogueAcc, seg));
                 if (named_bar_any(1, 128, !ok)) break;
                 tc_fence_after();
                 const int n = nt * kTileN + r;
@@ -458,27 +497,39 @@ __global__ void __launch_bounds__(kThreads, 1)
                         bool got = true;
                         if (leader)
                             for (uint32_t c = c_first; c <= c_last && got; ++c)
-                                got = wait_flag_bounded(p.flags + c, wd);
+                                got = wait_flag_bounded(p.flags + c, wd, (int)c);
                         __syncwarp();
                         if (named_bar_any(1, 128, !got)) break;
                         __threadfence();
                     }
+                    // 16 token columns at a time; the partial sums of up to four
+                    // contributors are loaded together (one L2 round trip).
+                    constexpr int CO = 16;
 #pragma unroll 1
-                    for (int c0 = 0; c0 < TOK; c0 += CH) {
-                        uint32_t v[CH];
-                        tmem_load<CH>(acc_addr + (uint32_t)c0, v);
-                        if (c0 + CH >= TOK) {
+                    for (int c0 = 0; c0 < TOK; c0 += CO) {
+                        uint32_t v[CO];
+                        tmem_load<CO>(acc_addr + (uint32_t)c0, v);
+                        if (c0 + CO >= TOK) {
                             tc_fence_before();
                             __syncwarp();
                             if (lane == 0) mbar_arrive(&ctl->acc_empty[buf]);
                         }
-                        for (uint32_t c = c_first; c <= c_last; ++c) {
-                            const int32_t *part = p.partials + (long long)c * TOK * kTileN;
+#pragma unroll 1
+                        for (uint32_t c = c_first; c <= c_last; c += 4) {
+                            int32_t t[4][CO];
 #pragma unroll
-                            for (int j = 0; j < CH; ++j)
-                                v[j] = (uint32_t)((int32_t)v[j] + ld_cg_s32(part + (c0 + j) * kTileN + r));
+                            for (int cc = 0; cc < 4; ++cc) {
+                                const int32_t *part = p.partials + (long long)(c + cc) * TOK * kTileN + c0 * kTileN + r;
+#pragma unroll
+                                for (int j = 0; j < CO; ++j)
+                                    t[cc][j] = (c + cc <= c_last) ? ld_cg_s32(part + j * kTileN) : 0;
+                            }
+#pragma unroll
+                            for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+                                for (int j = 0; j < CO; ++j) v[j] = (uint32_t)((int32_t)v[j] + t[cc][j]);
                         }
-                        store_outputs<CH, MODE>(p, v, m0 + c0, n, col_scale, col_zero);
+                        store_outputs<CO, MODE>(p, v, m0 + c0, n, col_scale, col_zero);
                     }
                     if (c_last >= c_first) {
                         named_bar_sync(1, 128);
@@ -591,13 +642,17 @@ static qoq_status launch_gemm_t(const GemmArgs &a, cudaStream_t stream) {
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = C::kSmemBytes;
     cfg.stream = stream;
-    cfg.numAttrs = 0;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = kProgrammaticLaunch ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, qoq_gemm_kernel<TOK, MODE>, p, tmap) == cudaSuccess ? QOQ_OK : QOQ_ERR_CUDA;
 }
 
 template <int MODE>
 static qoq_status launch_gemm_mode(const GemmArgs &a, cudaStream_t stream) {
-    switch (token_tile_for(a.M)) {
+    switch (token_tile_for(a.M, a.N, a.K)) {
         case 16: return launch_gemm_t<16, MODE>(a, stream);
         case 32: return launch_gemm_t<32, MODE>(a, stream);
         case 64: return launch_gemm_t<64, MODE>(a, stream);

@@ -31,7 +31,7 @@ qoq_status gemm_common(const int8_t *X8, const void *s_x, const int32_t *rowsum,
     if (st != QOQ_OK) return st;
     if ((st = check_group(group)) != QOQ_OK) return st;
     if (M * N > (int64_t)1 << 40) return QOQ_ERR_UNSUPPORTED;
-    const size_t need = workspace_bytes_for(M);
+    const size_t need = workspace_bytes_for(M, N, K);
     if (ws == nullptr) {
         *ws_bytes = need;
         return QOQ_OK;

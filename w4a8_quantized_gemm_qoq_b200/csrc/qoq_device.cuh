@@ -60,22 +60,38 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // HBM reads of a few KB), so running out means a lost arrival.
 constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;  // 1 s
 
-// Shared abort flag + global status word used by the bounded waits.
+// Where a bounded wait gave up (workspace word 1 after QOQ_ERR_TIMEOUT).
+enum WaitSite : int {
+    kSiteProducerFreed = 1,   // TMA producer waiting for a free stage
+    kSiteMmaAccEmpty = 2,     // MMA warp waiting for the epilogue to drain an accumulator
+    kSiteMmaOperands = 3,     // MMA warp waiting for a token tile / dequantised weights
+    kSiteDequantFull = 4,     // dequant warp waiting for a stage's copies
+    kSiteEpilogueAcc = 5,     // epilogue waiting for an accumulator
+    kSiteOwnerFlag = 6,       // tile owner waiting for a contributor's partial sums
+};
+
+// Shared abort flag + global status word used by the bounded waits. The CTA
+// that first fails also records, after the status word, the wait site, its
+// block index and a site-specific detail (unit, segment or contributor).
 struct Watchdog {
     volatile int *abort_flag;  // shared memory, 0 = healthy
     int *status;               // global status word (workspace[0]); may be null
     __device__ __forceinline__ bool aborted() const { return *abort_flag != 0; }
-    __device__ __forceinline__ void fail(int code) const {
+    __device__ __forceinline__ void fail(int code, int site = 0, int detail = 0) const {
         *abort_flag = 1;
-        if (status) atomicCAS(status, 0, code);
+        if (status && atomicCAS(status, 0, code) == 0) {
+            status[1] = site;
+            status[2] = (int)blockIdx.x;
+            status[3] = detail;
+        }
     }
 };
 
 // Wait for the phase of `bar` with the given parity to complete. Returns
 // false (after raising the CTA abort flag and the status word) when the wait
 // runs past `limit_ns`, or when another role of the CTA has aborted.
-__device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, const Watchdog &wd,
-                                             uint64_t limit_ns = kWaitLimitNs) {
+__device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, const Watchdog &wd, int site,
+                                             int detail, uint64_t limit_ns = kWaitLimitNs) {
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait(a, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
@@ -84,7 +100,7 @@ __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, con
         if ((it & 31u) == 0) {
             if (wd.aborted()) return false;
             if (globaltimer_ns() - t0 > limit_ns) {
-                wd.fail(QOQ_ERR_TIMEOUT);
+                wd.fail(QOQ_ERR_TIMEOUT, site, detail);
                 return false;
             }
         }
@@ -205,41 +221,18 @@ __device__ __forceinline__ uint64_t smem_desc_k_sw128(uint32_t saddr) {
     return d;
 }
 
-// 32 lanes x 32 columns of 32-bit values: thread t <-> lane base+t.
-// The store and its completion wait are one asm block so the source
-// registers are never reused early.
-__device__ __forceinline__ void tmem_st32_wait(uint32_t taddr, const uint32_t (&r)[32]) {
+// 32 lanes x 16 columns of 32-bit values: thread t <-> lane base+t. The
+// store and its completion wait are one asm block so the source registers
+// are never reused early.
+__device__ __forceinline__ void tmem_st16_wait(uint32_t taddr, const uint32_t (&r)[16]) {
+    __syncwarp();   // warp-collective (.sync.aligned)
     asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
-        "%13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};\n\t"
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
+        "%13, %14, %15, %16};\n\t"
         "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
         "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
-        "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
-        "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
         : "memory");
-}
-
-// 32 lanes x 8 columns store; the source registers are read at issue. A later
-// tmem_st_wait() makes all prior stores of this thread visible to the MMA.
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3,
-                                         uint32_t r4, uint32_t r5, uint32_t r6, uint32_t r7) {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
-                 "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(r4), "r"(r5), "r"(r6), "r"(r7)
-                 : "memory");
-}
-
-__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
-// One lane of the (fully active) warp gets true.
-__device__ __forceinline__ bool elect_one() {
-    uint32_t pred;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t.reg .b32 r;\n\t"
-        "elect.sync r|p, 0xffffffff;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(pred));
-    return pred != 0;
 }
 
 // Load + wait in one asm block so no use of the destination registers can be
@@ -296,7 +289,7 @@ __device__ __forceinline__ int32_t ld_acquire_gpu(const int32_t *p) {
 }
 
 // Spin until *flag != 0, bounded like the pipeline waits.
-__device__ __forceinline__ bool wait_flag_bounded(const int32_t *flag, const Watchdog &wd,
+__device__ __forceinline__ bool wait_flag_bounded(const int32_t *flag, const Watchdog &wd, int detail,
                                                   uint64_t limit_ns = kWaitLimitNs) {
     if (ld_acquire_gpu(flag) != 0) return true;
     const uint64_t t0 = globaltimer_ns();
@@ -306,7 +299,7 @@ __device__ __forceinline__ bool wait_flag_bounded(const int32_t *flag, const Wat
         if ((it & 15u) == 0) {
             if (wd.aborted()) return false;
             if (globaltimer_ns() - t0 > limit_ns) {
-                wd.fail(QOQ_ERR_TIMEOUT);
+                wd.fail(QOQ_ERR_TIMEOUT, kSiteOwnerFlag, detail);
                 return false;
             }
         }

@@ -14,6 +14,17 @@ constexpr int kTileK = 128;        // K per tile = one quantisation group
 constexpr int kGroup = 128;
 constexpr int kMaxK = 65536;
 constexpr int kMaxGrid = 256;      // upper bound of the persistent grid (>= SM count)
+
+// Programmatic dependent launch (griddepcontrol) between the activation
+// quantiser and the GEMM. The kernels are written for it -- everything a
+// predecessor may write is touched only after griddepcontrol.wait, and the
+// GEMM starts its weight copies before that wait -- but it is off: with it on,
+// GEMMs with 256-token tiles stalled until their bounded waits ran out
+// (QOQ_ERR_TIMEOUT) in back-to-back CUDA graph replays of large prefill
+// shapes, whichever of the two launches carried the attribute, and the cause
+// is not identified. Without the launch attribute griddepcontrol.wait and
+// griddepcontrol.launch_dependents do nothing.
+constexpr bool kProgrammaticLaunch = false;
 constexpr uint32_t kMagic = 0x57514F51u;   // 'Q','O','Q','W'
 constexpr uint32_t kVersion = 1u;
 constexpr int kHeaderBytes = 256;
@@ -44,13 +55,22 @@ inline BlobLayout blob_layout(int64_t N, int64_t K, int group) {
     return L;
 }
 
-// Token-tile width (MMA N) chosen for M tokens.
-inline int token_tile_for(int64_t M) {
+// Token-tile width (MMA N) for an M x N x K problem. Small M uses the
+// smallest tile that holds all tokens. Beyond that the choice trades weight
+// re-reads and dequantisation (once per token tile) against enough work units
+// for every SM and the stream-K partial-sum traffic; the thresholds below come
+// from B200 measurements on Llama-3-8B linear shapes. Long K (>= 64 k-tiles)
+// prefers the widest tile, whose tensor work per k-tile hides the dequant.
+inline int token_tile_for(int64_t M, int64_t N, int64_t K) {
+    const int64_t NT = N / kTileN, KT = K / kTileK;
+    auto blocks = [&](int64_t tok) { return ((M + tok - 1) / tok) * NT * KT; };
     if (M <= 16) return 16;
     if (M <= 32) return 32;
-    if (M <= 64) return 64;
-    if (M <= 128) return 128;
-    return 256;
+    if (M <= 64) return blocks(64) >= 2500 ? 64 : 32;
+    if (M <= 128) return 64;
+    if (M <= 256) return blocks(128) >= 7000 ? 128 : 64;
+    if (M <= 512) return 128;
+    return KT >= 64 ? 256 : 128;
 }
 
 // Workspace: [0, 256) status word + reserved; then int32 flags [kMaxGrid]
@@ -58,8 +78,8 @@ inline int token_tile_for(int64_t M) {
 // partial tiles [kMaxGrid][tok][128] (scratch).
 static_assert(256 + 4 * kMaxGrid == QOQ_WORKSPACE_CONTROL_BYTES, "workspace control layout");
 
-inline size_t workspace_bytes_for(int64_t M) {
-    const int tok = token_tile_for(M);
+inline size_t workspace_bytes_for(int64_t M, int64_t N, int64_t K) {
+    const int tok = token_tile_for(M, N, K);
     return 256 + sizeof(int32_t) * kMaxGrid + sizeof(int32_t) * (size_t)kMaxGrid * tok * kTileN;
 }
 

@@ -53,7 +53,8 @@ __global__ void __launch_bounds__(kActThreads) act_quant_kernel(const __half *__
     __shared__ int red_i[kActThreads / 32];
     __shared__ float s_shared;
     // X may come from the previous kernel in the stream; release the next one
-    // (the GEMM) so its set-up and weight copies overlap this kernel.
+    // (the GEMM) so its set-up and weight copies could overlap this kernel
+    // under programmatic launch (kProgrammaticLaunch).
     griddep_wait();
     griddep_launch_dependents();
     const int64_t m = blockIdx.x;
@@ -63,12 +64,15 @@ __global__ void __launch_bounds__(kActThreads) act_quant_kernel(const __half *__
 
     uint4 v[NR];
     float amax = 0.0f;
+    // The eight halves of a 16-byte chunk are taken apart with shifts only:
+    // no local has its address taken, so the kernel keeps no stack frame.
     auto absmax8 = [&](const uint4 &u) {
-        const __half2 *h = reinterpret_cast<const __half2 *>(&u);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            float2 f = __half22float2(h[i]);
-            amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+            const float lo = __half2float(__ushort_as_half((unsigned short)(w[i] & 0xFFFFu)));
+            const float hi = __half2float(__ushort_as_half((unsigned short)(w[i] >> 16)));
+            amax = fmaxf(amax, fmaxf(fabsf(lo), fabsf(hi)));
         }
     };
     if (NCH > 0) {
@@ -100,16 +104,21 @@ __global__ void __launch_bounds__(kActThreads) act_quant_kernel(const __half *__
     int sum = 0;
     int8_t *out = X8 + m * K;
     auto quant8 = [&](const uint4 &u, int k) {
-        const __half2 *h = reinterpret_cast<const __half2 *>(&u);
-        uint32_t packed[2] = {0u, 0u};
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+        uint32_t packed0 = 0u, packed1 = 0u;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            float2 f = __half22float2(h[i]);
-            int q0 = quant_code(f.x, s, 127), q1 = quant_code(f.y, s, 127);
+            const float lo = __half2float(__ushort_as_half((unsigned short)(w[i] & 0xFFFFu)));
+            const float hi = __half2float(__ushort_as_half((unsigned short)(w[i] >> 16)));
+            const int q0 = quant_code(lo, s, 127), q1 = quant_code(hi, s, 127);
             sum += q0 + q1;
-            packed[i >> 1] |= ((uint32_t)(q0 & 0xFF) << (16 * (i & 1))) | ((uint32_t)(q1 & 0xFF) << (16 * (i & 1) + 8));
+            const uint32_t pair = ((uint32_t)(q0 & 0xFF) | ((uint32_t)(q1 & 0xFF) << 8)) << (16 * (i & 1));
+            if (i < 2)
+                packed0 |= pair;
+            else
+                packed1 |= pair;
         }
-        *reinterpret_cast<uint2 *>(out + k) = make_uint2(packed[0], packed[1]);
+        *reinterpret_cast<uint2 *>(out + k) = make_uint2(packed0, packed1);
     };
     if (NCH > 0) {
 #pragma unroll
@@ -143,7 +152,7 @@ static cudaError_t launch_act_quant_t(const void *X, int64_t M, int64_t K, int8_
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = kProgrammaticLaunch ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, act_quant_kernel<NCH>, static_cast<const __half *>(X), (int)K, X8,
                               static_cast<__half *>(s_x), rowsum);
 }

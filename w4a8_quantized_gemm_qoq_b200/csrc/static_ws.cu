@@ -62,7 +62,7 @@ extern "C" qoq_status qoq_gemm_fp16_out_static_ws(const int8_t *X8, const void *
         return QOQ_ERR_CUDA;
     // Scratch this call needs: control words plus one partial tile per CTA
     // of the persistent grid.
-    const int64_t tok = token_tile_for(M);
+    const int64_t tok = token_tile_for(M, N, K);
     const int64_t blocks = ((M + tok - 1) / tok) * (N / kTileN) * (K / kTileK);
     int64_t grid = sms < kMaxGrid ? sms : kMaxGrid;
     if (blocks < grid) grid = blocks;

@@ -135,6 +135,12 @@ class Workspace:
     def status(self) -> int:
         return int(self.buf[:4].view(dtype=__import__("torch").int32).item())
 
+    def timeout_site(self):
+        """(wait site, block index, detail) recorded with QOQ_ERR_TIMEOUT."""
+        import torch
+        w = self.buf[:16].view(dtype=torch.int32).tolist()
+        return tuple(w[1:4])
+
     def control_clear(self) -> bool:
         return not bool(self.buf[:WORKSPACE_CONTROL_BYTES].any().item())
 
