@@ -123,8 +123,13 @@ qoq_status qoq_quantize_weights(const void *W_fp16, int64_t N, int64_t K, int gr
  * stream-K partial sums. So one workspace serves any number of calls on one
  * stream; calls that may overlap on the device need separate workspaces. The
  * status word is 0, or a qoq_status code (QOQ_ERR_BAD_BLOB, QOQ_ERR_TIMEOUT)
- * written by the device; after such an error, zero-fill the control bytes
- * again. Size query: workspace == NULL stores the required size for
+ * written by the device. With QOQ_ERR_TIMEOUT the next three int32 words say
+ * where a bounded wait (1 s) gave up: the wait site (1 producer waiting for a
+ * free stage, 2 MMA waiting for a drained accumulator, 3 MMA waiting for a
+ * stage's operands, 4 dequantiser waiting for a stage's copies, 5 epilogue
+ * waiting for an accumulator, 6 tile owner waiting for a contributor), the
+ * CTA index, and the unit, segment or contributor index. After such an error,
+ * zero-fill the control bytes again. Size query: workspace == NULL stores the required size for
  * (M, N, K, group_size) in *workspace_bytes and returns QOQ_OK.
  */
 qoq_status qoq_w4a8_gemm(const int8_t *X8, const int32_t *rowsum, const void *blob,

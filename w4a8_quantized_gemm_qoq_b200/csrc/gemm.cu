@@ -29,10 +29,10 @@
 //   * a pipeline unit is up to KB consecutive k-tiles of one n-tile: one bulk
 //     copy of the packed weights, one TMA per token tile, one TMEM A buffer,
 //     one commit that frees both the shared-memory stage and the TMEM buffer.
-//   * ready for programmatic dependent launch: everything the previous kernel
-//     may write (activations, scales, outputs, workspace) is touched only
-//     after griddepcontrol.wait, and the first weight copies are issued
-//     before it (the launch attribute is off; see kProgrammaticLaunch).
+//   * programmatic dependent launch: the set-up and the first weight copies
+//     overlap the previous kernel in the stream; everything the previous
+//     kernel may write (activations, scales, outputs, workspace) is touched
+//     only after griddepcontrol.wait.
 //   * persistent stream-K at k-tile granularity: the (token tile, n-tile,
 //     k-tile) blocks are split evenly over at most one CTA per SM. A tile cut
 //     between CTAs is finished by its owner -- the CTA holding the tile's

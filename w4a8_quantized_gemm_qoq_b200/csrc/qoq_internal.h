@@ -16,15 +16,13 @@ constexpr int kMaxK = 65536;
 constexpr int kMaxGrid = 256;      // upper bound of the persistent grid (>= SM count)
 
 // Programmatic dependent launch (griddepcontrol) between the activation
-// quantiser and the GEMM. The kernels are written for it -- everything a
-// predecessor may write is touched only after griddepcontrol.wait, and the
-// GEMM starts its weight copies before that wait -- but it is off: with it on,
-// GEMMs with 256-token tiles stalled until their bounded waits ran out
-// (QOQ_ERR_TIMEOUT) in back-to-back CUDA graph replays of large prefill
-// shapes, whichever of the two launches carried the attribute, and the cause
-// is not identified. Without the launch attribute griddepcontrol.wait and
-// griddepcontrol.launch_dependents do nothing.
-constexpr bool kProgrammaticLaunch = false;
+// quantiser and the GEMM: each kernel releases its successor right after its
+// own set-up, and touches what a predecessor may write only after
+// griddepcontrol.wait; the GEMM issues its first weight copies before that
+// wait. Kernels of other libraries in the stream are unaffected: a launch
+// without the attribute, or after a kernel that never releases early, waits
+// for full completion as usual.
+constexpr bool kProgrammaticLaunch = true;
 constexpr uint32_t kMagic = 0x57514F51u;   // 'Q','O','Q','W'
 constexpr uint32_t kVersion = 1u;
 constexpr int kHeaderBytes = 256;

@@ -53,8 +53,7 @@ __global__ void __launch_bounds__(kActThreads) act_quant_kernel(const __half *__
     __shared__ int red_i[kActThreads / 32];
     __shared__ float s_shared;
     // X may come from the previous kernel in the stream; release the next one
-    // (the GEMM) so its set-up and weight copies could overlap this kernel
-    // under programmatic launch (kProgrammaticLaunch).
+    // (the GEMM) so its set-up and weight copies overlap this kernel.
     griddep_wait();
     griddep_launch_dependents();
     const int64_t m = blockIdx.x;
