@@ -75,6 +75,29 @@ def load_peaks():
         return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
 
 
+def measured_traffic(workload):
+    """DRAM bytes per GEMM launch (dram__bytes_read.sum + dram__bytes_write.sum)
+    from the committed ncu summary of this workload, or None when there is
+    none or the GEMM sources have changed since it was taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "qoq_gemm_%s_llama3_8b_dram.md" % workload)
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and line.split(":")[0] in ("kernel_sources_sha256", "traffic_per_launch_bytes"):
+                k, v = line.split(":", 1)
+                vals[k] = v.strip()
+    h = hashlib.sha256()
+    for name in ("gemm.cu", "qoq_device.cuh"):
+        with open(os.path.join(ROOT, "w4a8_quantized_gemm_qoq_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    if vals.get("kernel_sources_sha256") != h.hexdigest() or "traffic_per_launch_bytes" not in vals:
+        return None
+    return int(vals["traffic_per_launch_bytes"])
+
+
 def roof_us(M, N, K, peaks):
     """Roofline time: the slower of HBM bytes and INT8 tensor work (INT8 peak =
     2 x the measured dense bf16 peak, the nominal 4.5/2.25 PFLOP/s ratio)."""
@@ -296,7 +319,8 @@ def run_gpu(args, rank, world, local_rank):
     if args.workload == "decode":
         achieved = tot_bytes / tot_gemm_us / 1e3
         roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm"], "unit": "GB/s",
-                    "frac": round(achieved / peaks["hbm"], 4), "traffic": None,
+                    "frac": round(achieved / peaks["hbm"], 4), "traffic": measured_traffic("decode"),
+                    "algorithmic_bytes_per_launch": round(tot_bytes / len(probs)),
                     "peak_source": peaks["src"], "kernel": "qoq_gemm_kernel",
                     "frac_of_time_roofline": round(sum(x["roof_us"] for x in per) / tot_gemm_us, 4)}
     else:
