@@ -18,14 +18,14 @@
 //     MMA's N dimension (16..256), staged by TMA in shared memory with the
 //     128-byte swizzle. Dequantised weights go registers -> TMEM and never
 //     touch shared memory, leaving shared-memory bandwidth to the copies.
-//   * one dequant thread owns half of one weight row of a 128-wide k-tile,
-//     which lies in exactly one quantisation group, so the group's (s, z*s)
-//     is a per-thread scalar. 8 nibbles per 32-bit word decode with and/shift, one 32-bit
+//   * one dequant thread owns one weight row of a 128-wide k-tile, which is
+//     exactly one quantisation group, so the group's (s, z*s) is a per-thread
+//     scalar. 8 nibbles per 32-bit word decode with and/shift, one 32-bit
 //     multiply-add (q*s <= 240 and q*s + 128 - z*s in [7, 249] never carry
 //     between bytes) and one xor that turns excess-128 bytes into int8.
-//   * warp roles: 1 TMA producer warp, 1 MMA warp, two dequant warpgroups that
-//     split every pipeline unit by columns, one epilogue warpgroup; the role
-//     loops are warp-uniform and lane 0 issues TMA / MMA / commit.
+//   * warp roles: 1 TMA producer warp, 2 MMA issuer warps (lane 0 each), two
+//     dequant warpgroups that take alternate pipeline units, one epilogue
+//     warpgroup.
 //   * a pipeline unit is up to KB consecutive k-tiles of one n-tile: one bulk
 //     copy of the packed weights, one TMA per token tile, one TMEM A buffer,
 //     one commit that frees both the shared-memory stage and the TMEM buffer.
@@ -52,7 +52,8 @@ namespace qoq {
 
 constexpr int kThreads = 512;            // 16 warps
 constexpr int kWarpProducer = 0;
-constexpr int kWarpMma = 1;
+constexpr int kWarpMma = 1;             // warps 1, 2: the two MMA issuers
+constexpr int kIssuers = 2;
 constexpr int kWarpDequant0 = 4;         // warps 4..11: two dequant warpgroups
 constexpr int kWarpEpilogue = 12;        // warps 12..15
 constexpr uint64_t kDrainNs = 100ull * 1000ull * 1000ull;   // 100 ms
@@ -71,8 +72,13 @@ struct GemmCfg {
     static constexpr int kStageBytes = (kXBytes + kWBytes + 1023) / 1024 * 1024;
     static constexpr int kSmemLimit = 232448;                   // 227 KB per CTA
     static constexpr int kReserve = 2048;                       // alignment slack + barriers
-    static constexpr int kAccBufs = TOK <= 128 ? 2 : 1;
-    static constexpr int kACol0 = kAccBufs * TOK;
+    // Two MMA issuers. With two-k-tile units, issuer j takes the units of
+    // index parity j (those its dequant warpgroup serves) into its own
+    // accumulator, and the epilogue adds the two; with one-k-tile units, issuer
+    // j takes token columns j*TOK/2 .. of every unit.
+    static constexpr int kAccCols = kKB == 2 ? 2 * TOK : TOK;   // TMEM columns per accumulator buffer
+    static constexpr int kAccBufs = (TOK == 64 || TOK == 256) ? 1 : 2;
+    static constexpr int kACol0 = kAccBufs * kAccCols;
     // One CTA per SM (shared memory use guarantees it), so the CTA takes all
     // 512 TMEM columns: accumulators first, then one A buffer per stage
     // (32 columns per dequantised 128x128 k-tile).
@@ -80,9 +86,12 @@ struct GemmCfg {
     static constexpr int kStagesSmem = (kSmemLimit - kReserve) / kStageBytes;
     static constexpr int kStagesTmem = (kTmemCols - kACol0) / (kKB * 32);
     static constexpr int kStagesMin = kStagesSmem < kStagesTmem ? kStagesSmem : kStagesTmem;
-    static constexpr int kStages = kStagesMin > 16 ? 16 : kStagesMin;
+    // Even, so that stage s is always dequantised by warpgroup s % 2 (the two
+    // warpgroups take alternate units); each warpgroup then waits on every
+    // phase of the stages it reads.
+    static constexpr int kStages = (kStagesMin > 16 ? 16 : kStagesMin) & ~1;
     static constexpr int kSmemBytes = kStages * kStageBytes + kReserve;
-    static_assert(kStages >= 3, "pipeline too shallow");
+    static_assert(kStages >= 4, "pipeline too shallow");
     static_assert(kACol0 + kStages * kKB * 32 <= kTmemCols, "TMEM over-subscribed");
     static_assert(kSmemBytes > 232448 / 2, "two CTAs per SM would contend for TMEM");
     static_assert(kXTile % 1024 == 0, "token tile must keep the swizzle atom aligned");
@@ -107,7 +116,7 @@ struct GemmParams {
 struct SharedCtl {
     uint64_t full[16], freed[16], a_full[16];
     uint64_t acc_full[2], acc_empty[2];
-    uint64_t final_bar;
+    uint64_t final_bar[2];
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -200,11 +209,20 @@ __device__ __forceinline__ void tmem_load<32>(uint32_t taddr, uint32_t (&v)[32])
     tmem_ld32_wait(taddr, v);
 }
 
+// v += the CH columns at taddr (the second issuer's accumulator); exact INT32.
+template <int CH>
+__device__ __forceinline__ void add_second(uint32_t taddr, uint32_t (&v)[CH]) {
+    uint32_t w[CH];
+    tmem_load<CH>(taddr, w);
+#pragma unroll
+    for (int j = 0; j < CH; ++j) v[j] = (uint32_t)((int32_t)v[j] + (int32_t)w[j]);
+}
+
 template <int TOK, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     qoq_gemm_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ CUtensorMap tmap_x) {
     using C = GemmCfg<TOK, MODE>;
-    constexpr int CH = TOK < 32 ? TOK : 32;
+    constexpr int CH = (TOK < 32 || C::kKB == 2) ? 16 : 32;   // epilogue TMEM chunk (16 when two accumulators are summed)
     constexpr int S = C::kStages;
     constexpr int KB = C::kKB;
     extern __shared__ uint8_t smem_raw[];
@@ -219,14 +237,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         ctl->abort_flag = 0;
         for (int s = 0; s < S; ++s) {
             mbar_init(&ctl->full[s], 1);
-            mbar_init(&ctl->freed[s], 1);
-            mbar_init(&ctl->a_full[s], 8);   // the eight dequant warps
+            mbar_init(&ctl->freed[s], C::kKB == 2 ? 1 : kIssuers);
+            mbar_init(&ctl->a_full[s], 4);   // the four warps of one dequant warpgroup
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&ctl->acc_full[b], 1);
+            mbar_init(&ctl->acc_full[b], kIssuers);
             mbar_init(&ctl->acc_empty[b], 4);
         }
-        mbar_init(&ctl->final_bar, 1);
+        mbar_init(&ctl->final_bar[0], 1);
+        mbar_init(&ctl->final_bar[1], 1);
         mbar_fence_init();
         // No kernel that releases its dependents early (this GEMM, the
         // activation quantiser) writes a blob, so the blob may be read before
@@ -323,70 +342,76 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int i = issued > S ? issued - S : 0; i < issued; ++i)
                     wait_drain(&ctl->full[i % S], (uint32_t)(i / S) & 1u, kDrainNs);
             __syncwarp();
-        } else if (warp == kWarpMma) {
-            // ------------------------------------------------ MMA issuer
-            constexpr uint32_t idesc = idesc_i8(128, TOK, true, true);
-            UnitCursor<KB> cur;
-            cur.init(b0, b1, KT, p.NT);
-            int s = 0, seg = 0, unit = 0;
-            uint32_t ph = 0;
-            bool ok = true;
-            while (ok && !cur.done()) {
-                const int buf = seg % C::kAccBufs;
-                const uint32_t aph = (uint32_t)(seg / C::kAccBufs) & 1u;
-                ok = __all_sync(0xffffffffu, wait_bounded(&ctl->acc_empty[buf], aph ^ 1u, wd, kSiteMmaAccEmpty, seg));
-                if (!ok) break;
-                tc_fence_after();
-                const uint32_t d_tmem = tmem_base + (uint32_t)(buf * TOK);
-                bool first = true, seg_done = false;
-                while (!seg_done) {
-                    // The token tile (shared memory) and the dequantised weights
-                    // (TMEM) of this unit.
-                    ok = __all_sync(0xffffffffu,
-                                    wait_bounded(&ctl->full[s], ph, wd, kSiteMmaOperands, 2 * unit) &&
-                                        wait_bounded(&ctl->a_full[s], ph, wd, kSiteMmaOperands, 2 * unit + 1));
-                    if (!ok) break;
-                    tc_fence_after();
-                    if (lane == 0) {
-                        const uint32_t a_tmem = tmem_base + (uint32_t)(C::kACol0 + s * KB * 32);
-                        const uint32_t xaddr = smem_u32(stage_x(s));
-                        for (int j = 0; j < cur.nk; ++j) {
-                            const uint64_t bdesc = smem_desc_k_sw128(xaddr + j * C::kXTile);
-#pragma unroll
-                            for (int q = 0; q < 4; ++q)   // 4 x K=32 per 128-wide k-tile
-                                mma_i8_ts(d_tmem, a_tmem + (uint32_t)(j * 32 + q * 8), bdesc + (uint64_t)(q * 2),
-                                          idesc, (first && j == 0 && q == 0) ? 0u : 1u);
-                        }
-                        tc_commit(&ctl->freed[s]);
-                    }
-                    __syncwarp();
-                    first = false;
-                    ++unit;
-                    if (++s == S) {
-                        s = 0;
-                        ph ^= 1u;
-                    }
-                    seg_done = cur.advance();
-                }
-                if (!ok) break;
-                if (lane == 0) tc_commit(&ctl->acc_full[buf]);
-                __syncwarp();
-                ++seg;
-            }
-            // Every MMA must have completed before tensor memory is freed.
+        } else if (warp == kWarpMma || warp == kWarpMma + 1) {
+            // ------------------------------------------------ MMA issuers
+            // Lane 0 of each issuer warp runs the role. A thread's mbarrier
+            // waits stall its own queued tensor-core work, so two issuers that
+            // take turns keep the tensor core busy through each other's waits.
+            // Two-k-tile units: issuer k takes the units of parity k (with an
+            // even stage count always the same stages, whose every phase it
+            // waits on) into its own accumulator and commits their freed[s].
+            // One-k-tile units: both issuers take every unit, each half of the
+            // token columns, and both commit freed[s]. Both commit acc_full.
+            const int k = warp - kWarpMma;
             if (lane == 0) {
-                tc_commit(&ctl->final_bar);
-                wait_drain(&ctl->final_bar, 0, kDrainNs);
+                constexpr uint32_t idesc = idesc_i8(128, KB == 2 ? TOK : TOK / 2, true, true);
+                UnitCursor<KB> cur;
+                cur.init(b0, b1, KT, p.NT);
+                int s = 0, seg = 0, unit = 0;
+                uint32_t ph = 0;
+                bool ok = true;
+                while (ok && !cur.done()) {
+                    const int buf = seg % C::kAccBufs;
+                    const uint32_t aph = (uint32_t)(seg / C::kAccBufs) & 1u;
+                    ok = wait_bounded(&ctl->acc_empty[buf], aph ^ 1u, wd, kSiteMmaAccEmpty, seg);
+                    if (!ok) break;
+                    const uint32_t d_tmem = tmem_base + (uint32_t)(buf * C::kAccCols + k * (KB == 2 ? TOK : TOK / 2));
+                    uint32_t acc = 0u;   // this issuer's first MMA of the segment overwrites its accumulator
+                    bool seg_done = false;
+                    while (!seg_done) {
+                        if (KB == 1 || (unit & 1) == k) {
+                            // The token tile (shared memory) and the
+                            // dequantised weights (TMEM) of this unit.
+                            ok = wait_bounded(&ctl->full[s], ph, wd, kSiteMmaOperands, 2 * unit) &&
+                                 wait_bounded(&ctl->a_full[s], ph, wd, kSiteMmaOperands, 2 * unit + 1);
+                            if (!ok) break;
+                            tc_fence_after();
+                            const uint32_t a_tmem = tmem_base + (uint32_t)(C::kACol0 + s * KB * 32);
+                            const uint64_t bdesc = smem_desc_k_sw128(smem_u32(stage_x(s)));
+                            if (KB == 2) {
+                                mma4_i8_ts(d_tmem, a_tmem, bdesc, idesc, acc);
+                                if (cur.nk == 2)
+                                    mma4_i8_ts(d_tmem, a_tmem + 32u, bdesc + (uint64_t)(C::kXTile >> 4), idesc, 1u);
+                            } else {
+                                // token rows k*TOK/2 .. of the tile: (TOK/2) x 128 bytes further on
+                                mma4_i8_ts(d_tmem, a_tmem, bdesc + (uint64_t)(k * (TOK / 2) * 128 / 16), idesc, acc);
+                            }
+                            acc = 1u;
+                            tc_commit(&ctl->freed[s]);
+                        }
+                        ++unit;
+                        if (++s == S) {
+                            s = 0;
+                            ph ^= 1u;
+                        }
+                        seg_done = cur.advance();
+                    }
+                    if (!ok) break;
+                    tc_commit(&ctl->acc_full[buf]);
+                    ++seg;
+                }
+                // Every MMA must have completed before tensor memory is freed.
+                tc_commit(&ctl->final_bar[k]);
+                wait_drain(&ctl->final_bar[k], 0, kDrainNs);
             }
             __syncwarp();
         } else if (warp >= kWarpDequant0 && warp < kWarpEpilogue) {
             // ------------------------------------------------ dequant
-            // Both warpgroups work on every unit: warpgroup h decodes code
-            // chunks 2h, 2h+1 of each row (k 64h .. 64h+63 of the k-tile, TMEM
-            // columns 16h .. 16h+15). Every waiter thus sees every phase of
-            // every stage barrier, so parity waits cannot alias for any stage
-            // count.
-            const int h = (warp - kWarpDequant0) >> 2;
+            // Warpgroup g takes the units i with i % 2 == g, i.e. (the stage
+            // count being even) always the same stages: it waits on every phase
+            // of those stage barriers and on no others, so parity waits cannot
+            // alias. Thread (quarter, lane) decodes weight row r of each k-tile.
+            const int g = (warp - kWarpDequant0) >> 2;
             const int quarter = warp & 3;                    // TMEM lanes 32q .. 32q+31
             const int r = quarter * 32 + lane;               // weight row in the tile
             const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
@@ -395,48 +420,63 @@ __global__ void __launch_bounds__(kThreads, 1)
             int s = 0;
             uint32_t ph = 0;
             for (int i = 0; !cur.done(); ++i, cur.advance()) {
-                // full[s] for this unit implies the producer saw freed[s] for
-                // the unit S earlier, i.e. TMEM A buffer s is no longer read.
-                const bool ok = __all_sync(0xffffffffu, wait_bounded(&ctl->full[s], ph, wd, kSiteDequantFull, i));
-                if (!ok) break;
-                tc_fence_after();   // the TMEM writes below come after the wait (and the MMA reads it implies)
-                const uint32_t a_col = tmem_base + lane_addr + (uint32_t)(C::kACol0 + s * KB * 32 + 16 * h);
-                for (int j = 0; j < cur.nk; ++j) {
-                    const uint32_t wbase = smem_u32(stage_w(s) + j * C::kWTile);
-                    uint32_t sc = 0u, c4 = 0u;
-                    if (MODE == 0) {
-                        const uint32_t sz = lds16(wbase + 8192 + 2 * r);
-                        sc = sz & 0xFFu;
-                        c4 = (uint32_t)(128 - (int)(int8_t)(sz >> 8)) * 0x01010101u;
-                    }
-                    uint32_t o[16];
-#pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        const uint4 v = lds128(wbase + (2 * h + c) * 2048 + r * 16);
-                        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const uint32_t lo = w[q] & 0x0F0F0F0Fu;
-                            const uint32_t hi = (w[q] >> 4) & 0x0F0F0F0Fu;
-                            if (MODE == 0) {
-                                o[8 * c + 2 * q] = (lo * sc + c4) ^ 0x80808080u;
-                                o[8 * c + 2 * q + 1] = (hi * sc + c4) ^ 0x80808080u;
-                            } else {
-                                o[8 * c + 2 * q] = lo;
-                                o[8 * c + 2 * q + 1] = hi;
-                            }
-                        }
-                    }
-                    tmem_st16_wait(a_col + (uint32_t)(j * 32), o);
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&ctl->a_full[s]);
-                __syncwarp();
+                const int unit_s = s;
+                const uint32_t unit_ph = ph;
                 if (++s == S) {
                     s = 0;
                     ph ^= 1u;
                 }
+                if ((i & 1) != g) continue;
+                // full[s] for this unit implies the producer saw freed[s] for
+                // the unit S earlier, i.e. TMEM A buffer s is no longer read.
+                const bool ok = __all_sync(0xffffffffu, wait_bounded(&ctl->full[unit_s], unit_ph, wd, kSiteDequantFull, i));
+                if (!ok) break;
+                tc_fence_after();   // the TMEM writes below come after the wait (and the MMA reads it implies)
+                const uint32_t a_col = tmem_base + lane_addr + (uint32_t)(C::kACol0 + unit_s * KB * 32);
+                const int nk = cur.nk;
+                // All shared-memory loads of the unit first (four 16-byte code
+                // chunks and the (s, z*s) pair per k-tile), then per k-tile the
+                // decode and one 32-column TMEM store.
+                uint4 v[KB][4];
+                uint32_t sz[KB];
+#pragma unroll
+                for (int j = 0; j < KB; ++j) {
+                    if (j < nk) {
+                        const uint32_t wbase = smem_u32(stage_w(unit_s) + j * C::kWTile);
+                        sz[j] = MODE == 0 ? lds16(wbase + 8192 + 2 * r) : 0u;
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) v[j][c] = lds128(wbase + c * 2048 + r * 16);
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < KB; ++j) {
+                    if (j < nk) {
+                        const uint32_t sc = sz[j] & 0xFFu;
+                        const uint32_t c4 = (uint32_t)(128 - (int)(int8_t)(sz[j] >> 8)) * 0x01010101u;
+                        uint32_t o[32];
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            const uint32_t w[4] = {v[j][c].x, v[j][c].y, v[j][c].z, v[j][c].w};
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                const uint32_t lo = w[q] & 0x0F0F0F0Fu;
+                                const uint32_t hi = (w[q] >> 4) & 0x0F0F0F0Fu;
+                                if (MODE == 0) {
+                                    o[8 * c + 2 * q] = (lo * sc + c4) ^ 0x80808080u;
+                                    o[8 * c + 2 * q + 1] = (hi * sc + c4) ^ 0x80808080u;
+                                } else {
+                                    o[8 * c + 2 * q] = lo;
+                                    o[8 * c + 2 * q + 1] = hi;
+                                }
+                            }
+                        }
+                        tmem_st32_wait(a_col + (uint32_t)(j * 32), o);
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ctl->a_full[unit_s]);
+                __syncwarp();
             }
         } else if (warp >= kWarpEpilogue) {
             // ------------------------------------------------ epilogue
@@ -447,30 +487,58 @@ __global__ void __launch_bounds__(kThreads, 1)
             griddep_wait();   // outputs, scales, row sums and workspace belong to the previous kernel until now
             UnitCursor<KB> cur;
             cur.init(b0, b1, KT, p.NT);
-            int seg = 0;
+            int seg = 0, ubase = 0;
             while (!cur.done()) {
                 const uint32_t seg_b = cur.b, seg_e = cur.seg_end;
                 const int kt_lo = cur.kt, kt_hi = cur.kt + (int)(seg_e - seg_b);
                 const int mt = cur.mt, nt = cur.nt;
                 const uint32_t tile_b = seg_b - (uint32_t)kt_lo;
-                while (!cur.advance()) {
-                }
+                int nunits = 1;
+                while (!cur.advance()) ++nunits;
+                // Two-k-tile units: the segment's first unit went to issuer
+                // (ubase & 1), whose accumulator is `prim`; the other issuer's
+                // (`second`) holds data only if the segment has two units or more.
+                const int prim = KB == 2 ? (ubase & 1) : 0;
+                ubase += nunits;
                 const int buf = seg % C::kAccBufs;
                 const uint32_t aph = (uint32_t)(seg / C::kAccBufs) & 1u;
+                const int n = nt * kTileN + r;
+                const int64_t m0 = (int64_t)mt * TOK;
+                const bool two = KB == 2 && nunits >= 2;
+                // Owner (or sole computer) of a tile: the CTA holding its first
+                // k-tile. Contributors c_first .. c_last (none if c_last < c_first).
+                const bool owner = kt_lo == 0;
+                const uint32_t c_first = blockIdx.x + 1;
+                const uint32_t c_last =
+                    (!owner || kt_hi == KT) ? blockIdx.x : cta_of(tile_b + (uint32_t)KT - 1, B, G);
+                constexpr int CO = 16;   // owner: token columns per step
+                if (c_last >= c_first) {
+                    // Contributors reach their share of the tile first, so their
+                    // flags are usually up before this CTA's own accumulator is:
+                    // poll them now (lanes of the first epilogue warp in
+                    // parallel, acquire loads). The barrier orders everyone's
+                    // partial-sum reads after the polls.
+                    bool got = true;
+                    if (warp == kWarpEpilogue) {
+                        for (uint32_t c = c_first + (uint32_t)lane; c <= c_last && got; c += 32)
+                            got = wait_flag_bounded(p.flags + c, wd, (int)c);
+                        got = __all_sync(0xffffffffu, got);
+                    }
+                    if (named_bar_any(1, 128, !got)) break;
+                }
                 // Every lane spins on its own; the vote reconverges the warp
                 // before the named barrier, and all four epilogue warps leave
                 // together (the shared-tile paths below meet at named barriers).
                 const bool ok = __all_sync(0xffffffffu, wait_bounded(&ctl->acc_full[buf], aph, wd, kSiteEpilogueAcc, seg));
                 if (named_bar_any(1, 128, !ok)) break;
                 tc_fence_after();
-                const int n = nt * kTileN + r;
-                const int64_t m0 = (int64_t)mt * TOK;
                 const float col_scale = __half2float(reinterpret_cast<const __half *>(p.blob + p.off_scale)[n]);
                 int col_zero = 0;
                 if (MODE == 1)
                     col_zero = __half2int_rn(reinterpret_cast<const __half *>(p.blob + p.off_zero)[n]);
-                const uint32_t acc_addr = tmem_base + lane_addr + (uint32_t)(buf * TOK);
-                if (kt_lo > 0) {
+                const uint32_t acc_addr = tmem_base + lane_addr + (uint32_t)(buf * C::kAccCols + prim * TOK);
+                const uint32_t acc2_addr = tmem_base + lane_addr + (uint32_t)(buf * C::kAccCols + (prim ^ 1) * TOK);
+                if (!owner) {
                     // Contributor: this tile's first k-tile belongs to an earlier
                     // CTA. Store the partial sums in this CTA's slot, raise its flag.
                     int32_t *part = p.partials + (long long)blockIdx.x * TOK * kTileN;
@@ -478,37 +546,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int c0 = 0; c0 < TOK; c0 += CH) {
                         uint32_t v[CH];
                         tmem_load<CH>(acc_addr + (uint32_t)c0, v);
+                        if (two) add_second<CH>(acc2_addr + (uint32_t)c0, v);
 #pragma unroll
                         for (int j = 0; j < CH; ++j) part[(c0 + j) * kTileN + r] = (int32_t)v[j];
                     }
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&ctl->acc_empty[buf]);
-                    __threadfence();
+                    // The barrier orders every thread's partial-sum stores
+                    // before the leader's release store of the flag (release is
+                    // cumulative), so the owner's acquire load sees them all.
                     named_bar_sync(1, 128);
                     if (leader) st_release_gpu(p.flags + blockIdx.x, 1);
                     __syncwarp();
                 } else {
-                    // Owner (or sole computer) of the tile: add the contributors'
-                    // partial sums, run the epilogue, clear their flags.
-                    const uint32_t c_first = blockIdx.x + 1;
-                    const uint32_t c_last = (kt_hi == KT) ? blockIdx.x : cta_of(tile_b + (uint32_t)KT - 1, B, G);
-                    if (c_last >= c_first) {
-                        bool got = true;
-                        if (leader)
-                            for (uint32_t c = c_first; c <= c_last && got; ++c)
-                                got = wait_flag_bounded(p.flags + c, wd, (int)c);
-                        __syncwarp();
-                        if (named_bar_any(1, 128, !got)) break;
-                        __threadfence();
-                    }
-                    // 16 token columns at a time; the partial sums of up to four
-                    // contributors are loaded together (one L2 round trip).
-                    constexpr int CO = 16;
+                    // Owner: add the contributors' partial sums (loaded four
+                    // contributors at a time, one L2 round trip), run the
+                    // epilogue, clear their flags.
 #pragma unroll 1
                     for (int c0 = 0; c0 < TOK; c0 += CO) {
                         uint32_t v[CO];
                         tmem_load<CO>(acc_addr + (uint32_t)c0, v);
+                        if (two) add_second<CO>(acc2_addr + (uint32_t)c0, v);
                         if (c0 + CO >= TOK) {
                             tc_fence_before();
                             __syncwarp();
@@ -521,8 +580,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             for (int cc = 0; cc < 4; ++cc) {
                                 const int32_t *part = p.partials + (long long)(c + cc) * TOK * kTileN + c0 * kTileN + r;
 #pragma unroll
-                                for (int j = 0; j < CO; ++j)
-                                    t[cc][j] = (c + cc <= c_last) ? ld_cg_s32(part + j * kTileN) : 0;
+                                for (int j = 0; j < CO; ++j) t[cc][j] = (c + cc <= c_last) ? ld_cg_s32(part + j * kTileN) : 0;
                             }
 #pragma unroll
                             for (int cc = 0; cc < 4; ++cc)
@@ -533,8 +591,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     if (c_last >= c_first) {
                         named_bar_sync(1, 128);
-                        if (leader)
-                            for (uint32_t c = c_first; c <= c_last; ++c) p.flags[c] = 0;
+                        if (warp == kWarpEpilogue)
+                            for (uint32_t c = c_first + (uint32_t)lane; c <= c_last; c += 32) p.flags[c] = 0;
                         __syncwarp();
                     }
                 }

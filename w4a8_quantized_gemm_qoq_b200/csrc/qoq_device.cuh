@@ -189,14 +189,22 @@ __device__ __forceinline__ void tc_commit(uint64_t *bar) {
                  : "memory");
 }
 
-// D[tmem] (+)= A[tmem] . B[smem]^T, kind::i8, INT32 accumulate.
-__device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                          uint32_t accumulate) {
+// One 128-wide k-tile: four tcgen05.mma (K = 32 each) issued back to back,
+// D[tmem] (+)= A[tmem] . B[smem]^T, kind::i8, INT32 accumulate. A columns
+// a .. a+31 (8 per MMA); the B descriptor advances 32 bytes (2 units of 16 B)
+// per MMA inside the 128-byte swizzle row. `accumulate` applies to the first
+// MMA only; the other three always accumulate.
+__device__ __forceinline__ void mma4_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%5], %6, %3, 1;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%7], %8, %3, 1;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%9], %10, %3, 1;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(a_tmem + 8u), "l"(b_desc + 2ull),
+        "r"(a_tmem + 16u), "l"(b_desc + 4ull), "r"(a_tmem + 24u), "l"(b_desc + 6ull)
         : "memory");
 }
 
@@ -219,20 +227,6 @@ __device__ __forceinline__ uint64_t smem_desc_k_sw128(uint32_t saddr) {
     d |= static_cast<uint64_t>(1) << 46;                   // descriptor version (sm_100)
     d |= static_cast<uint64_t>(2) << 61;                   // SWIZZLE_128B
     return d;
-}
-
-// 32 lanes x 16 columns of 32-bit values: thread t <-> lane base+t. The
-// store and its completion wait are one asm block so the source registers
-// are never reused early.
-__device__ __forceinline__ void tmem_st16_wait(uint32_t taddr, const uint32_t (&r)[16]) {
-    __syncwarp();   // warp-collective (.sync.aligned)
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
-        "%13, %14, %15, %16};\n\t"
-        "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-        : "memory");
 }
 
 // Load + wait in one asm block so no use of the destination registers can be
@@ -262,6 +256,21 @@ __device__ __forceinline__ void tmem_ld16_wait(uint32_t taddr, uint32_t (&r)[16]
           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
           "=r"(r[15])
         : "r"(taddr)
+        : "memory");
+}
+
+// 32 lanes x 32 columns store and its completion wait in one asm block, so
+// the source registers are never reused early.
+__device__ __forceinline__ void tmem_st32_wait(uint32_t taddr, const uint32_t (&r)[32]) {
+    __syncwarp();   // warp-collective (.sync.aligned)
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
+        "%13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};\n\t"
+        "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+        "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+        "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
         : "memory");
 }
 
