@@ -176,10 +176,11 @@ struct UnitCursor {
     }
 };
 
-// Epilogue for CH consecutive tokens (m_first ..) of weight row n.
+// Epilogue for CH consecutive tokens (m_first ..) of weight row n. sx[j] is
+// FP32(s_x[m_first + j]) (the value for tokens past M is unused).
 template <int CH, int MODE>
 __device__ __forceinline__ void store_outputs(const GemmParams &p, const uint32_t (&v)[CH], int64_t m_first,
-                                              int n, float col_scale, int col_zero) {
+                                              int n, float col_scale, int col_zero, const float (&sx)[CH]) {
     const int64_t N = p.N;
 #pragma unroll
     for (int j = 0; j < CH; ++j) {
@@ -188,13 +189,22 @@ __device__ __forceinline__ void store_outputs(const GemmParams &p, const uint32_
             int32_t acc = (int32_t)v[j];
             if (MODE == 1) acc -= col_zero * p.rowsum[m];
             if (p.fp16_out) {
-                const float sx = __half2float(p.s_x[m]);
-                const float y = __fmul_rn(__int2float_rn(acc), __fmul_rn(sx, col_scale));
+                const float y = __fmul_rn(__int2float_rn(acc), __fmul_rn(sx[j], col_scale));
                 static_cast<__half *>(p.out)[m * N + n] = __float2half_rn(y);
             } else {
                 static_cast<int32_t *>(p.out)[m * N + n] = acc;
             }
         }
+    }
+}
+
+// FP32 token scales of CH tokens from m_first (tokens past M repeat the last).
+template <int CH>
+__device__ __forceinline__ void load_token_scales(const GemmParams &p, int64_t m_first, float (&sx)[CH]) {
+#pragma unroll
+    for (int j = 0; j < CH; ++j) {
+        const int64_t m = m_first + j < p.M ? m_first + j : p.M - 1;
+        sx[j] = p.fp16_out ? __half2float(p.s_x[m]) : 0.0f;
     }
 }
 
@@ -250,9 +260,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         // No kernel that releases its dependents early (this GEMM, the
         // activation quantiser) writes a blob, so the blob may be read before
         // griddepcontrol.wait; read at L2, as the TMA weight copies are.
+        // The five words are loaded together (one round trip), then compared.
         const int32_t *h = reinterpret_cast<const int32_t *>(p.blob);
-        if ((uint32_t)ld_cg_s32(h) != kMagic || (uint32_t)ld_cg_s32(h + 1) != kVersion ||
-            ld_cg_s32(h + 2) != p.N || ld_cg_s32(h + 3) != p.K || ld_cg_s32(h + 4) != p.group)
+        const int32_t h0 = ld_cg_s32(h), h1 = ld_cg_s32(h + 1), h2 = ld_cg_s32(h + 2), h3 = ld_cg_s32(h + 3),
+                      h4 = ld_cg_s32(h + 4);
+        if ((uint32_t)h0 != kMagic || (uint32_t)h1 != kVersion || h2 != p.N || h3 != p.K || h4 != p.group)
             ctl->abort_flag = 1;   // reported on the status word after griddepcontrol.wait
     }
     if (warp == kWarpProducer && lane == 0) prefetch_tensormap(&tmap_x);
@@ -526,16 +538,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     if (named_bar_any(1, 128, !got)) break;
                 }
+                // Inputs of the first output step that do not depend on the
+                // accumulator are fetched before waiting for it.
+                const float col_scale = __half2float(reinterpret_cast<const __half *>(p.blob + p.off_scale)[n]);
+                int col_zero = 0;
+                if (MODE == 1)
+                    col_zero = __half2int_rn(reinterpret_cast<const __half *>(p.blob + p.off_zero)[n]);
+                float sx0[CO];
+                if (owner) load_token_scales<CO>(p, m0, sx0);
                 // Every lane spins on its own; the vote reconverges the warp
                 // before the named barrier, and all four epilogue warps leave
                 // together (the shared-tile paths below meet at named barriers).
                 const bool ok = __all_sync(0xffffffffu, wait_bounded(&ctl->acc_full[buf], aph, wd, kSiteEpilogueAcc, seg));
                 if (named_bar_any(1, 128, !ok)) break;
                 tc_fence_after();
-                const float col_scale = __half2float(reinterpret_cast<const __half *>(p.blob + p.off_scale)[n]);
-                int col_zero = 0;
-                if (MODE == 1)
-                    col_zero = __half2int_rn(reinterpret_cast<const __half *>(p.blob + p.off_zero)[n]);
                 const uint32_t acc_addr = tmem_base + lane_addr + (uint32_t)(buf * C::kAccCols + prim * TOK);
                 const uint32_t acc2_addr = tmem_base + lane_addr + (uint32_t)(buf * C::kAccCols + (prim ^ 1) * TOK);
                 if (!owner) {
@@ -587,7 +603,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                                 for (int j = 0; j < CO; ++j) v[j] = (uint32_t)((int32_t)v[j] + t[cc][j]);
                         }
-                        store_outputs<CO, MODE>(p, v, m0 + c0, n, col_scale, col_zero);
+                        if (c0 == 0) {
+                            store_outputs<CO, MODE>(p, v, m0, n, col_scale, col_zero, sx0);
+                        } else {
+                            float sx[CO];
+                            load_token_scales<CO>(p, m0 + c0, sx);
+                            store_outputs<CO, MODE>(p, v, m0 + c0, n, col_scale, col_zero, sx);
+                        }
                     }
                     if (c_last >= c_first) {
                         named_bar_sync(1, 128);
