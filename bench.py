@@ -393,6 +393,39 @@ def run_gpu(args, rank, world, local_rank):
     return res
 
 
+def run_shape(args):
+    """One M x N x K GEMM alone: weights packed and activations quantised
+    once, then `steps` launches of qoq_gemm_fp16_out back to back (after
+    `warmup` launches) between CUDA events. Two weight copies alternate when
+    one copy fits in L2."""
+    import torch
+    from w4a8_quantized_gemm_qoq_b200 import build as qbuild, qoq
+    qbuild.build()
+    M, N, K = (int(v) for v in args.shape.lower().split("x"))
+    dev = torch.device("cuda", 0)
+    W = torch.from_numpy(inputs.make_weights(N, K, seed=1)).to(dev)
+    blob = qoq.quantize_weights(W, GROUP)
+    del W
+    blobs = [blob] if blob.numel() > 130e6 else [blob, blob.clone()]
+    X = torch.from_numpy(inputs.make_activations(M, K, seed=1)).to(dev)
+    X8, s_x, rs = qoq.quantize_act_per_token(X)
+    ws = qoq.Workspace.for_shape(M, N, K, GROUP, dev)
+    Y = torch.empty((M, N), dtype=torch.float16, device=dev)
+    for i in range(max(1, args.warmup)):
+        qoq.gemm_fp16_out(X8, s_x, blobs[i % len(blobs)], N, K, GROUP, rowsum=rs, ws=ws, Y=Y)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(args.steps):
+        qoq.gemm_fp16_out(X8, s_x, blobs[i % len(blobs)], N, K, GROUP, rowsum=rs, ws=ws, Y=Y)
+    e1.record()
+    torch.cuda.synchronize()
+    assert ws.status() == 0, "device status %d" % ws.status()
+    us = 1000.0 * e0.elapsed_time(e1) / args.steps
+    return {"shape": [M, N, K], "launches": args.steps, "us_per_launch": round(us, 3),
+            "GBps": round(gemm_bytes(M, N, K) / us / 1e3, 1), "TOPS": round(gemm_ops(M, N, K) / us / 1e6, 2)}
+
+
 def run_e2e(args, probs, qoq, stream):
     """Same metric through the public API with host buffers: every step copies
     each problem's FP16 activations host->device (pinned), runs the two calls,
@@ -499,6 +532,9 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shape", default=None,
+                    help="MxNxK: one GEMM shape alone (act quant once, then --steps GEMM launches back to back); "
+                         "small footprint for profiling")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -508,6 +544,9 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args)))
+        return
+    if args.shape:
+        print(json.dumps(run_shape(args)))
         return
 
     if world > 1:
