@@ -66,7 +66,7 @@ inline int token_tile_for(int64_t M, int64_t N, int64_t K) {
     if (M <= 32) return 32;
     if (M <= 64) return blocks(64) >= 2500 ? 64 : 32;
     if (M <= 128) return 64;
-    if (M <= 256) return blocks(128) >= 7000 ? 128 : 64;
+    if (M <= 256) return blocks(128) >= 10000 ? 128 : 64;
     if (M <= 512) return 128;
     return KT >= 64 ? 256 : 128;
 }
