@@ -60,11 +60,10 @@ constexpr uint64_t kDrainNs = 100ull * 1000ull * 1000ull;   // 100 ms
 
 template <int TOK, int MODE>
 struct GemmCfg {
-    // KB = k-tiles per pipeline unit: two for decode-sized token tiles (halves
-    // the barrier and issue work per weight byte), one for wide token tiles
-    // (their MMA work per k-tile already hides it, and shared memory holds
-    // fewer wide stages).
-    static constexpr int kKB = TOK <= 64 ? 2 : 1;
+    // KB = k-tiles per pipeline unit: two up to 128-token tiles (halves the
+    // barrier and issue work per weight byte), one for 256-token tiles
+    // (shared memory holds only two two-k-tile stages of those).
+    static constexpr int kKB = TOK <= 128 ? 2 : 1;
     static constexpr int kXTile = TOK * 128;                    // token tile, 128 k
     static constexpr int kWTile = MODE == 0 ? 8448 : 8192;      // codes (+ s, z*s) per k-tile
     static constexpr int kXBytes = kKB * kXTile;
@@ -72,11 +71,13 @@ struct GemmCfg {
     static constexpr int kStageBytes = (kXBytes + kWBytes + 1023) / 1024 * 1024;
     static constexpr int kSmemLimit = 232448;                   // 227 KB per CTA
     static constexpr int kReserve = 2048;                       // alignment slack + barriers
-    // Two MMA issuers. With two-k-tile units, issuer j takes the units of
-    // index parity j (those its dequant warpgroup serves) into its own
-    // accumulator, and the epilogue adds the two; with one-k-tile units, issuer
-    // j takes token columns j*TOK/2 .. of every unit.
-    static constexpr int kAccCols = kKB == 2 ? 2 * TOK : TOK;   // TMEM columns per accumulator buffer
+    // Two MMA issuers. Up to 64-token tiles (kAlt), issuer j takes the units
+    // of index parity j (those its dequant warpgroup serves) into its own
+    // accumulator, and the epilogue adds the two; wider tiles have no TMEM for
+    // a second accumulator, and issuer j takes token columns j*TOK/2 .. of
+    // every unit.
+    static constexpr bool kAlt = TOK <= 64;
+    static constexpr int kAccCols = kAlt ? 2 * TOK : TOK;   // TMEM columns per accumulator buffer
     static constexpr int kAccBufs = (TOK == 64 || TOK == 256) ? 1 : 2;
     static constexpr int kACol0 = kAccBufs * kAccCols;
     // One CTA per SM (shared memory use guarantees it), so the CTA takes all
@@ -232,7 +233,7 @@ template <int TOK, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     qoq_gemm_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ CUtensorMap tmap_x) {
     using C = GemmCfg<TOK, MODE>;
-    constexpr int CH = (TOK < 32 || C::kKB == 2) ? 16 : 32;   // epilogue TMEM chunk (16 when two accumulators are summed)
+    constexpr int CH = (TOK < 32 || C::kAlt) ? 16 : 32;   // epilogue TMEM chunk (16 when two accumulators are summed)
     constexpr int S = C::kStages;
     constexpr int KB = C::kKB;
     extern __shared__ uint8_t smem_raw[];
@@ -247,7 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ctl->abort_flag = 0;
         for (int s = 0; s < S; ++s) {
             mbar_init(&ctl->full[s], 1);
-            mbar_init(&ctl->freed[s], C::kKB == 2 ? 1 : kIssuers);
+            mbar_init(&ctl->freed[s], C::kAlt ? 1 : kIssuers);
             mbar_init(&ctl->a_full[s], 4);   // the four warps of one dequant warpgroup
         }
         for (int b = 0; b < 2; ++b) {
@@ -359,14 +360,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             // Lane 0 of each issuer warp runs the role. A thread's mbarrier
             // waits stall its own queued tensor-core work, so two issuers that
             // take turns keep the tensor core busy through each other's waits.
-            // Two-k-tile units: issuer k takes the units of parity k (with an
-            // even stage count always the same stages, whose every phase it
+            // Up to 64-token tiles: issuer k takes the units of parity k (with
+            // an even stage count always the same stages, whose every phase it
             // waits on) into its own accumulator and commits their freed[s].
-            // One-k-tile units: both issuers take every unit, each half of the
+            // Wider tiles: both issuers take every unit, each half of the
             // token columns, and both commit freed[s]. Both commit acc_full.
             const int k = warp - kWarpMma;
             if (lane == 0) {
-                constexpr uint32_t idesc = idesc_i8(128, KB == 2 ? TOK : TOK / 2, true, true);
+                constexpr bool ALT = C::kAlt;
+                constexpr uint32_t idesc = idesc_i8(128, ALT ? TOK : TOK / 2, true, true);
                 UnitCursor<KB> cur;
                 cur.init(b0, b1, KT, p.NT);
                 int s = 0, seg = 0, unit = 0;
@@ -377,11 +379,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t aph = (uint32_t)(seg / C::kAccBufs) & 1u;
                     ok = wait_bounded(&ctl->acc_empty[buf], aph ^ 1u, wd, kSiteMmaAccEmpty, seg);
                     if (!ok) break;
-                    const uint32_t d_tmem = tmem_base + (uint32_t)(buf * C::kAccCols + k * (KB == 2 ? TOK : TOK / 2));
+                    const uint32_t d_tmem = tmem_base + (uint32_t)(buf * C::kAccCols + k * (ALT ? TOK : TOK / 2));
                     uint32_t acc = 0u;   // this issuer's first MMA of the segment overwrites its accumulator
                     bool seg_done = false;
                     while (!seg_done) {
-                        if (KB == 1 || (unit & 1) == k) {
+                        if (!ALT || (unit & 1) == k) {
                             // The token tile (shared memory) and the
                             // dequantised weights (TMEM) of this unit.
                             ok = wait_bounded(&ctl->full[s], ph, wd, kSiteMmaOperands, 2 * unit) &&
@@ -390,14 +392,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tc_fence_after();
                             const uint32_t a_tmem = tmem_base + (uint32_t)(C::kACol0 + s * KB * 32);
                             const uint64_t bdesc = smem_desc_k_sw128(smem_u32(stage_x(s)));
-                            if (KB == 2) {
-                                mma4_i8_ts(d_tmem, a_tmem, bdesc, idesc, acc);
-                                if (cur.nk == 2)
-                                    mma4_i8_ts(d_tmem, a_tmem + 32u, bdesc + (uint64_t)(C::kXTile >> 4), idesc, 1u);
-                            } else {
-                                // token rows k*TOK/2 .. of the tile: (TOK/2) x 128 bytes further on
-                                mma4_i8_ts(d_tmem, a_tmem, bdesc + (uint64_t)(k * (TOK / 2) * 128 / 16), idesc, acc);
-                            }
+                            // Per k-tile j of the unit: four MMAs; the token
+                            // tile of k-tile j lies kXTile bytes further on,
+                            // and (N split) issuer k's token rows k*TOK/2 ..
+                            // another (TOK/2) x 128 bytes on.
+                            const uint64_t bk = bdesc + (uint64_t)(ALT ? 0 : k * (TOK / 2) * 128 / 16);
+                            mma4_i8_ts(d_tmem, a_tmem, bk, idesc, acc);
+                            if (KB == 2 && cur.nk == 2)
+                                mma4_i8_ts(d_tmem, a_tmem + 32u, bk + (uint64_t)(C::kXTile >> 4), idesc, 1u);
                             acc = 1u;
                             tc_commit(&ctl->freed[s]);
                         }
@@ -507,16 +509,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t tile_b = seg_b - (uint32_t)kt_lo;
                 int nunits = 1;
                 while (!cur.advance()) ++nunits;
-                // Two-k-tile units: the segment's first unit went to issuer
+                // Up to 64-token tiles: the segment's first unit went to issuer
                 // (ubase & 1), whose accumulator is `prim`; the other issuer's
                 // (`second`) holds data only if the segment has two units or more.
-                const int prim = KB == 2 ? (ubase & 1) : 0;
+                const int prim = C::kAlt ? (ubase & 1) : 0;
                 ubase += nunits;
                 const int buf = seg % C::kAccBufs;
                 const uint32_t aph = (uint32_t)(seg / C::kAccBufs) & 1u;
                 const int n = nt * kTileN + r;
                 const int64_t m0 = (int64_t)mt * TOK;
-                const bool two = KB == 2 && nunits >= 2;
+                const bool two = C::kAlt && nunits >= 2;
                 // Owner (or sole computer) of a tile: the CTA holding its first
                 // k-tile. Contributors c_first .. c_last (none if c_last < c_first).
                 const bool owner = kt_lo == 0;
