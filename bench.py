@@ -374,6 +374,7 @@ def run_gpu(args, rank, world, local_rank):
                     "timing": timing}
 
     e2e = run_e2e(args, probs, qoq, stream) if rank == 0 else None
+    w8a8 = run_w8a8(probs, stream, gemm_only_us, max(K, 10)) if rank == 0 else None
     res = {
         "metric": METRIC, "value": round(world * ops_step / (step_ms * 1e-3) / 1e12, 3), "unit": "TOPS",
         "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup),
@@ -389,6 +390,7 @@ def run_gpu(args, rank, world, local_rank):
         "clocks": clk.summary(),
         "e2e": e2e,
         "per_gemm": per,
+        "w8a8_context": w8a8,
     }
     return res
 
@@ -424,6 +426,52 @@ def run_shape(args):
     us = 1000.0 * e0.elapsed_time(e1) / args.steps
     return {"shape": [M, N, K], "launches": args.steps, "us_per_launch": round(us, 3),
             "GBps": round(gemm_bytes(M, N, K) / us / 1e3, 1), "TOPS": round(gemm_ops(M, N, K) / us / 1e6, 2)}
+
+
+def run_w8a8(probs, stream, w4a8_us, reps):
+    """Context, not the product: the same GEMM shapes as a W8A8 INT8 GEMM
+    through PyTorch (torch._int_mm, cuBLASLt), each problem with its own
+    random INT8 weight matrix, replayed back to back in one graph like the
+    W4A8 GEMM-only timing. Rows are padded to at least 32 (that routine
+    needs more than 16)."""
+    import torch
+    try:
+        dev = probs[0].X8.device
+        g = torch.Generator(device=dev)
+        g.manual_seed(1234)
+        ws, xs, ys = [], [], []
+        for p in probs:
+            m = max(p.M, 32)
+            ws.append(torch.randint(-119, 120, (p.N, p.K), dtype=torch.int8, device=dev, generator=g))
+            xs.append(torch.randint(-127, 128, (m, p.K), dtype=torch.int8, device=dev, generator=g))
+            ys.append(torch.empty((m, p.N), dtype=torch.int32, device=dev))
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            for x, w, y in zip(xs, ws, ys):     # warm-up outside capture (library handles, kernels)
+                torch._int_mm(x, w.t(), out=y)
+        stream.synchronize()
+        with torch.cuda.graph(graph, stream=stream):
+            for x, w, y in zip(xs, ws, ys):
+                torch._int_mm(x, w.t(), out=y)
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                graph.replay()
+        stream.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record()
+            for _ in range(reps):
+                graph.replay()
+            e1.record()
+        stream.synchronize()
+        us = 1000.0 * e0.elapsed_time(e1) / reps
+        del graph, ws, xs, ys
+        return {"gemm_us_per_step": round(us, 2), "w4a8_gemm_us_per_step": round(w4a8_us, 2),
+                "w4a8_speedup": round(us / w4a8_us, 3),
+                "how": "torch._int_mm (cuBLASLt INT8) on the same shapes, rows padded to >= 32, one graph "
+                       "of the step's GEMMs replayed back to back, events around the replays"}
+    except Exception as exc:   # context only: never fails the run
+        return {"unavailable": "%s: %s" % (type(exc).__name__, str(exc)[:200])}
 
 
 def run_e2e(args, probs, qoq, stream):

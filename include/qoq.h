@@ -186,6 +186,24 @@ qoq_status qoq_gemm_fp16_out_static_ws(const int8_t *X8, const void *s_x_fp16, c
                                        const void *blob, int64_t M, int64_t N, int64_t K, int group_size,
                                        void *Y_fp16, int32_t *status, void *stream);
 
+/*
+ * Self-test of the device-side bounded waits (failure detection without a
+ * fault; the paper has no counterpart). One small kernel waits, each for at
+ * most limit_ns nanoseconds (1 .. 2e9), on an mbarrier phase that never
+ * completes and on a global flag that nothing sets; each wait must give up,
+ * record its failure and return. The kernel then exits normally and the
+ * context stays usable.
+ *
+ * status: device int32[32], 16-byte aligned, owned by the caller; zeroed by
+ * the call (on `stream`). After the stream completes: status[0..3] =
+ * {QOQ_ERR_TIMEOUT, wait site 4, block 0, detail 1} for the mbarrier wait and
+ * status[8..11] = {QOQ_ERR_TIMEOUT, wait site 6, block 0, detail 2} for the
+ * flag wait (sites as in the GEMM workspace status words).
+ * Returns QOQ_ERR_INVALID_ARG / QOQ_ERR_ALIGNMENT before any launch,
+ * QOQ_ERR_CUDA if the launch fails.
+ */
+qoq_status qoq_watchdog_selftest(int32_t *status, int64_t limit_ns, void *stream);
+
 /* Name of a status code (static string, never NULL). */
 const char *qoq_status_string(qoq_status status);
 

@@ -85,3 +85,11 @@ def test_argument_validation_without_launch(L):
     assert L.qoq_w4a8_gemm(ctypes.c_void_p(16 * 1024 + 8), None, dummy, 4, 128, 128, 128, dummy, dummy, ws,
                            None) == 3
     assert L.qoq_w4a8_gemm(dummy, None, dummy, 0, 128, 128, 128, dummy, dummy, ws, None) == 0   # M = 0
+
+
+def test_watchdog_selftest_validation_without_launch(L):
+    """Argument errors return before any CUDA call (so they work with no GPU)."""
+    assert L.qoq_watchdog_selftest(None, 1000, None) == 1            # QOQ_ERR_INVALID_ARG
+    assert L.qoq_watchdog_selftest(ctypes.c_void_p(16), 0, None) == 1
+    assert L.qoq_watchdog_selftest(ctypes.c_void_p(16), 3_000_000_000, None) == 1
+    assert L.qoq_watchdog_selftest(ctypes.c_void_p(18), 1000, None) == 3   # QOQ_ERR_ALIGNMENT

@@ -14,6 +14,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libqoq.so")
 
 QOQ_OK = 0
+QOQ_ERR_TIMEOUT = 7
 STATUS = {0: "QOQ_OK", 1: "QOQ_ERR_INVALID_ARG", 2: "QOQ_ERR_UNSUPPORTED", 3: "QOQ_ERR_ALIGNMENT",
           4: "QOQ_ERR_WORKSPACE", 5: "QOQ_ERR_BAD_BLOB", 6: "QOQ_ERR_CUDA", 7: "QOQ_ERR_TIMEOUT"}
 TILE = 128
@@ -42,6 +43,8 @@ def lib() -> ctypes.CDLL:
         L.qoq_quantize_weights.argtypes = [vp, i64, i64, i32, vp, sz, vp]
         L.qoq_w4a8_gemm.argtypes = [vp, vp, vp, i64, i64, i64, i32, vp, vp, sz, vp]
         L.qoq_gemm_fp16_out.argtypes = [vp, vp, vp, vp, i64, i64, i64, i32, vp, vp, sz, vp]
+        L.qoq_watchdog_selftest.argtypes = [vp, i64, vp]
+        L.qoq_watchdog_selftest.restype = ctypes.c_int
         L.qoq_status_string.argtypes = [ctypes.c_int]
         L.qoq_status_string.restype = ctypes.c_char_p
         for f in (L.qoq_quantize_act_per_token, L.qoq_quantize_weights, L.qoq_w4a8_gemm, L.qoq_gemm_fp16_out):
@@ -146,6 +149,16 @@ class Workspace:
 
     def reset(self):
         self.buf.zero_()
+
+
+def watchdog_selftest(limit_ns=50_000_000, stream=None):
+    """Run the device bounded-wait self-test; returns the 32 status words
+    (the mbarrier wait's record at [0:4], the flag wait's at [8:12])."""
+    import torch
+    status = torch.zeros(32, dtype=torch.int32, device="cuda")
+    _check("qoq_watchdog_selftest", lib().qoq_watchdog_selftest(_ptr(status), int(limit_ns), _stream(stream)))
+    torch.cuda.synchronize()
+    return status.cpu().tolist()
 
 
 def w4a8_gemm(X8, blob, N, K, group_size=GROUP, rowsum=None, ws=None, acc=None, stream=None):
