@@ -41,19 +41,31 @@ GROUP = 128
 SHAPES = [(K, N) for (K, N, _) in inputs.LLAMA3_8B]
 NAMES = [name for (_, _, name) in inputs.LLAMA3_8B]
 WORKLOADS = {
-    "decode": dict(M=inputs.DECODE_M, span=None,
+    "decode": dict(M=inputs.DECODE_M, span=None, shapes=inputs.LLAMA3_8B, group=GROUP, std=0.02, bound="hbm",
                    desc="Llama-3-8B decode GEMMs (qkv 4096->6144, o 4096->4096, gate_up 4096->28672, "
                         "down 14336->4096) x M in {1,4,16,64,256}, g128, act-quant + GEMM"),
-    "prefill": dict(M=inputs.PREFILL_M, span=(-3, 1),
+    "prefill": dict(M=inputs.PREFILL_M, span=(-3, 1), shapes=inputs.LLAMA3_8B, group=GROUP, std=0.02,
+                    bound="tensor",
                     desc="Llama-3-8B prefill GEMMs (same four shapes) x M in {2048,8192,16384}, g128, "
                          "per-token scales 1e-3..1e1, act-quant + GEMM"),
+    "qwen": dict(M=inputs.QWEN_M, span=None, shapes=inputs.QWEN15_72B, group=GROUP, std=0.01, bound="mixed",
+                 desc="Qwen1.5-72B GEMMs (qkv 8192->24576, o 8192->8192, gate_up 8192->49152, "
+                      "down 24576->8192) x M in {1,16,128,512,4096}, g128, act-quant + GEMM"),
+    "perchannel": dict(M=inputs.PER_CHANNEL_M, span=None, shapes=inputs.LLAMA2_7B, group=0, std=0.02,
+                       bound="mixed",
+                       desc="per-channel variant (no group level) on Llama-2-7B GEMMs (qkv 4096->12288, "
+                            "o 4096->4096, gate_up 4096->22016, down 11008->4096) x M in 1..1024 (powers of 2), "
+                            "act-quant + GEMM"),
 }
 
 
-def gemm_bytes(M, N, K):
+def gemm_bytes(M, N, K, group=GROUP):
     """Algorithmic HBM bytes of one W4A8 GEMM: 4-bit weights, (s, z*s) per
-    group, s_w, X8, s_x and the FP16 output."""
-    return 0.5 * N * K + 2 * N * (K // GROUP) + 2 * N + M * K + 2 * M + 2 * M * N
+    group and s_w (group 128), or the FP16 s and z per channel plus the row
+    sums (per-channel variant); X8, s_x and the FP16 output."""
+    if group:
+        return 0.5 * N * K + 2 * N * (K // group) + 2 * N + M * K + 2 * M + 2 * M * N
+    return 0.5 * N * K + 4 * N + M * K + 2 * M + 4 * M + 2 * M * N
 
 
 def gemm_ops(M, N, K):
@@ -98,10 +110,10 @@ def measured_traffic(workload):
     return int(vals["traffic_per_launch_bytes"])
 
 
-def roof_us(M, N, K, peaks):
+def roof_us(M, N, K, peaks, group=GROUP):
     """Roofline time: the slower of HBM bytes and INT8 tensor work (INT8 peak =
     2 x the measured dense bf16 peak, the nominal 4.5/2.25 PFLOP/s ratio)."""
-    t_mem = gemm_bytes(M, N, K) / (peaks["hbm"] * 1e9)
+    t_mem = gemm_bytes(M, N, K, group) / (peaks["hbm"] * 1e9)
     t_tc = gemm_ops(M, N, K) / (2.0 * peaks["bf16"] * 1e12)
     return max(t_mem, t_tc) * 1e6, ("hbm" if t_mem >= t_tc else "tensor")
 
@@ -189,17 +201,18 @@ def sum_over_ranks(x: float, device=None) -> float:
 # ------------------------------------------------------------- GPU arm
 
 class Problem:
-    def __init__(self, K, N, M, blob, X, span, device):
+    def __init__(self, K, N, M, blob, X, span, device, group=GROUP, name=""):
         import torch
         from w4a8_quantized_gemm_qoq_b200 import qoq
         self.K, self.N, self.M = K, N, M
+        self.group, self.name = group, name
         self.blob = blob
         self.X = X
         self.X8 = torch.empty((M, K), dtype=torch.int8, device=device)
         self.s_x = torch.empty((M,), dtype=torch.float16, device=device)
         self.rowsum = torch.empty((M,), dtype=torch.int32, device=device)
         self.Y = torch.empty((M, N), dtype=torch.float16, device=device)
-        self.ws = qoq.Workspace.for_shape(M, N, K, GROUP, device)
+        self.ws = qoq.Workspace.for_shape(M, N, K, group, device)
 
     def run(self, qoq, ev=None):
         if ev is not None:
@@ -207,14 +220,14 @@ class Problem:
         qoq.quantize_act_per_token(self.X, self.X8, self.s_x, self.rowsum)
         if ev is not None:
             ev[1].record()
-        qoq.gemm_fp16_out(self.X8, self.s_x, self.blob, self.N, self.K, GROUP, rowsum=self.rowsum, ws=self.ws,
-                          Y=self.Y)
+        qoq.gemm_fp16_out(self.X8, self.s_x, self.blob, self.N, self.K, self.group, rowsum=self.rowsum,
+                          ws=self.ws, Y=self.Y)
         if ev is not None:
             ev[2].record()
 
     def run_gemm(self, qoq):
-        qoq.gemm_fp16_out(self.X8, self.s_x, self.blob, self.N, self.K, GROUP, rowsum=self.rowsum, ws=self.ws,
-                          Y=self.Y)
+        qoq.gemm_fp16_out(self.X8, self.s_x, self.blob, self.N, self.K, self.group, rowsum=self.rowsum,
+                          ws=self.ws, Y=self.Y)
 
 
 def build_problems(workload, device, seed):
@@ -222,15 +235,15 @@ def build_problems(workload, device, seed):
     from w4a8_quantized_gemm_qoq_b200 import qoq
     wl = WORKLOADS[workload]
     probs = []
-    for si, (K, N) in enumerate(SHAPES):
-        W = torch.from_numpy(inputs.make_weights(N, K, seed=seed + si)).to(device)
-        blob0 = qoq.quantize_weights(W, GROUP)
+    for si, (K, N, name) in enumerate(wl["shapes"]):
+        W = torch.from_numpy(inputs.make_weights(N, K, seed=seed + si, std=wl["std"])).to(device)
+        blob0 = qoq.quantize_weights(W, wl["group"])
         del W
         for mi, M in enumerate(wl["M"]):
             blob = blob0 if mi == 0 else blob0.clone()        # one copy per GEMM: no L2 reuse in a step
             X = torch.from_numpy(inputs.make_activations(M, K, seed=seed + 100 * si + mi,
                                                          token_scale_span=wl["span"])).to(device)
-            probs.append(Problem(K, N, M, blob, X, wl["span"], device))
+            probs.append(Problem(K, N, M, blob, X, wl["span"], device, wl["group"], name))
     torch.cuda.synchronize()
     return probs
 
@@ -345,10 +358,12 @@ def run_gpu(args, rank, world, local_rank):
     tot_bytes = tot_gemm_us = 0.0
     for i, p in enumerate(probs):
         us = 1000.0 * gemm_ms[i]
-        b = gemm_bytes(p.M, p.N, p.K)
-        r_us, bound = roof_us(p.M, p.N, p.K, peaks)
-        per.append({"shape": NAMES[SHAPES.index((p.K, p.N))], "K": p.K, "N": p.N, "M": p.M,
-                    "gemm_us_in_step": round(us, 3), "act_quant_us_in_step": round(1000.0 * act_ms[i], 3),
+        b = gemm_bytes(p.M, p.N, p.K, p.group)
+        r_us, bound = roof_us(p.M, p.N, p.K, peaks, p.group)
+        aq_us = 1000.0 * act_ms[i]
+        per.append({"shape": p.name, "K": p.K, "N": p.N, "M": p.M,
+                    "gemm_us_in_step": round(us, 3), "act_quant_us_in_step": round(aq_us, 3),
+                    "act_quant_GBps_in_step": round((3.0 * p.M * p.K + 6 * p.M) / aq_us / 1e3, 1),
                     "TOPS": round(gemm_ops(p.M, p.N, p.K) / us / 1e6, 2), "GBps": round(b / us / 1e3, 1),
                     "roof_us": round(r_us, 3), "bound": bound, "frac_of_roofline": round(r_us / us, 3)})
         tot_bytes += b
@@ -356,7 +371,7 @@ def run_gpu(args, rank, world, local_rank):
     timing = {"launch_us": round(gemm_only_us / nP, 3), "launches": nP, "replays": KG,
               "how": "graph of the step's %d GEMM launches replayed back to back; CUDA events around the "
                      "replays on the launching stream" % nP}
-    if args.workload == "decode":
+    if wl["bound"] == "hbm":
         achieved = tot_bytes / gemm_only_us / 1e3
         roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm"], "unit": "GB/s",
                     "frac": round(achieved / peaks["hbm"], 4), "traffic": measured_traffic("decode"),
@@ -364,7 +379,7 @@ def run_gpu(args, rank, world, local_rank):
                     "peak_source": peaks["src"], "kernel": "qoq_gemm_kernel",
                     "frac_of_time_roofline": round(sum(x["roof_us"] for x in per) / gemm_only_us, 4),
                     "timing": timing}
-    else:
+    elif wl["bound"] == "tensor":
         achieved = ops_step / gemm_only_us / 1e6
         pk = 2.0 * peaks["bf16"]
         roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": pk, "unit": "TOPS",
@@ -372,6 +387,14 @@ def run_gpu(args, rank, world, local_rank):
                     " (INT8 = 2 x measured bf16 burst, nominal ratio)", "kernel": "qoq_gemm_kernel",
                     "frac_of_time_roofline": round(sum(x["roof_us"] for x in per) / gemm_only_us, 4),
                     "timing": timing}
+    else:
+        # Shapes on both sides of the crossover: the fraction is roofline time
+        # (each GEMM's slower bound) over measured time, summed over the step.
+        roof = sum(x["roof_us"] for x in per)
+        roofline = {"bound": "mixed", "achieved": round(roof / gemm_only_us, 4), "peak": 1.0,
+                    "unit": "fraction of each GEMM's roofline time", "frac": round(roof / gemm_only_us, 4),
+                    "traffic": None, "peak_source": peaks["src"], "kernel": "qoq_gemm_kernel",
+                    "frac_of_time_roofline": round(roof / gemm_only_us, 4), "timing": timing}
 
     e2e = run_e2e(args, probs, qoq, stream) if rank == 0 else None
     w8a8 = run_w8a8(probs, stream, gemm_only_us, max(K, 10)) if rank == 0 else None
@@ -380,9 +403,11 @@ def run_gpu(args, rank, world, local_rank):
         "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup),
         "ms_per_step": round(step_ms, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "int8", "data": "synthetic",
-        "config": {"workload": wl["desc"], "M": wl["M"], "shapes_K_N": SHAPES, "group_size": GROUP,
+        "config": {"workload": wl["desc"], "M": wl["M"], "shapes_K_N": [(K, N) for (K, N, _) in wl["shapes"]],
+                   "group_size": wl["group"],
                    "l2": "inputs larger than L2: each GEMM of a step reads its own packed-weight copy "
-                         "(%.0f MB per step)" % (sum(0.5 * p.N * p.K + p.N * p.K / 64 for p in probs) / 1e6),
+                         "(%.0f MB per step)" % (sum(0.5 * p.N * p.K + (p.N * p.K / 64 if p.group else 4 * p.N)
+                                                     for p in probs) / 1e6),
                    "launch": "CUDA graph replay of the step; per-launch events from the last %d steps" % n_ev,
                    "parallelism": "replicas (one independent step per GPU)" if world > 1 else "single GPU"},
         "roofline": roofline,
@@ -489,7 +514,7 @@ def run_e2e(args, probs, qoq, stream):
         for p, a, b, c in zip(probs, hx, dx, hy):
             b.copy_(a, non_blocking=True)
             X8, s_x, rs = qoq.quantize_act_per_token(b, p.X8, p.s_x, p.rowsum)
-            qoq.gemm_fp16_out(X8, s_x, p.blob, p.N, p.K, GROUP, rowsum=rs, ws=p.ws, Y=p.Y)
+            qoq.gemm_fp16_out(X8, s_x, p.blob, p.N, p.K, p.group, rowsum=rs, ws=p.ws, Y=p.Y)
             c.copy_(p.Y, non_blocking=True)
 
     steps = max(1, args.steps)
@@ -515,21 +540,31 @@ def run_e2e(args, probs, qoq, stream):
 
 def oracle_sample(workload, seed=0):
     """A bounded sample of the workload for the CPU oracle: the o-projection
-    GEMM (K=N=4096) at M=16 (decode) or M=64 (prefill), weights quantised
-    beforehand (offline), act-quant + int64 GEMM + FP16 epilogue timed."""
+    GEMM (K=N=4096) at M=16 (decode-sized workloads) or M=64 (prefill), weights
+    quantised beforehand (offline), act-quant + int64 GEMM + FP16 epilogue
+    timed; the per-channel workload uses the per-channel scheme."""
     import oracle
     K, N = 4096, 4096
-    M = 16 if workload == "decode" else 64
-    W = inputs.make_weights(N, K, seed=seed)
-    X = inputs.make_activations(M, K, seed=seed, token_scale_span=WORKLOADS[workload]["span"])
-    d = oracle.quantize_weights_group(W)
+    M = 64 if workload == "prefill" else 16
+    wl = WORKLOADS[workload]
+    W = inputs.make_weights(N, K, seed=seed, std=wl["std"])
+    X = inputs.make_activations(M, K, seed=seed, token_scale_span=wl["span"])
+    if wl["group"]:
+        d = oracle.quantize_weights_group(W)
 
-    def once():
-        X8, s_x, rowsum = oracle.quantize_act_per_token(X)
-        acc = oracle.gemm_int(X8, d["Wint"])
-        oracle.epilogue_fp16(acc, s_x, d["s_w"])
+        def once():
+            X8, s_x, rowsum = oracle.quantize_act_per_token(X)
+            acc = oracle.gemm_int(X8, d["Wint"])
+            oracle.epilogue_fp16(acc, s_x, d["s_w"])
+    else:
+        d = oracle.quantize_weights_per_channel(W)
+
+        def once():
+            X8, s_x, rowsum = oracle.quantize_act_per_token(X)
+            t = oracle.w4a8_gemm_per_channel(X8, rowsum, d["q"], d["z"])
+            oracle.epilogue_fp16(t, s_x, d["s"])
     desc = "o-proj GEMM K=N=4096, M=%d: act quant + int64 triple-loop GEMM + FP16 epilogue " \
-           "(weights pre-quantised)" % M
+           "(weights pre-quantised%s)" % (M, "" if wl["group"] else ", per-channel variant")
     return once, gemm_ops(M, N, K), desc
 
 
