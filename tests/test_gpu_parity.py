@@ -201,3 +201,33 @@ def test_graph_replays_are_bit_identical():
             _, d = oracle.quantize_weights(p["W"][nt * 128:(nt + 1) * 128], 128)
             want = oracle.epilogue_fp16(oracle.gemm_int(X8s, d["Wint"]), s_xs, d["s_w"])
             assert_fp16_close(Yh[:, nt * 128:(nt + 1) * 128], want, "graph case %d tile %d" % (i, nt))
+
+
+# ------------------------------------------------ full matrices at prefill sizes
+
+@pytest.mark.parametrize("M,N,K", [(2048, 4096, 14336), (4096, 28672, 4096)])
+def test_full_matrix_against_library_int8_gemm(M, N, K):
+    """Every element at a prefill size: X8 against the oracle's activation
+    quantiser; the INT32 GEMM against a library INT8 GEMM (torch._int_mm,
+    independent of this library's kernels) of the oracle's X8 and Wint; the
+    FP16 output against the oracle's epilogue of those sums (<= 1 ulp)."""
+    t = torch()
+    W = inputs.make_weights(N, K, seed=31)
+    X = inputs.make_activations(M, K, seed=31, token_scale_span=(-3, 1))
+    d = oracle.quantize_weights_group(W)
+    X8o, s_xo, _ = oracle.quantize_act_per_token(X)
+    ref = t._int_mm(dev(X8o), dev(d["Wint"]).t())
+    t.cuda.synchronize()
+
+    blob = qoq.quantize_weights(dev(W), 128)
+    X8, s_x, rs = qoq.quantize_act_per_token(dev(X))
+    ws = qoq.Workspace.for_shape(M, N, K, 128)
+    acc = qoq.w4a8_gemm(X8, blob, N, K, 128, rowsum=rs, ws=ws)
+    Y = qoq.gemm_fp16_out(X8, s_x, blob, N, K, 128, rowsum=rs, ws=ws)
+    t.cuda.synchronize()
+    assert ws.status() == 0
+    assert t.equal(X8, dev(X8o)), "X8 differs from the oracle"
+    assert np.array_equal(host(s_x).view(np.uint16), s_xo.view(np.uint16))
+    assert t.equal(acc, ref), "INT32 sums differ from the library INT8 GEMM of the oracle's operands"
+    want = oracle.epilogue_fp16(host(ref), s_xo, d["s_w"])
+    assert_fp16_close(host(Y), want, "full FP16 output")

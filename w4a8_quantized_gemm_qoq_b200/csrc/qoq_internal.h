@@ -57,7 +57,7 @@ inline BlobLayout blob_layout(int64_t N, int64_t K, int group) {
 // smallest tile that holds all tokens. Beyond that the choice trades weight
 // re-reads and dequantisation (once per token tile) against enough work units
 // for every SM and the stream-K partial-sum traffic; the thresholds below come
-// from B200 measurements on Llama-3-8B linear shapes. Long K (>= 64 k-tiles)
+// from B200 measurements on Llama-3-8B and Qwen1.5-72B linear shapes. Long K
 // prefers the widest tile, whose tensor work per k-tile hides the dequant.
 inline int token_tile_for(int64_t M, int64_t N, int64_t K) {
     const int64_t NT = N / kTileN, KT = K / kTileK;
@@ -65,9 +65,9 @@ inline int token_tile_for(int64_t M, int64_t N, int64_t K) {
     if (M <= 16) return 16;
     if (M <= 32) return 32;
     if (M <= 64) return blocks(64) >= 2500 ? 64 : 32;
-    if (M <= 128) return 64;
+    if (M <= 128) return blocks(128) >= 6000 ? 128 : 64;
     if (M <= 256) return blocks(128) >= 10000 ? 128 : 64;
-    if (M <= 512) return 128;
+    if (M <= 512) return KT >= 128 ? 256 : 128;
     return KT >= 64 ? 256 : 128;
 }
 
