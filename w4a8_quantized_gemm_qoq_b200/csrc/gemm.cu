@@ -70,7 +70,7 @@ struct GemmCfg {
     static constexpr int kWBytes = kKB * kWTile;
     static constexpr int kStageBytes = (kXBytes + kWBytes + 1023) / 1024 * 1024;
     static constexpr int kSmemLimit = 232448;                   // 227 KB per CTA
-    static constexpr int kReserve = 2048;                       // alignment slack + barriers
+    static constexpr int kReserve = 4096;                       // alignment slack + control block
     // Two MMA issuers. Up to 64-token tiles (kAlt), issuer j takes the units
     // of index parity j (those its dequant warpgroup serves) into its own
     // accumulator, and the epilogue adds the two; wider tiles have no TMEM for
@@ -120,7 +120,12 @@ struct SharedCtl {
     uint64_t final_bar[2];
     uint32_t tmem_base;
     int abort_flag;
+    // The owner's epilogue inputs of the current token tile, staged once per
+    // tile: FP32(s_x) and (per-channel variant) the row sums.
+    float tok_scale[256];
+    int32_t tok_rowsum[256];
 };
+static_assert(sizeof(SharedCtl) + 1023 <= GemmCfg<16, 0>::kReserve, "control block outgrows the reserve");
 
 // First k-tile block of CTA c (the stream-K split), and the CTA holding block b.
 __device__ __forceinline__ uint32_t cta_begin(uint32_t c, uint32_t B, uint32_t G) {
@@ -178,17 +183,19 @@ struct UnitCursor {
 };
 
 // Epilogue for CH consecutive tokens (m_first ..) of weight row n. sx[j] is
-// FP32(s_x[m_first + j]) (the value for tokens past M is unused).
+// FP32(s_x[m_first + j]) and rs[j] the row sum of that token (shared memory;
+// values for tokens past M are unused).
 template <int CH, int MODE>
 __device__ __forceinline__ void store_outputs(const GemmParams &p, const uint32_t (&v)[CH], int64_t m_first,
-                                              int n, float col_scale, int col_zero, const float (&sx)[CH]) {
+                                              int n, float col_scale, int col_zero, const float *sx,
+                                              const int32_t *rs) {
     const int64_t N = p.N;
 #pragma unroll
     for (int j = 0; j < CH; ++j) {
         const int64_t m = m_first + j;
         if (m < p.M) {
             int32_t acc = (int32_t)v[j];
-            if (MODE == 1) acc -= col_zero * p.rowsum[m];
+            if (MODE == 1) acc -= col_zero * rs[j];
             if (p.fp16_out) {
                 const float y = __fmul_rn(__int2float_rn(acc), __fmul_rn(sx[j], col_scale));
                 static_cast<__half *>(p.out)[m * N + n] = __float2half_rn(y);
@@ -196,16 +203,6 @@ __device__ __forceinline__ void store_outputs(const GemmParams &p, const uint32_
                 static_cast<int32_t *>(p.out)[m * N + n] = acc;
             }
         }
-    }
-}
-
-// FP32 token scales of CH tokens from m_first (tokens past M repeat the last).
-template <int CH>
-__device__ __forceinline__ void load_token_scales(const GemmParams &p, int64_t m_first, float (&sx)[CH]) {
-#pragma unroll
-    for (int j = 0; j < CH; ++j) {
-        const int64_t m = m_first + j < p.M ? m_first + j : p.M - 1;
-        sx[j] = p.fp16_out ? __half2float(p.s_x[m]) : 0.0f;
     }
 }
 
@@ -546,8 +543,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 int col_zero = 0;
                 if (MODE == 1)
                     col_zero = __half2int_rn(reinterpret_cast<const __half *>(p.blob + p.off_zero)[n]);
-                float sx0[CO];
-                if (owner) load_token_scales<CO>(p, m0, sx0);
+                if (owner) {
+                    // Stage the tile's token scales (and row sums) in shared
+                    // memory: one round trip per tile instead of one per step.
+                    // The previous segment's readers have passed its closing
+                    // barrier; the barrier after the accumulator wait orders
+                    // these stores before every read.
+                    for (int j = threadIdx.x - kWarpEpilogue * 32; j < TOK; j += 128) {
+                        const int64_t m = m0 + j < p.M ? m0 + j : p.M - 1;
+                        ctl->tok_scale[j] = p.fp16_out ? __half2float(p.s_x[m]) : 0.0f;
+                        if (MODE == 1) ctl->tok_rowsum[j] = p.rowsum[m];
+                    }
+                }
                 // Every lane spins on its own; the vote reconverges the warp
                 // before the named barrier, and all four epilogue warps leave
                 // together (the shared-tile paths below meet at named barriers).
@@ -605,16 +612,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                                 for (int j = 0; j < CO; ++j) v[j] = (uint32_t)((int32_t)v[j] + t[cc][j]);
                         }
-                        if (c0 == 0) {
-                            store_outputs<CO, MODE>(p, v, m0, n, col_scale, col_zero, sx0);
-                        } else {
-                            float sx[CO];
-                            load_token_scales<CO>(p, m0 + c0, sx);
-                            store_outputs<CO, MODE>(p, v, m0 + c0, n, col_scale, col_zero, sx);
-                        }
+                        store_outputs<CO, MODE>(p, v, m0 + c0, n, col_scale, col_zero, ctl->tok_scale + c0,
+                                                ctl->tok_rowsum + c0);
                     }
+                    // Closing barrier: every read of the staged scales (and of
+                    // the contributors' partial sums) is done.
+                    named_bar_sync(1, 128);
                     if (c_last >= c_first) {
-                        named_bar_sync(1, 128);
                         if (warp == kWarpEpilogue)
                             for (uint32_t c = c_first + (uint32_t)lane; c <= c_last; c += 32) p.flags[c] = 0;
                         __syncwarp();
