@@ -40,6 +40,7 @@
 //     (which reach their share of the tile first) have stored their INT32
 //     partial sums and raised a flag. The sum is exact in any order.
 #include <algorithm>
+#include <cstring>
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_fp16.h>
@@ -70,7 +71,7 @@ struct GemmCfg {
     static constexpr int kWBytes = kKB * kWTile;
     static constexpr int kStageBytes = (kXBytes + kWBytes + 1023) / 1024 * 1024;
     static constexpr int kSmemLimit = 232448;                   // 227 KB per CTA
-    static constexpr int kReserve = 4096;                       // alignment slack + control block
+    static constexpr int kReserve = 12288;                      // alignment slack + control block
     // Two MMA issuers. Up to 64-token tiles (kAlt), issuer j takes the units
     // of index parity j (those its dequant warpgroup serves) into its own
     // accumulator, and the epilogue adds the two; wider tiles have no TMEM for
@@ -110,6 +111,8 @@ struct GemmParams {
     int NT, KT, MT;
     int grid;
     uint32_t total_blocks;  // MT * NT * KT (k-tile blocks)
+    int dp_waves;           // whole tiles per CTA taken in data-parallel waves
+    uint32_t sk_base;       // first block of the stream-K tail: dp_waves * grid * KT
     long long off_codes, off_scale, off_zero;
     int fp16_out;
 };
@@ -122,8 +125,11 @@ struct SharedCtl {
     int abort_flag;
     // The owner's epilogue inputs of the current token tile, staged once per
     // tile: FP32(s_x) and (per-channel variant) the row sums.
-    float tok_scale[256];
+    alignas(16) float tok_scale[256];
     int32_t tok_rowsum[256];
+    // Per epilogue warp, two alternating blocks of one step's FP16 outputs
+    // (16 tokens x 32 weight rows), the source of the TMA output stores.
+    alignas(128) __half out_stage[4][2][16 * 32];
 };
 static_assert(sizeof(SharedCtl) + 1023 <= GemmCfg<16, 0>::kReserve, "control block outgrows the reserve");
 
@@ -136,19 +142,53 @@ __device__ __forceinline__ uint32_t cta_of(uint32_t b, uint32_t B, uint32_t G) {
 }
 
 // Walks this CTA's k-tile blocks as pipeline units: up to KB consecutive
-// k-tiles of one tile, never crossing a tile boundary. No division per step.
+// k-tiles of one tile, never crossing a tile boundary. The schedule has two
+// phases. Data-parallel waves: CTA c takes whole tiles c, c + G, c + 2G, ...
+// (`waves` of them), so the G tiles in flight at a time are consecutive in
+// (token tile, n-tile) order and share activation and weight tiles in L2.
+// Stream-K tail: the remaining tiles' k-tile blocks [sk_base, B) are split
+// evenly over the G CTAs, CTA c taking blocks [sk_b0, sk_b1). Blocks are
+// numbered tile * KT + k-tile in both phases. No division per unit.
 template <int KB>
 struct UnitCursor {
-    uint32_t b, b1, seg_end;
+    uint32_t b, b1, seg_end;   // current block, end of the current range, end of the current segment
     int KT, NT;
     int kt, nk, nt, mt;
-    __device__ __forceinline__ void init(uint32_t b0, uint32_t b1_, int KT_, int NT_) {
-        b = b0;
-        b1 = b1_;
+    uint32_t tile, G;          // data-parallel phase: current tile, tile stride
+    int waves_left;            // data-parallel tiles after the current one
+    bool dp;
+    uint32_t sk_b0, sk_b1;
+    __device__ __forceinline__ void init(uint32_t c, uint32_t G_, int waves, uint32_t sk_b0_, uint32_t sk_b1_,
+                                         int KT_, int NT_) {
         KT = KT_;
         NT = NT_;
-        const uint32_t t = b0 / (uint32_t)KT;
-        kt = (int)(b0 - t * (uint32_t)KT);
+        G = G_;
+        sk_b0 = sk_b0_;
+        sk_b1 = sk_b1_;
+        if (waves > 0) {
+            dp = true;
+            waves_left = waves - 1;
+            tile = c;
+            start_tile();
+        } else {
+            dp = false;
+            waves_left = 0;
+            start_range();
+        }
+    }
+    __device__ __forceinline__ void start_tile() {
+        b = tile * (uint32_t)KT;
+        b1 = b + (uint32_t)KT;
+        kt = 0;
+        mt = (int)(tile / (uint32_t)NT);
+        nt = (int)(tile - (uint32_t)mt * (uint32_t)NT);
+        set_segment();
+    }
+    __device__ __forceinline__ void start_range() {
+        b = sk_b0;
+        b1 = sk_b1;
+        const uint32_t t = b / (uint32_t)KT;
+        kt = (int)(b - t * (uint32_t)KT);
         mt = (int)(t / (uint32_t)NT);
         nt = (int)(t - (uint32_t)mt * (uint32_t)NT);
         set_segment();
@@ -162,7 +202,7 @@ struct UnitCursor {
         const uint32_t left = seg_end - b;
         nk = left < (uint32_t)KB ? (int)left : KB;
     }
-    __device__ __forceinline__ bool done() const { return b >= b1; }
+    __device__ __forceinline__ bool done() const { return !dp && b >= b1; }
     // Advance one unit; returns true when the current segment (tile) ends.
     __device__ __forceinline__ bool advance() {
         b += (uint32_t)nk;
@@ -171,38 +211,81 @@ struct UnitCursor {
             set_nk();
             return false;
         }
-        if (b >= b1) return true;
-        kt = 0;
-        if (++nt == NT) {
-            nt = 0;
-            ++mt;
+        if (b < b1) {   // the stream-K range goes on with the next tile
+            kt = 0;
+            if (++nt == NT) {
+                nt = 0;
+                ++mt;
+            }
+            set_segment();
+            return true;
         }
-        set_segment();
+        if (dp) {
+            if (waves_left > 0) {
+                --waves_left;
+                tile += G;
+                start_tile();
+            } else {
+                dp = false;
+                start_range();   // may be empty: then done()
+            }
+        }
         return true;
     }
 };
 
-// Epilogue for CH consecutive tokens (m_first ..) of weight row n. sx[j] is
-// FP32(s_x[m_first + j]) and rs[j] the row sum of that token (shared memory;
-// values for tokens past M are unused).
+// Epilogue for CH consecutive tokens (m_first ..) of weight row n = n_warp +
+// lane (n_warp: the warp's first of 32 rows). sx[j] is FP32(s_x[m_first + j])
+// and rs[j] the row sum of that token (shared memory; values for tokens past M
+// are unused).
+//
+// FP16: the warp writes its CH x 32 block into `stage` (token-major, 64-byte
+// rows) and lane 0 stores it with one TMA copy, which leaves out the rows past
+// M. The two stage blocks of a warp alternate; before one is rewritten, the
+// copy issued from it two steps earlier must have finished reading it.
 template <int CH, int MODE>
-__device__ __forceinline__ void store_outputs(const GemmParams &p, const uint32_t (&v)[CH], int64_t m_first,
-                                              int n, float col_scale, int col_zero, const float *sx,
-                                              const int32_t *rs) {
+__device__ __forceinline__ void store_outputs_fp16(const CUtensorMap *tmap_y, const uint32_t (&v)[CH],
+                                                   int64_t m_first, int n_warp, int lane, float col_scale,
+                                                   int col_zero, const float *sx, const int32_t *rs,
+                                                   __half *stage) {
+    static_assert(CH == 16, "the output box is 16 tokens high");
+    if (lane == 0) bulk_wait_group_read<1>();
+    __syncwarp();
+    float scale[CH];
+#pragma unroll
+    for (int q = 0; q < CH / 4; ++q) {
+        const float4 f = reinterpret_cast<const float4 *>(sx)[q];
+        scale[4 * q] = f.x;
+        scale[4 * q + 1] = f.y;
+        scale[4 * q + 2] = f.z;
+        scale[4 * q + 3] = f.w;
+    }
+#pragma unroll
+    for (int j = 0; j < CH; ++j) {
+        int32_t acc = (int32_t)v[j];
+        if (MODE == 1) acc -= col_zero * rs[j];
+        const float y = __fmul_rn(__int2float_rn(acc), __fmul_rn(scale[j], col_scale));
+        stage[j * 32 + lane] = __float2half_rn(y);
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        tma_store_2d(tmap_y, stage, n_warp, (int)m_first);
+        bulk_commit_group();
+    }
+}
+
+// INT32 accumulators (after the per-channel zero-point term) of CH tokens.
+template <int CH, int MODE>
+__device__ __forceinline__ void store_outputs_i32(const GemmParams &p, const uint32_t (&v)[CH], int64_t m_first,
+                                                  int n, int col_zero, const int32_t *rs) {
     const int64_t N = p.N;
 #pragma unroll
     for (int j = 0; j < CH; ++j) {
         const int64_t m = m_first + j;
-        if (m < p.M) {
-            int32_t acc = (int32_t)v[j];
-            if (MODE == 1) acc -= col_zero * rs[j];
-            if (p.fp16_out) {
-                const float y = __fmul_rn(__int2float_rn(acc), __fmul_rn(sx[j], col_scale));
-                static_cast<__half *>(p.out)[m * N + n] = __float2half_rn(y);
-            } else {
-                static_cast<int32_t *>(p.out)[m * N + n] = acc;
-            }
-        }
+        int32_t acc = (int32_t)v[j];
+        if (MODE == 1) acc -= col_zero * rs[j];
+        if (m < p.M) static_cast<int32_t *>(p.out)[m * N + n] = acc;
     }
 }
 
@@ -228,7 +311,8 @@ __device__ __forceinline__ void add_second(uint32_t taddr, uint32_t (&v)[CH]) {
 
 template <int TOK, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
-    qoq_gemm_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ CUtensorMap tmap_x) {
+    qoq_gemm_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ CUtensorMap tmap_x,
+                    const __grid_constant__ CUtensorMap tmap_y) {
     using C = GemmCfg<TOK, MODE>;
     constexpr int CH = (TOK < 32 || C::kAlt) ? 16 : 32;   // epilogue TMEM chunk (16 when two accumulators are summed)
     constexpr int S = C::kStages;
@@ -266,6 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ctl->abort_flag = 1;   // reported on the status word after griddepcontrol.wait
     }
     if (warp == kWarpProducer && lane == 0) prefetch_tensormap(&tmap_x);
+    if (warp == kWarpEpilogue && lane == 0 && p.fp16_out) prefetch_tensormap(&tmap_y);
     if (warp == kWarpMma) {
         tmem_alloc(&ctl->tmem_base, C::kTmemCols);
         tmem_relinquish();
@@ -281,11 +366,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         atomicCAS(p.status, 0, QOQ_ERR_BAD_BLOB);
     }
 
-    // Stream-K share of this CTA: k-tile blocks [b0, b1) in (token tile,
-    // n-tile, k-tile) order, k-tile fastest.
-    const uint32_t B = p.total_blocks, G = (uint32_t)p.grid;
-    const uint32_t b0 = cta_begin(blockIdx.x, B, G);
-    const uint32_t b1 = cta_begin(blockIdx.x + 1, B, G);
+    // This CTA's schedule: p.dp_waves whole tiles (blockIdx.x + w * grid),
+    // then its stream-K share [b0, b1) of the tail blocks [sk_base, total)
+    // in (token tile, n-tile, k-tile) order, k-tile fastest.
+    const uint32_t G = (uint32_t)p.grid;
+    const uint32_t BS = p.total_blocks - p.sk_base;   // stream-K tail blocks
+    const uint32_t b0 = p.sk_base + cta_begin(blockIdx.x, BS, G);
+    const uint32_t b1 = p.sk_base + cta_begin(blockIdx.x + 1, BS, G);
     const int KT = p.KT;
 
     auto stage_x = [&](int s) { return smem + s * C::kStageBytes; };
@@ -297,7 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t pol_w = policy_evict_first();   // weights: streamed once
             const uint64_t pol_x = policy_evict_last();    // activations: reused by every n-tile
             UnitCursor<KB> cur;
-            cur.init(b0, b1, KT, p.NT);
+            cur.init(blockIdx.x, G, p.dp_waves, b0, b1, KT, p.NT);
             auto issue_w = [&](int s, const UnitCursor<KB> &c) {
                 mbar_arrive_expect_tx(&ctl->full[s], (uint32_t)(c.nk * (C::kWTile + C::kXTile)));
                 const uint8_t *wsrc = p.blob + p.off_codes + ((long long)c.nt * KT + c.kt) * C::kWTile;
@@ -367,7 +454,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 constexpr bool ALT = C::kAlt;
                 constexpr uint32_t idesc = idesc_i8(128, ALT ? TOK : TOK / 2, true, true);
                 UnitCursor<KB> cur;
-                cur.init(b0, b1, KT, p.NT);
+                cur.init(blockIdx.x, G, p.dp_waves, b0, b1, KT, p.NT);
                 int s = 0, seg = 0, unit = 0;
                 uint32_t ph = 0;
                 bool ok = true;
@@ -427,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int r = quarter * 32 + lane;               // weight row in the tile
             const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
             UnitCursor<KB> cur;
-            cur.init(b0, b1, KT, p.NT);
+            cur.init(blockIdx.x, G, p.dp_waves, b0, b1, KT, p.NT);
             int s = 0;
             uint32_t ph = 0;
             for (int i = 0; !cur.done(); ++i, cur.advance()) {
@@ -497,8 +584,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool leader = (threadIdx.x == kWarpEpilogue * 32);
             griddep_wait();   // outputs, scales, row sums and workspace belong to the previous kernel until now
             UnitCursor<KB> cur;
-            cur.init(b0, b1, KT, p.NT);
+            cur.init(blockIdx.x, G, p.dp_waves, b0, b1, KT, p.NT);
             int seg = 0, ubase = 0;
+            int obuf = 0;   // this warp's next output stage block
             while (!cur.done()) {
                 const uint32_t seg_b = cur.b, seg_e = cur.seg_end;
                 const int kt_lo = cur.kt, kt_hi = cur.kt + (int)(seg_e - seg_b);
@@ -516,12 +604,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int n = nt * kTileN + r;
                 const int64_t m0 = (int64_t)mt * TOK;
                 const bool two = C::kAlt && nunits >= 2;
+                // Token columns of the tile that hold tokens (>= 1): the steps
+                // past them (a ragged last tile) are neither loaded nor stored.
+                const int m_live = (int)(p.M - m0 < TOK ? p.M - m0 : TOK);
                 // Owner (or sole computer) of a tile: the CTA holding its first
                 // k-tile. Contributors c_first .. c_last (none if c_last < c_first).
                 const bool owner = kt_lo == 0;
                 const uint32_t c_first = blockIdx.x + 1;
                 const uint32_t c_last =
-                    (!owner || kt_hi == KT) ? blockIdx.x : cta_of(tile_b + (uint32_t)KT - 1, B, G);
+                    (!owner || kt_hi == KT) ? blockIdx.x : cta_of(tile_b + (uint32_t)KT - 1 - p.sk_base, BS, G);
                 constexpr int CO = 16;   // owner: token columns per step
                 if (c_last >= c_first) {
                     // Contributors reach their share of the tile first, so their
@@ -568,7 +659,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // CTA. Store the partial sums in this CTA's slot, raise its flag.
                     int32_t *part = p.partials + (long long)blockIdx.x * TOK * kTileN;
 #pragma unroll 1
-                    for (int c0 = 0; c0 < TOK; c0 += CH) {
+                    for (int c0 = 0; c0 < (m_live + CH - 1) / CH * CH; c0 += CH) {
                         uint32_t v[CH];
                         tmem_load<CH>(acc_addr + (uint32_t)c0, v);
                         if (two) add_second<CH>(acc2_addr + (uint32_t)c0, v);
@@ -588,12 +679,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // Owner: add the contributors' partial sums (loaded four
                     // contributors at a time, one L2 round trip), run the
                     // epilogue, clear their flags.
+                    const int c_end = (m_live + CO - 1) / CO * CO;
 #pragma unroll 1
-                    for (int c0 = 0; c0 < TOK; c0 += CO) {
+                    for (int c0 = 0; c0 < c_end; c0 += CO) {
                         uint32_t v[CO];
                         tmem_load<CO>(acc_addr + (uint32_t)c0, v);
                         if (two) add_second<CO>(acc2_addr + (uint32_t)c0, v);
-                        if (c0 + CO >= TOK) {
+                        if (c0 + CO >= c_end) {
                             tc_fence_before();
                             __syncwarp();
                             if (lane == 0) mbar_arrive(&ctl->acc_empty[buf]);
@@ -612,8 +704,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                                 for (int j = 0; j < CO; ++j) v[j] = (uint32_t)((int32_t)v[j] + t[cc][j]);
                         }
-                        store_outputs<CO, MODE>(p, v, m0 + c0, n, col_scale, col_zero, ctl->tok_scale + c0,
-                                                ctl->tok_rowsum + c0);
+                        if (p.fp16_out) {
+                            store_outputs_fp16<CO, MODE>(&tmap_y, v, m0 + c0, n - lane, lane, col_scale, col_zero,
+                                                         ctl->tok_scale + c0, ctl->tok_rowsum + c0,
+                                                         ctl->out_stage[quarter][obuf]);
+                            obuf ^= 1;
+                        } else {
+                            store_outputs_i32<CO, MODE>(p, v, m0 + c0, n, col_zero, ctl->tok_rowsum + c0);
+                        }
                     }
                     // Closing barrier: every read of the staged scales (and of
                     // the contributors' partial sums) is done.
@@ -626,6 +724,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 ++seg;
             }
+            // The output copies must be complete (not only done reading shared
+            // memory) before the CTA ends.
+            if (lane == 0) bulk_wait_group<0>();
+            __syncwarp();
         }
     }
 
@@ -677,6 +779,20 @@ static bool encode_x_map(CUtensorMap *map, const int8_t *X8, int64_t M, int64_t 
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// FP16 output Y [M][N]: boxes of 32 weight rows x 16 tokens, no swizzle (the
+// epilogue's stage blocks are plain token-major 64-byte rows).
+static bool encode_y_map(CUtensorMap *map, void *Y, int64_t M, int64_t N) {
+    auto encode = get_encode_fn();
+    if (!encode) return false;
+    const cuuint64_t gdim[2] = {(cuuint64_t)N, (cuuint64_t)M};
+    const cuuint64_t gstride[1] = {(cuuint64_t)N * 2};
+    const cuuint32_t box[2] = {32, 16};
+    const cuuint32_t estride[2] = {1, 1};
+    return encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, Y, gdim, gstride, box, estride,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int TOK, int MODE>
 static qoq_status launch_gemm_t(const GemmArgs &a, cudaStream_t stream) {
     using C = GemmCfg<TOK, MODE>;
@@ -694,8 +810,13 @@ static qoq_status launch_gemm_t(const GemmArgs &a, cudaStream_t stream) {
     });
     if (attr_err[dev] != cudaSuccess) return QOQ_ERR_CUDA;
 
-    CUtensorMap tmap;
+    CUtensorMap tmap, tmap_y;
     if (!encode_x_map(&tmap, a.X8, a.M, a.K, TOK)) return QOQ_ERR_CUDA;
+    if (a.fp16_out) {
+        if (!encode_y_map(&tmap_y, a.out, a.M, a.N)) return QOQ_ERR_CUDA;
+    } else {
+        memset(&tmap_y, 0, sizeof(tmap_y));   // INT32 outputs use plain stores
+    }
 
     const BlobLayout L = blob_layout(a.N, a.K, a.group);
     GemmParams p;
@@ -718,6 +839,11 @@ static qoq_status launch_gemm_t(const GemmArgs &a, cudaStream_t stream) {
     if (blocks >= (1ll << 31)) return QOQ_ERR_UNSUPPORTED;
     p.total_blocks = (uint32_t)blocks;
     p.grid = (int)std::min<long long>(std::min(sms, kMaxGrid), blocks);
+    // Whole tiles in data-parallel waves while at least one to two waves of
+    // tiles remain for the stream-K tail, which evens out the last wave.
+    const long long tiles = (long long)p.MT * p.NT;
+    p.dp_waves = tiles >= 2ll * p.grid ? (int)(tiles / p.grid) - 1 : 0;
+    p.sk_base = (uint32_t)((long long)p.dp_waves * p.grid * p.KT);
     p.off_codes = L.off_codes;
     p.off_scale = L.off_scale;
     p.off_zero = L.off_zero;
@@ -733,7 +859,8 @@ static qoq_status launch_gemm_t(const GemmArgs &a, cudaStream_t stream) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = kProgrammaticLaunch ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, qoq_gemm_kernel<TOK, MODE>, p, tmap) == cudaSuccess ? QOQ_OK : QOQ_ERR_CUDA;
+    return cudaLaunchKernelEx(&cfg, qoq_gemm_kernel<TOK, MODE>, p, tmap, tmap_y) == cudaSuccess ? QOQ_OK
+                                                                                               : QOQ_ERR_CUDA;
 }
 
 template <int MODE>

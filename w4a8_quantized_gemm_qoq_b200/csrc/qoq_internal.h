@@ -68,7 +68,7 @@ inline int token_tile_for(int64_t M, int64_t N, int64_t K) {
     if (M <= 128) return blocks(128) >= 6000 ? 128 : 64;
     if (M <= 256) return blocks(128) >= 10000 ? 128 : 64;
     if (M <= 512) return KT >= 128 ? 256 : 128;
-    return KT >= 64 ? 256 : 128;
+    return 256;
 }
 
 // Workspace: [0, 256) status word + reserved; then int32 flags [kMaxGrid]
