@@ -614,7 +614,31 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t c_last =
                     (!owner || kt_hi == KT) ? blockIdx.x : cta_of(tile_b + (uint32_t)KT - 1 - p.sk_base, BS, G);
                 constexpr int CO = 16;   // owner: token columns per step
-                if (c_last >= c_first) {
+                const bool polls = c_last >= c_first;
+                float col_scale = 0.0f;
+                int col_zero = 0;
+                if (owner) {
+                    // Inputs that depend neither on the accumulator nor on the
+                    // contributors, fetched first: the weight row's scale (and
+                    // zero point), and the tile's token scales (and row sums),
+                    // staged in shared memory once per tile. The previous
+                    // segment's readers have passed its closing barrier; the
+                    // barrier after the accumulator wait orders these stores
+                    // before every read. While contributors are polled, the
+                    // polling warp takes no part in the staging.
+                    col_scale = __half2float(reinterpret_cast<const __half *>(p.blob + p.off_scale)[n]);
+                    if (MODE == 1)
+                        col_zero = __half2int_rn(reinterpret_cast<const __half *>(p.blob + p.off_zero)[n]);
+                    if (!polls || warp != kWarpEpilogue) {
+                        const int t0 = threadIdx.x - kWarpEpilogue * 32;
+                        for (int j = polls ? t0 - 32 : t0; j < TOK; j += polls ? 96 : 128) {
+                            const int64_t m = m0 + j < p.M ? m0 + j : p.M - 1;
+                            ctl->tok_scale[j] = p.fp16_out ? __half2float(p.s_x[m]) : 0.0f;
+                            if (MODE == 1) ctl->tok_rowsum[j] = p.rowsum[m];
+                        }
+                    }
+                }
+                if (polls) {
                     // Contributors reach their share of the tile first, so their
                     // flags are usually up before this CTA's own accumulator is:
                     // poll them now (lanes of the first epilogue warp in
@@ -627,24 +651,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                         got = __all_sync(0xffffffffu, got);
                     }
                     if (named_bar_any(1, 128, !got)) break;
-                }
-                // Inputs of the first output step that do not depend on the
-                // accumulator are fetched before waiting for it.
-                const float col_scale = __half2float(reinterpret_cast<const __half *>(p.blob + p.off_scale)[n]);
-                int col_zero = 0;
-                if (MODE == 1)
-                    col_zero = __half2int_rn(reinterpret_cast<const __half *>(p.blob + p.off_zero)[n]);
-                if (owner) {
-                    // Stage the tile's token scales (and row sums) in shared
-                    // memory: one round trip per tile instead of one per step.
-                    // The previous segment's readers have passed its closing
-                    // barrier; the barrier after the accumulator wait orders
-                    // these stores before every read.
-                    for (int j = threadIdx.x - kWarpEpilogue * 32; j < TOK; j += 128) {
-                        const int64_t m = m0 + j < p.M ? m0 + j : p.M - 1;
-                        ctl->tok_scale[j] = p.fp16_out ? __half2float(p.s_x[m]) : 0.0f;
-                        if (MODE == 1) ctl->tok_rowsum[j] = p.rowsum[m];
-                    }
                 }
                 // Every lane spins on its own; the vote reconverges the warp
                 // before the named barrier, and all four epilogue warps leave
@@ -664,7 +670,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tmem_load<CH>(acc_addr + (uint32_t)c0, v);
                         if (two) add_second<CH>(acc2_addr + (uint32_t)c0, v);
 #pragma unroll
-                        for (int j = 0; j < CH; ++j) part[(c0 + j) * kTileN + r] = (int32_t)v[j];
+                        for (int j = 0; j < CH; ++j)
+                            if (c0 + j < m_live) part[(c0 + j) * kTileN + r] = (int32_t)v[j];
                     }
                     tc_fence_before();
                     __syncwarp();
@@ -676,8 +683,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (leader) st_release_gpu(p.flags + blockIdx.x, 1);
                     __syncwarp();
                 } else {
-                    // Owner: add the contributors' partial sums (loaded four
-                    // contributors at a time, one L2 round trip), run the
+                    // Owner: add the contributors' partial sums, run the
                     // epilogue, clear their flags.
                     const int c_end = (m_live + CO - 1) / CO * CO;
 #pragma unroll 1
@@ -690,19 +696,45 @@ __global__ void __launch_bounds__(kThreads, 1)
                             __syncwarp();
                             if (lane == 0) mbar_arrive(&ctl->acc_empty[buf]);
                         }
+                        // Contributors' partial sums: eight contributors per L2
+                        // round trip when at most four columns hold tokens, four
+                        // otherwise. Columns past the live ones hold stale values
+                        // (contributors store only the live ones); they belong to
+                        // no token and are never stored.
+                        if (m_live <= 4) {
 #pragma unroll 1
-                        for (uint32_t c = c_first; c <= c_last; c += 4) {
-                            int32_t t[4][CO];
+                            for (uint32_t c = c_first; c <= c_last; c += 8) {
+                                int32_t t[8][4];
 #pragma unroll
-                            for (int cc = 0; cc < 4; ++cc) {
-                                const int32_t *part = p.partials + (long long)(c + cc) * TOK * kTileN + c0 * kTileN + r;
+                                for (int cc = 0; cc < 8; ++cc) {
+                                    const int32_t *part =
+                                        p.partials + (long long)(c + cc) * TOK * kTileN + c0 * kTileN + r;
 #pragma unroll
-                                for (int j = 0; j < CO; ++j) t[cc][j] = (c + cc <= c_last) ? ld_cg_s32(part + j * kTileN) : 0;
+                                    for (int j = 0; j < 4; ++j)
+                                        t[cc][j] = (c + cc <= c_last) ? ld_cg_s32(part + j * kTileN) : 0;
+                                }
+#pragma unroll
+                                for (int cc = 0; cc < 8; ++cc)
+#pragma unroll
+                                    for (int j = 0; j < 4; ++j) v[j] += (uint32_t)t[cc][j];   // modulo 2^32: exact where the sum fits
                             }
+                        } else {
+#pragma unroll 1
+                            for (uint32_t c = c_first; c <= c_last; c += 4) {
+                                int32_t t[4][CO];
 #pragma unroll
-                            for (int cc = 0; cc < 4; ++cc)
+                                for (int cc = 0; cc < 4; ++cc) {
+                                    const int32_t *part =
+                                        p.partials + (long long)(c + cc) * TOK * kTileN + c0 * kTileN + r;
 #pragma unroll
-                                for (int j = 0; j < CO; ++j) v[j] = (uint32_t)((int32_t)v[j] + t[cc][j]);
+                                    for (int j = 0; j < CO; ++j)
+                                        t[cc][j] = (c + cc <= c_last) ? ld_cg_s32(part + j * kTileN) : 0;
+                                }
+#pragma unroll
+                                for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+                                    for (int j = 0; j < CO; ++j) v[j] += (uint32_t)t[cc][j];   // modulo 2^32: exact where the sum fits
+                            }
                         }
                         if (p.fp16_out) {
                             store_outputs_fp16<CO, MODE>(&tmap_y, v, m0 + c0, n - lane, lane, col_scale, col_zero,
@@ -724,9 +756,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 ++seg;
             }
-            // The output copies must be complete (not only done reading shared
-            // memory) before the CTA ends.
-            if (lane == 0) bulk_wait_group<0>();
+            // The output copies must have finished reading shared memory
+            // before the CTA ends (their global writes complete with the grid).
+            if (lane == 0) bulk_wait_group_read<0>();
             __syncwarp();
         }
     }

@@ -320,20 +320,31 @@ __device__ __forceinline__ void st_release_gpu(int32_t *p, int32_t v) {
     asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-__device__ __forceinline__ int32_t ld_acquire_gpu(const int32_t *p) {
+
+// Spin until *flag != 0, bounded like the pipeline waits.
+__device__ __forceinline__ int32_t ld_relaxed_gpu(const int32_t *p) {
     int32_t v;
-    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    asm volatile("ld.relaxed.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
 
-// Spin until *flag != 0, bounded like the pipeline waits.
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+
+// Spins until *flag != 0: relaxed loads back to back (a few lanes poll, so no
+// sleep between them), then one acquire fence, which with the relaxed load
+// that saw the releasing store orders every later access after that store.
 __device__ __forceinline__ bool wait_flag_bounded(const int32_t *flag, const Watchdog &wd, int detail,
                                                   uint64_t limit_ns = kWaitLimitNs) {
-    if (ld_acquire_gpu(flag) != 0) return true;
+    if (ld_relaxed_gpu(flag) != 0) {
+        fence_acq_rel_gpu();
+        return true;
+    }
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
-        __nanosleep(64);
-        if (ld_acquire_gpu(flag) != 0) return true;
+        if (ld_relaxed_gpu(flag) != 0) {
+            fence_acq_rel_gpu();
+            return true;
+        }
         if ((it & 15u) == 0) {
             if (wd.aborted()) return false;
             if (globaltimer_ns() - t0 > limit_ns) {
