@@ -111,8 +111,8 @@ struct GemmParams {
     int NT, KT, MT;
     int grid;
     uint32_t total_blocks;  // MT * NT * KT (k-tile blocks)
-    int dp_waves;           // whole tiles per CTA taken in data-parallel waves
-    uint32_t sk_base;       // first block of the stream-K tail: dp_waves * grid * KT
+    uint32_t dp_tiles;      // tiles 0 .. dp_tiles-1 go whole to CTAs in data-parallel waves
+    uint32_t sk_base;       // first block of the stream-K tail: dp_tiles * KT
     long long off_codes, off_scale, off_zero;
     int fp16_out;
 };
@@ -366,10 +366,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         atomicCAS(p.status, 0, QOQ_ERR_BAD_BLOB);
     }
 
-    // This CTA's schedule: p.dp_waves whole tiles (blockIdx.x + w * grid),
-    // then its stream-K share [b0, b1) of the tail blocks [sk_base, total)
-    // in (token tile, n-tile, k-tile) order, k-tile fastest.
+    // This CTA's schedule: the whole tiles blockIdx.x + w * grid below
+    // p.dp_tiles (`waves` of them), then its stream-K share [b0, b1) of the
+    // tail blocks [sk_base, total) in (token tile, n-tile, k-tile) order,
+    // k-tile fastest.
     const uint32_t G = (uint32_t)p.grid;
+    const int waves = p.dp_tiles > blockIdx.x ? (int)((p.dp_tiles - blockIdx.x + G - 1) / G) : 0;
     const uint32_t BS = p.total_blocks - p.sk_base;   // stream-K tail blocks
     const uint32_t b0 = p.sk_base + cta_begin(blockIdx.x, BS, G);
     const uint32_t b1 = p.sk_base + cta_begin(blockIdx.x + 1, BS, G);
@@ -384,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t pol_w = policy_evict_first();   // weights: streamed once
             const uint64_t pol_x = policy_evict_last();    // activations: reused by every n-tile
             UnitCursor<KB> cur;
-            cur.init(blockIdx.x, G, p.dp_waves, b0, b1, KT, p.NT);
+            cur.init(blockIdx.x, G, waves, b0, b1, KT, p.NT);
             auto issue_w = [&](int s, const UnitCursor<KB> &c) {
                 mbar_arrive_expect_tx(&ctl->full[s], (uint32_t)(c.nk * (C::kWTile + C::kXTile)));
                 const uint8_t *wsrc = p.blob + p.off_codes + ((long long)c.nt * KT + c.kt) * C::kWTile;
@@ -454,7 +456,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 constexpr bool ALT = C::kAlt;
                 constexpr uint32_t idesc = idesc_i8(128, ALT ? TOK : TOK / 2, true, true);
                 UnitCursor<KB> cur;
-                cur.init(blockIdx.x, G, p.dp_waves, b0, b1, KT, p.NT);
+                cur.init(blockIdx.x, G, waves, b0, b1, KT, p.NT);
                 int s = 0, seg = 0, unit = 0;
                 uint32_t ph = 0;
                 bool ok = true;
@@ -514,7 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int r = quarter * 32 + lane;               // weight row in the tile
             const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
             UnitCursor<KB> cur;
-            cur.init(blockIdx.x, G, p.dp_waves, b0, b1, KT, p.NT);
+            cur.init(blockIdx.x, G, waves, b0, b1, KT, p.NT);
             int s = 0;
             uint32_t ph = 0;
             for (int i = 0; !cur.done(); ++i, cur.advance()) {
@@ -584,7 +586,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool leader = (threadIdx.x == kWarpEpilogue * 32);
             griddep_wait();   // outputs, scales, row sums and workspace belong to the previous kernel until now
             UnitCursor<KB> cur;
-            cur.init(blockIdx.x, G, p.dp_waves, b0, b1, KT, p.NT);
+            cur.init(blockIdx.x, G, waves, b0, b1, KT, p.NT);
             int seg = 0, ubase = 0;
             int obuf = 0;   // this warp's next output stage block
             while (!cur.done()) {
@@ -874,8 +876,9 @@ static qoq_status launch_gemm_t(const GemmArgs &a, cudaStream_t stream) {
     // Whole tiles in data-parallel waves while at least one to two waves of
     // tiles remain for the stream-K tail, which evens out the last wave.
     const long long tiles = (long long)p.MT * p.NT;
-    p.dp_waves = tiles >= 2ll * p.grid ? (int)(tiles / p.grid) - 1 : 0;
-    p.sk_base = (uint32_t)((long long)p.dp_waves * p.grid * p.KT);
+    const long long dp_tiles = tiles >= 2ll * p.grid ? (tiles / p.grid - 1) * p.grid : 0;
+    p.dp_tiles = (uint32_t)dp_tiles;
+    p.sk_base = (uint32_t)(dp_tiles * p.KT);
     p.off_codes = L.off_codes;
     p.off_scale = L.off_scale;
     p.off_zero = L.off_zero;
