@@ -9,6 +9,9 @@ Contents
   qoq_ref.py   quantisers, packer, integer GEMM driver and FP32 epilogue in
                plain numpy, each step written from the QServe pages.
   qoq_gemm.c   the integer GEMM as a plain int64 triple loop (gcc, no tiling).
+  producers.py the fused activation producers (RMSNorm or SiLU-gated product,
+               then per-token INT8 quantisation) in plain numpy and Python
+               integers.
 
 Pinning: every function here is checked in ``tests/test_oracle_*.py`` against
 something other than itself -- exact rational arithmetic (``fractions``),
@@ -18,3 +21,4 @@ brute force with Python integers and hand-worked fixtures in
 from a printed value.
 """
 from .qoq_ref import *  # noqa: F401,F403
+from . import producers  # noqa: F401
