@@ -75,6 +75,42 @@ qoq_status qoq_quantize_act_per_token(const void *X_fp16, int64_t M, int64_t K,
                                       void *stream);
 
 /*
+ * Fused activation producers: the layer in front of a GEMM writes the GEMM's
+ * per-token INT8 activations directly, with no FP16 tensor in between.
+ * (paperlayer.ai summary, section 5 "QServe Serving System", "Runtime and
+ *  precision mapping": activation quantisation is fused into the preceding
+ *  normalisation or activation layer.)
+ *
+ * Both compute an FP32 row h per token and quantise it like
+ * qoq_quantize_act_per_token: s_x = FP16(max_k |h_k| / 127),
+ * X8 = clamp(RNE(h / FP32(s_x)), -127, 127) (0 where s_x == 0),
+ * rowsum = sum_k X8. Every floating-point step is one correctly rounded
+ * binary32 operation, so the results are reproducible bit for bit:
+ *
+ * qoq_rmsnorm_quant (RMSNorm):
+ *   ss = sum_k x_k^2 computed exactly, then rounded once to FP32;
+ *   r = sqrt(ss / K + eps);  h_k = (x_k / r) * gamma_k.
+ *   X_fp16 [M][K] FP16, read.   gamma_fp16 [K] FP16, read.   eps > 0, finite.
+ *
+ * qoq_silu_mul_quant (SiLU-gated product of a merged gate/up projection):
+ *   h_k = (g_k / (1 + e^-g_k)) * u_k, with g = GU[m][0..I), u = GU[m][I..2I)
+ *   and e^x in FP32 by Cody-Waite argument reduction (x = n ln2 + r), the
+ *   degree-7 Taylor polynomial of e^r (Horner) and an exact scaling by 2^n
+ *   (0 below x = -87.33654, +inf above x = 88.72284).
+ *   GU_fp16 [M][2I] FP16, read.
+ *
+ * Outputs: X8 [M][K or I] int8, s_x [M] FP16, rowsum [M] int32 (may be NULL).
+ * K (or I) must be a positive multiple of 8, at most 32768 (otherwise
+ * QOQ_ERR_UNSUPPORTED); X, gamma, GU and X8 16-byte aligned. M == 0 is a no-op.
+ */
+qoq_status qoq_rmsnorm_quant(const void *X_fp16, const void *gamma_fp16, int64_t M,
+                             int64_t K, float eps, int8_t *X8, void *s_x_fp16,
+                             int32_t *rowsum, void *stream);
+
+qoq_status qoq_silu_mul_quant(const void *GU_fp16, int64_t M, int64_t I, int8_t *X8,
+                              void *s_x_fp16, int32_t *rowsum, void *stream);
+
+/*
  * Offline weight quantisation and packing into the compute-order blob.
  * (paperlayer.ai summary, section 4 "Progressive Group Quantization" and
  *  section 5 "compute-aware weight reordering"; study.space summary.)

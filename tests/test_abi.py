@@ -85,6 +85,22 @@ def test_argument_validation_without_launch(L):
     assert L.qoq_w4a8_gemm(ctypes.c_void_p(16 * 1024 + 8), None, dummy, 4, 128, 128, 128, dummy, dummy, ws,
                            None) == 3
     assert L.qoq_w4a8_gemm(dummy, None, dummy, 0, 128, 128, 128, dummy, dummy, ws, None) == 0   # M = 0
+    # fused producers
+    f = ctypes.c_float
+    assert L.qoq_rmsnorm_quant(dummy, dummy, -1, 4096, f(1e-5), dummy, dummy, None, None) == 1
+    assert L.qoq_rmsnorm_quant(dummy, dummy, 4, 4096, f(0.0), dummy, dummy, None, None) == 1      # eps > 0
+    assert L.qoq_rmsnorm_quant(dummy, dummy, 4, 4096, f(float("inf")), dummy, dummy, None, None) == 1
+    assert L.qoq_rmsnorm_quant(dummy, dummy, 4, 4100, f(1e-5), dummy, dummy, None, None) == 2     # K % 8
+    assert L.qoq_rmsnorm_quant(dummy, dummy, 4, 65536, f(1e-5), dummy, dummy, None, None) == 2    # too wide
+    assert L.qoq_rmsnorm_quant(dummy, None, 4, 4096, f(1e-5), dummy, dummy, None, None) == 1
+    assert L.qoq_rmsnorm_quant(dummy, ctypes.c_void_p(16 * 1024 + 2), 4, 4096, f(1e-5), dummy, dummy, None,
+                               None) == 3
+    assert L.qoq_rmsnorm_quant(None, None, 0, 4096, f(1e-5), None, None, None, None) == 0        # M = 0
+    assert L.qoq_silu_mul_quant(dummy, 4, 0, dummy, dummy, None, None) == 1
+    assert L.qoq_silu_mul_quant(dummy, 4, 14340, dummy, dummy, None, None) == 2                  # I % 8
+    assert L.qoq_silu_mul_quant(dummy, 4, 14336, ctypes.c_void_p(16 * 1024 + 4), dummy, None, None) == 3
+    assert L.qoq_silu_mul_quant(dummy, 4, 14336, dummy, ctypes.c_void_p(16 * 1024 + 1), None, None) == 3
+    assert L.qoq_silu_mul_quant(None, 0, 14336, None, None, None, None) == 0
 
 
 def test_watchdog_selftest_validation_without_launch(L):

@@ -1,6 +1,7 @@
 // C-ABI entry points of libqoq.so (declared in include/qoq.h): argument
 // validation, size queries and dispatch to the kernels. Nothing here
 // allocates, frees or synchronises; every launch goes to the caller's stream.
+#include <cmath>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -71,6 +72,37 @@ qoq_status qoq_quantize_act_per_token(const void *X_fp16, int64_t M, int64_t K, 
     if (!aligned(X_fp16, 16) || !aligned(X8, 16) || !aligned(s_x_fp16, 2) || (rowsum && !aligned(rowsum, 4)))
         return QOQ_ERR_ALIGNMENT;
     return launch_act_quant(X_fp16, M, K, X8, s_x_fp16, rowsum, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? QOQ_OK
+               : QOQ_ERR_CUDA;
+}
+
+qoq_status qoq_rmsnorm_quant(const void *X_fp16, const void *gamma_fp16, int64_t M, int64_t K, float eps,
+                             int8_t *X8, void *s_x_fp16, int32_t *rowsum, void *stream) {
+    if (M < 0 || M > INT32_MAX || K <= 0) return QOQ_ERR_INVALID_ARG;
+    if (!(eps > 0.0f) || !(eps < INFINITY)) return QOQ_ERR_INVALID_ARG;
+    if (K % 8 != 0 || K > kMaxProducerWidth) return QOQ_ERR_UNSUPPORTED;
+    if (M == 0) return QOQ_OK;
+    if (X_fp16 == nullptr || gamma_fp16 == nullptr || X8 == nullptr || s_x_fp16 == nullptr)
+        return QOQ_ERR_INVALID_ARG;
+    if (!aligned(X_fp16, 16) || !aligned(gamma_fp16, 16) || !aligned(X8, 16) || !aligned(s_x_fp16, 2) ||
+        (rowsum && !aligned(rowsum, 4)))
+        return QOQ_ERR_ALIGNMENT;
+    return launch_rmsnorm_quant(X_fp16, gamma_fp16, M, K, eps, X8, s_x_fp16, rowsum,
+                                static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? QOQ_OK
+               : QOQ_ERR_CUDA;
+}
+
+qoq_status qoq_silu_mul_quant(const void *GU_fp16, int64_t M, int64_t I, int8_t *X8, void *s_x_fp16,
+                              int32_t *rowsum, void *stream) {
+    if (M < 0 || M > INT32_MAX || I <= 0) return QOQ_ERR_INVALID_ARG;
+    if (I % 8 != 0 || I > kMaxProducerWidth) return QOQ_ERR_UNSUPPORTED;
+    if (M == 0) return QOQ_OK;
+    if (GU_fp16 == nullptr || X8 == nullptr || s_x_fp16 == nullptr) return QOQ_ERR_INVALID_ARG;
+    if (!aligned(GU_fp16, 16) || !aligned(X8, 16) || !aligned(s_x_fp16, 2) || (rowsum && !aligned(rowsum, 4)))
+        return QOQ_ERR_ALIGNMENT;
+    return launch_silu_mul_quant(GU_fp16, M, I, X8, s_x_fp16, rowsum, static_cast<cudaStream_t>(stream)) ==
+                   cudaSuccess
                ? QOQ_OK
                : QOQ_ERR_CUDA;
 }

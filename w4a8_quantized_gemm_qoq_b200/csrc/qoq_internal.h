@@ -86,6 +86,13 @@ cudaError_t launch_act_quant(const void *X, int64_t M, int64_t K, int8_t *X8, vo
                              cudaStream_t stream);
 cudaError_t launch_weight_quant(const void *W, int64_t N, int64_t K, int group, void *blob,
                                 const BlobLayout &L, cudaStream_t stream);
+cudaError_t launch_rmsnorm_quant(const void *X, const void *gamma, int64_t M, int64_t K, float eps, int8_t *X8,
+                                 void *s_x, int32_t *rowsum, cudaStream_t stream);
+cudaError_t launch_silu_mul_quant(const void *GU, int64_t M, int64_t I, int8_t *X8, void *s_x, int32_t *rowsum,
+                                  cudaStream_t stream);
+
+// Row width limit of the fused producers (the FP32 row lives in shared memory).
+constexpr int kMaxProducerWidth = 32768;
 
 struct GemmArgs {
     const int8_t *X8;

@@ -13,8 +13,14 @@ activations are not available here, so these stand in for them):
     scale then lands near 10**u_m (the prefill workload uses 1e-3 .. 1e1).
   * W (weights, FP16, [N][K]): i.i.d. N(0, std), std = 0.02 (Llama shapes) or
     0.01 (Qwen shapes).
-Streams: numpy ``Generator(PCG64([seed, 1]))`` for W and
-``Generator(PCG64([seed, 2]))`` for X, so X and W can be drawn independently.
+  * gamma (RMSNorm weight, FP16, [K]): 1 + 0.1 * N(0, 1), the spread of a
+    trained normalisation weight around 1.
+  * GU (merged gate/up projection output, FP16, [M][2I]): gate half
+    N(0, 2^2) so that SiLU sees both its negative tail and its linear part,
+    up half N(0, 1); 4 outlier columns x20 in each half.
+Streams: numpy ``Generator(PCG64([seed, 1]))`` for W,
+``Generator(PCG64([seed, 2]))`` for X, ``[seed, 4]`` for gamma and
+``[seed, 5]`` for GU, so each can be drawn independently.
 """
 from __future__ import annotations
 
@@ -85,3 +91,21 @@ def sample_rows(M: int, count: int = 64, seed: int = 0) -> np.ndarray:
         keep = [0, M - 1] + [p for p in out if p not in (0, M - 1)]
         out = sorted(set(keep[:count]))
     return np.asarray(out, dtype=np.int64)
+
+
+def make_norm_weight(K: int, seed: int = 0) -> np.ndarray:
+    """FP16 RMSNorm weight [K] ~ 1 + 0.1 * N(0, 1)."""
+    rng = _rng(seed, 4)
+    return (1.0 + 0.1 * rng.standard_normal(K, dtype=np.float32)).astype(np.float16)
+
+
+def make_gate_up(M: int, I: int, seed: int = 0) -> np.ndarray:
+    """FP16 merged gate/up output [M][2I]: gate ~ N(0, 4), up ~ N(0, 1), each
+    half with 4 outlier columns x20."""
+    rng = _rng(seed, 5)
+    gu = rng.standard_normal((M, 2 * I), dtype=np.float32)
+    gu[:, :I] *= np.float32(2.0)
+    for half in (0, 1):
+        cols = half * I + rng.choice(I, size=min(N_OUTLIERS, I), replace=False)
+        gu[:, cols] *= np.float32(OUTLIER_GAIN)
+    return gu.astype(np.float16)

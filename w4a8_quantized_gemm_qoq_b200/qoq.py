@@ -41,6 +41,8 @@ def lib() -> ctypes.CDLL:
         vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t)
         L.qoq_quantize_act_per_token.argtypes = [vp, i64, i64, vp, vp, vp, vp]
         L.qoq_quantize_weights.argtypes = [vp, i64, i64, i32, vp, sz, vp]
+        L.qoq_rmsnorm_quant.argtypes = [vp, vp, i64, i64, ctypes.c_float, vp, vp, vp, vp]
+        L.qoq_silu_mul_quant.argtypes = [vp, i64, i64, vp, vp, vp, vp]
         L.qoq_w4a8_gemm.argtypes = [vp, vp, vp, i64, i64, i64, i32, vp, vp, sz, vp]
         L.qoq_gemm_fp16_out.argtypes = [vp, vp, vp, vp, i64, i64, i64, i32, vp, vp, sz, vp]
         L.qoq_watchdog_selftest.argtypes = [vp, i64, vp]
@@ -106,6 +108,40 @@ def quantize_act_per_token(X, X8=None, s_x=None, rowsum=None, stream=None):
     rowsum = torch.empty((M,), dtype=torch.int32, device=X.device) if rowsum is None else rowsum
     _check("qoq_quantize_act_per_token",
            lib().qoq_quantize_act_per_token(_ptr(X), M, K, _ptr(X8), _ptr(s_x), _ptr(rowsum), _stream(stream)))
+    return X8, s_x, rowsum
+
+
+def rmsnorm_quant(X, gamma, eps: float, X8=None, s_x=None, rowsum=None, stream=None):
+    """Fused RMSNorm + per-token INT8 quantisation: X [M][K] fp16, gamma [K]
+    fp16 -> (X8 int8 [M][K], s_x fp16 [M], rowsum int32 [M])."""
+    import torch
+    X = _cuda_tensor(X, torch.float16, "X")
+    gamma = _cuda_tensor(gamma, torch.float16, "gamma")
+    M, K = X.shape
+    if tuple(gamma.shape) != (K,):
+        raise ValueError("gamma must have shape (%d,)" % K)
+    X8 = torch.empty((M, K), dtype=torch.int8, device=X.device) if X8 is None else X8
+    s_x = torch.empty((M,), dtype=torch.float16, device=X.device) if s_x is None else s_x
+    rowsum = torch.empty((M,), dtype=torch.int32, device=X.device) if rowsum is None else rowsum
+    _check("qoq_rmsnorm_quant", lib().qoq_rmsnorm_quant(_ptr(X), _ptr(gamma), M, K, float(eps), _ptr(X8),
+                                                        _ptr(s_x), _ptr(rowsum), _stream(stream)))
+    return X8, s_x, rowsum
+
+
+def silu_mul_quant(GU, X8=None, s_x=None, rowsum=None, stream=None):
+    """Fused SiLU(gate) * up + per-token INT8 quantisation: GU [M][2I] fp16
+    (gate | up) -> (X8 int8 [M][I], s_x fp16 [M], rowsum int32 [M])."""
+    import torch
+    GU = _cuda_tensor(GU, torch.float16, "GU")
+    M, I2 = GU.shape
+    if I2 % 2:
+        raise ValueError("GU must have an even number of columns (gate | up)")
+    I = I2 // 2
+    X8 = torch.empty((M, I), dtype=torch.int8, device=GU.device) if X8 is None else X8
+    s_x = torch.empty((M,), dtype=torch.float16, device=GU.device) if s_x is None else s_x
+    rowsum = torch.empty((M,), dtype=torch.int32, device=GU.device) if rowsum is None else rowsum
+    _check("qoq_silu_mul_quant", lib().qoq_silu_mul_quant(_ptr(GU), M, I, _ptr(X8), _ptr(s_x), _ptr(rowsum),
+                                                          _stream(stream)))
     return X8, s_x, rowsum
 
 
