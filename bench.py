@@ -398,6 +398,7 @@ def run_gpu(args, rank, world, local_rank):
 
     e2e = run_e2e(args, probs, qoq, stream) if rank == 0 else None
     w8a8 = run_w8a8(probs, stream, gemm_only_us, max(K, 10)) if rank == 0 else None
+    producers = run_producers(stream, peaks) if rank == 0 and not args.no_context else None
     res = {
         "metric": METRIC, "value": round(world * ops_step / (step_ms * 1e-3) / 1e12, 3), "unit": "TOPS",
         "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup),
@@ -416,6 +417,7 @@ def run_gpu(args, rank, world, local_rank):
         "e2e": e2e,
         "per_gemm": per,
         "w8a8_context": w8a8,
+        "producers_context": producers,
     }
     return res
 
@@ -463,6 +465,72 @@ def run_shape(args):
     return {"shape": [M, N, K], "launches": args.steps, "us_per_launch": round(us, 3),
             "how": "one CUDA graph of back-to-back launches, replayed",
             "GBps": round(gemm_bytes(M, N, K) / us / 1e3, 1), "TOPS": round(gemm_ops(M, N, K) / us / 1e6, 2)}
+
+
+def run_producers(stream, peaks, reps=20):
+    """Context for the fused activation producers (not in the timed step):
+    RMSNorm + per-token INT8 on Llama-3-8B hidden rows (K = 4096) and
+    SiLU(gate) * up + per-token INT8 on its FFN rows (I = 14336), at decode and
+    prefill token counts, next to the stand-alone FP16 activation quantiser on
+    the same rows. Each case: `reps` launches back to back in one CUDA graph,
+    events around two replays; inputs of 64 MB and more alternate between two
+    copies (larger than L2 together), smaller ones stay L2-resident (a latency
+    figure). Algorithmic bytes: every input element read once, every code
+    written once, plus 6 bytes (scale, row sum) per row."""
+    import torch
+    from w4a8_quantized_gemm_qoq_b200 import qoq
+    dev = torch.device("cuda", torch.cuda.current_device())
+    out = []
+
+    def timed(fn, n_in):
+        with torch.cuda.stream(stream):
+            for i in range(max(2, n_in)):
+                fn(i)
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(reps):
+                fn(i)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            g.replay()
+            e0.record(stream)
+            g.replay()
+            g.replay()
+            e1.record(stream)
+        stream.synchronize()
+        del g
+        return 1000.0 * e0.elapsed_time(e1) / (2 * reps)
+
+    for kind, width, Ms in (("rmsnorm_quant", 4096, (16, 2048, 16384)), ("silu_mul_quant", 14336, (16, 2048, 16384))):
+        for M in Ms:
+            if kind == "rmsnorm_quant":
+                x = torch.from_numpy(inputs.make_activations(M, width, seed=M)).to(dev)
+                g = torch.from_numpy(inputs.make_norm_weight(width, seed=1)).to(dev)
+                nbytes_in = 2 * M * width
+            else:
+                x = torch.from_numpy(inputs.make_gate_up(M, width, seed=M)).to(dev)
+                nbytes_in = 4 * M * width
+            xs = [x, x.clone()] if nbytes_in >= 64e6 else [x]
+            X8 = torch.empty((M, width), dtype=torch.int8, device=dev)
+            s_x = torch.empty((M,), dtype=torch.float16, device=dev)
+            rs = torch.empty((M,), dtype=torch.int32, device=dev)
+            if kind == "rmsnorm_quant":
+                us = timed(lambda i: qoq.rmsnorm_quant(xs[i % len(xs)], g, 1e-5, X8, s_x, rs, stream=stream), len(xs))
+                fp16_in = xs
+            else:
+                us = timed(lambda i: qoq.silu_mul_quant(xs[i % len(xs)], X8, s_x, rs, stream=stream), len(xs))
+                fp16_in = [t[:, :width].contiguous() for t in xs]   # an FP16 row of the same width
+            aq_us = timed(lambda i: qoq.quantize_act_per_token(fp16_in[i % len(fp16_in)], X8, s_x, rs,
+                                                               stream=stream), len(fp16_in))
+            b = nbytes_in + M * width + 6 * M
+            out.append({"kernel": kind, "M": M, "width": width, "us": round(us, 3),
+                        "GBps": round(b / us / 1e3, 1), "frac_of_hbm": round(b / us / 1e3 / peaks["hbm"], 3),
+                        "act_quant_alone_us": round(aq_us, 3),
+                        "inputs": "two copies, > L2" if len(xs) > 1 else "L2-resident"})
+            del xs, fp16_in, x
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_w8a8(probs, stream, w4a8_us, reps):
@@ -627,6 +695,8 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-context", action="store_true",
+                    help="skip the fused-producer context measurements (not part of the timed step)")
     ap.add_argument("--shape", default=None,
                     help="MxNxK: one GEMM shape alone (act quant once, then --steps GEMM launches back to back); "
                          "small footprint for profiling")

@@ -12,8 +12,9 @@
 //   SiLU-gated:     h_k = (g_k / (1 + e^-g_k)) * u_k   (gate | up halves of a row)
 // then s = FP16(max_k |h| / 127), X8 = clamp(RNE(h / FP32(s)), -127, 127)
 // (0 where s == 0) and rowsum = sum_k X8. Every floating-point step is one
-// correctly rounded binary32 operation (__fdiv_rn, __fsqrt_rn, ...; no
-// contraction), the sum of squares is exact (128-bit integer accumulation,
+// correctly rounded binary32 operation (__fdiv_rn, __fsqrt_rn, ...; the
+// quantising division takes the exact reciprocal shortcut of qoq_device.cuh;
+// no contraction), the sum of squares is exact (128-bit integer accumulation,
 // then one rounding), and e^x is computed here from Cody and Waite's argument
 // reduction and the degree-7 Taylor polynomial, so that the codes these
 // floating-point values decide are reproducible bit for bit.
@@ -21,11 +22,13 @@
 // B200 layout: one 256-thread CTA per token row (memory-bound: each row is
 // read once from HBM and written once as INT8). Thread t owns the 8-element
 // chunks t, t+256, ...; the FP32 row h lives in shared memory between the
-// passes (each thread reads back only its own chunks).
+// passes, element i of chunk c at h[i * K/8 + c] so that a warp's accesses
+// fall in distinct banks (each thread reads back only its own chunks).
 #include <cuda_fp16.h>
 
 #include "qoq_device.cuh"
 #include "qoq_internal.h"
+#include "quant_math.cuh"
 
 namespace qoq {
 
@@ -172,26 +175,28 @@ __device__ __forceinline__ int block_sum(int v, int *red) {
 __device__ __forceinline__ float half_lo(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w & 0xFFFFu))); }
 __device__ __forceinline__ float half_hi(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w >> 16))); }
 
-// Quantise the FP32 row h (shared memory, this thread's chunks) and write the
-// codes, the scale and the row sum of token m.
+// Quantise the FP32 row h (shared memory, element i of chunk c at
+// h[i * K/8 + c]; this thread's chunks) and write the codes, the scale and the
+// row sum of token m.
 __device__ __forceinline__ void quantize_row(const float *h, int K, float amax_row, int64_t m, int8_t *X8,
                                              __half *s_x, int32_t *rowsum, int *red_i) {
-    __shared__ float s_shared;
+    __shared__ float s_shared, inv_shared;
     if (threadIdx.x == 0) {
         const __half sh = __float2half_rn(__fdiv_rn(amax_row, 127.0f));
         s_x[m] = sh;
         s_shared = __half2float(sh);
+        inv_shared = __frcp_rn(__half2float(sh));
     }
     __syncthreads();
-    const float s = s_shared;
+    const float s = s_shared, inv = inv_shared;
+    const int nc = K / 8;
     int8_t *out = X8 + m * K;
     int sum = 0;
     for (int c = threadIdx.x; c * 8 < K; c += kProdThreads) {
         uint32_t packed[2] = {0u, 0u};
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            int q = 0;
-            if (s != 0.0f) q = max(-127, min(127, __float2int_rn(__fdiv_rn(h[c * 8 + i], s))));
+            const int q = quant_code_recip(h[i * nc + c], s, inv, 127);
             sum += q;
             packed[i >> 2] |= (uint32_t)(q & 0xFF) << (8 * (i & 3));
         }
@@ -221,6 +226,7 @@ __global__ void __launch_bounds__(kProdThreads) rmsnorm_quant_kernel(const __hal
     griddep_launch_dependents();
     const int64_t m = blockIdx.x;
     const __half *row = X + m * K;
+    const int nc = K / 8;   // chunks per row; element i of chunk c sits at h[i * nc + c] (no bank conflicts)
 
     // Pass 1: the row's exact sum of squares; keep x (FP32) in shared memory.
     U128 acc{0ull, 0ull};
@@ -231,8 +237,8 @@ __global__ void __launch_bounds__(kProdThreads) rmsnorm_quant_kernel(const __hal
         for (int i = 0; i < 4; ++i) {
             add_square(acc, w[i] & 0xFFFFu);
             add_square(acc, w[i] >> 16);
-            h[c * 8 + 2 * i] = half_lo(w[i]);
-            h[c * 8 + 2 * i + 1] = half_hi(w[i]);
+            h[(2 * i) * nc + c] = half_lo(w[i]);
+            h[(2 * i + 1) * nc + c] = half_hi(w[i]);
         }
     }
     const U128 S = block_sum128(acc, red128);
@@ -251,10 +257,10 @@ __global__ void __launch_bounds__(kProdThreads) rmsnorm_quant_kernel(const __hal
         const uint32_t g[4] = {gu.x, gu.y, gu.z, gu.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const float h0 = __fmul_rn(__fdiv_rn(h[c * 8 + 2 * i], r), half_lo(g[i]));
-            const float h1 = __fmul_rn(__fdiv_rn(h[c * 8 + 2 * i + 1], r), half_hi(g[i]));
-            h[c * 8 + 2 * i] = h0;
-            h[c * 8 + 2 * i + 1] = h1;
+            const float h0 = __fmul_rn(__fdiv_rn(h[(2 * i) * nc + c], r), half_lo(g[i]));
+            const float h1 = __fmul_rn(__fdiv_rn(h[(2 * i + 1) * nc + c], r), half_hi(g[i]));
+            h[(2 * i) * nc + c] = h0;
+            h[(2 * i + 1) * nc + c] = h1;
             amax = fmaxf(amax, fmaxf(fabsf(h0), fabsf(h1)));
         }
     }
@@ -272,6 +278,7 @@ __global__ void __launch_bounds__(kProdThreads) silu_mul_quant_kernel(const __ha
     griddep_wait();
     griddep_launch_dependents();
     const int64_t m = blockIdx.x;
+    const int nc = I / 8;   // chunks per row; element i of chunk c sits at h[i * nc + c]
     const __half *gate = GU + m * 2 * (int64_t)I;
     const __half *up = gate + I;
     float amax = 0.0f;
@@ -289,7 +296,7 @@ __global__ void __launch_bounds__(kProdThreads) silu_mul_quant_kernel(const __ha
                 const float e = exp_cw(-gf);
                 const float sg = __fdiv_rn(gf, __fadd_rn(1.0f, e));
                 const float hv = __fmul_rn(sg, uf);
-                h[c * 8 + 2 * i + j] = hv;
+                h[(2 * i + j) * nc + c] = hv;
                 amax = fmaxf(amax, fabsf(hv));
             }
         }

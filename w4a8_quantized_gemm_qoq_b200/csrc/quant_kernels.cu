@@ -15,6 +15,7 @@
 
 #include "qoq_device.cuh"
 #include "qoq_internal.h"
+#include "quant_math.cuh"
 
 namespace qoq {
 
@@ -51,7 +52,7 @@ __global__ void __launch_bounds__(kActThreads) act_quant_kernel(const __half *__
                                                                  int32_t *__restrict__ rowsum) {
     __shared__ float red_f[kActThreads / 32];
     __shared__ int red_i[kActThreads / 32];
-    __shared__ float s_shared;
+    __shared__ float s_shared, inv_shared;
     // X may come from the previous kernel in the stream; release the next one
     // (the GEMM) so its set-up and weight copies overlap this kernel.
     griddep_wait();
@@ -96,9 +97,10 @@ __global__ void __launch_bounds__(kActThreads) act_quant_kernel(const __half *__
         __half sh = __float2half_rn(__fdiv_rn(a, 127.0f));
         s_x[m] = sh;
         s_shared = __half2float(sh);
+        inv_shared = __frcp_rn(__half2float(sh));
     }
     __syncthreads();
-    const float s = s_shared;
+    const float s = s_shared, inv = inv_shared;
 
     int sum = 0;
     int8_t *out = X8 + m * K;
@@ -109,7 +111,7 @@ __global__ void __launch_bounds__(kActThreads) act_quant_kernel(const __half *__
         for (int i = 0; i < 4; ++i) {
             const float lo = __half2float(__ushort_as_half((unsigned short)(w[i] & 0xFFFFu)));
             const float hi = __half2float(__ushort_as_half((unsigned short)(w[i] >> 16)));
-            const int q0 = quant_code(lo, s, 127), q1 = quant_code(hi, s, 127);
+            const int q0 = quant_code_recip(lo, s, inv, 127), q1 = quant_code_recip(hi, s, inv, 127);
             sum += q0 + q1;
             const uint32_t pair = ((uint32_t)(q0 & 0xFF) | ((uint32_t)(q1 & 0xFF) << 8)) << (16 * (i & 1));
             if (i < 2)
