@@ -444,6 +444,7 @@ def run_shape(args):
     ws = qoq.Workspace.for_shape(M, N, K, GROUP, dev)
     Y = torch.empty((M, N), dtype=torch.float16, device=dev)
     stream = torch.cuda.Stream(dev)
+    stream.wait_stream(torch.cuda.current_stream())   # inputs and the zeroed workspace were made on the default stream
     with torch.cuda.stream(stream):
         for i in range(max(1, args.warmup)):
             qoq.gemm_fp16_out(X8, s_x, blobs[i % copies], N, K, GROUP, rowsum=rs, ws=ws, Y=Y)
@@ -483,6 +484,7 @@ def run_producers(stream, peaks, reps=20):
     out = []
 
     def timed(fn, n_in):
+        stream.wait_stream(torch.cuda.current_stream())   # inputs were made on the default stream
         with torch.cuda.stream(stream):
             for i in range(max(2, n_in)):
                 fn(i)
@@ -551,6 +553,7 @@ def run_w8a8(probs, stream, w4a8_us, reps):
             xs.append(torch.randint(-127, 128, (m, p.K), dtype=torch.int8, device=dev, generator=g))
             ys.append(torch.empty((m, p.N), dtype=torch.int32, device=dev))
         graph = torch.cuda.CUDAGraph()
+        stream.wait_stream(torch.cuda.current_stream())   # operands were drawn on the default stream
         with torch.cuda.stream(stream):
             for x, w, y in zip(xs, ws, ys):     # warm-up outside capture (library handles, kernels)
                 torch._int_mm(x, w.t(), out=y)
@@ -598,6 +601,7 @@ def run_e2e(args, probs, qoq, stream):
             c.copy_(p.Y, non_blocking=True)
 
     steps = max(1, args.steps)
+    stream.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(stream):
         for _ in range(3):
             once()

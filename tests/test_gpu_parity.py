@@ -176,6 +176,7 @@ def test_graph_replays_are_bit_identical():
             qoq.gemm_fp16_out(p["X8"], p["s_x"], p["blob"], p["N"], p["K"], 128, rowsum=p["rs"], ws=p["ws"], Y=p["Y"])
 
     stream = t.cuda.Stream()
+    stream.wait_stream(t.cuda.current_stream())   # inputs and zeroed workspaces were made on the default stream
     with t.cuda.stream(stream):
         step()
     stream.synchronize()

@@ -470,10 +470,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     bool seg_done = false;
                     while (!seg_done) {
                         if (!ALT || (unit & 1) == k) {
-                            // The token tile (shared memory) and the
-                            // dequantised weights (TMEM) of this unit.
-                            ok = wait_bounded(&ctl->full[s], ph, wd, kSiteMmaOperands, 2 * unit) &&
-                                 wait_bounded(&ctl->a_full[s], ph, wd, kSiteMmaOperands, 2 * unit + 1);
+                            // The dequantised weights (TMEM) of this unit.
+                            // One wait covers the token tile too: the dequant
+                            // warps arrive on a_full[s] only after their own
+                            // wait on full[s], which counts the token tile's
+                            // bytes, and the arrivals order that completion
+                            // before this thread's MMAs. Each wait of an
+                            // issuing thread costs it hundreds of cycles, so
+                            // the issuer waits once per unit.
+                            ok = wait_bounded(&ctl->a_full[s], ph, wd, kSiteMmaOperands, unit);
                             if (!ok) break;
                             tc_fence_after();
                             const uint32_t a_tmem = tmem_base + (uint32_t)(C::kACol0 + s * KB * 32);
