@@ -55,8 +55,7 @@ constexpr int kThreads = 512;            // 16 warps
 constexpr int kWarpProducer = 0;
 constexpr int kWarpMma = 1;             // warps 1, 2: the two MMA issuers
 constexpr int kIssuers = 2;
-constexpr int kWarpDequant0 = 4;         // warps 4..11: two dequant warpgroups
-constexpr int kWarpEpilogue = 12;        // warps 12..15
+constexpr int kWarpDequant0 = 4;         // warps 4..: the dequant warpgroups, then the epilogue warpgroups
 constexpr uint64_t kDrainNs = 100ull * 1000ull * 1000ull;   // 100 ms
 
 template <int TOK, int MODE>
@@ -71,7 +70,7 @@ struct GemmCfg {
     static constexpr int kWBytes = kKB * kWTile;
     static constexpr int kStageBytes = (kXBytes + kWBytes + 1023) / 1024 * 1024;
     static constexpr int kSmemLimit = 232448;                   // 227 KB per CTA
-    static constexpr int kReserve = 12288;                      // alignment slack + control block
+    static constexpr int kReserve = 20480;                      // alignment slack + control block
     // Two MMA issuers. Up to 64-token tiles (kAlt), issuer j takes the units
     // of index parity j (those its dequant warpgroup serves) into its own
     // accumulator, and the epilogue adds the two; wider tiles have no TMEM for
@@ -81,6 +80,20 @@ struct GemmCfg {
     static constexpr int kAccCols = kAlt ? 2 * TOK : TOK;   // TMEM columns per accumulator buffer
     static constexpr int kAccBufs = (TOK == 64 || TOK == 256) ? 1 : 2;
     static constexpr int kACol0 = kAccBufs * kAccCols;
+    // 256-token tiles have no second accumulator buffer. Each issuer's half of
+    // the token columns goes to the epilogue and back on its own barrier pair
+    // (acc_full[k], acc_empty[k]), so issuer 0 starts the next tile as soon as
+    // the epilogue has read the first half.
+    static constexpr bool kHalves = TOK == 256;
+    // Warpgroups after the producer/issuer warps (12 warps): two dequant and
+    // one epilogue warpgroup, except for 256-token tiles, whose main loop needs
+    // one k-tile decoded per 512 tensor-core cycles (one warpgroup keeps up)
+    // and whose epilogue is not overlapped with the next tile's main loop:
+    // there one dequant warpgroup and two epilogue warpgroups, one per half.
+    static constexpr int kDqGroups = kHalves ? 1 : 2;
+    static constexpr int kEpiGroups = kHalves ? 2 : 1;
+    static constexpr int kWarpEpi0 = kWarpDequant0 + 4 * kDqGroups;
+    static_assert(kWarpEpi0 + 4 * kEpiGroups == kThreads / 32, "warp roles must fill the CTA");
     // One CTA per SM (shared memory use guarantees it), so the CTA takes all
     // 512 TMEM columns: accumulators first, then one A buffer per stage
     // (32 columns per dequantised 128x128 k-tile).
@@ -129,7 +142,7 @@ struct SharedCtl {
     int32_t tok_rowsum[256];
     // Per epilogue warp, two alternating blocks of one step's FP16 outputs
     // (16 tokens x 32 weight rows), the source of the TMA output stores.
-    alignas(128) __half out_stage[4][2][16 * 32];
+    alignas(128) __half out_stage[8][2][16 * 32];
 };
 static_assert(sizeof(SharedCtl) + 1023 <= GemmCfg<16, 0>::kReserve, "control block outgrows the reserve");
 
@@ -275,6 +288,54 @@ __device__ __forceinline__ void store_outputs_fp16(const CUtensorMap *tmap_y, co
     }
 }
 
+// FP16 values of CH tokens of this lane's weight row, packed in token pairs
+// (pk[t]: token 2t low, 2t + 1 high); the same arithmetic as the store above.
+template <int CH, int MODE>
+__device__ __forceinline__ void convert_fp16(const uint32_t (&v)[CH], uint32_t *pk, float col_scale, int col_zero,
+                                             const float *sx, const int32_t *rs) {
+    float scale[CH];
+#pragma unroll
+    for (int q = 0; q < CH / 4; ++q) {
+        const float4 f = reinterpret_cast<const float4 *>(sx)[q];
+        scale[4 * q] = f.x;
+        scale[4 * q + 1] = f.y;
+        scale[4 * q + 2] = f.z;
+        scale[4 * q + 3] = f.w;
+    }
+#pragma unroll
+    for (int j = 0; j < CH; j += 2) {
+        int32_t a0 = (int32_t)v[j], a1 = (int32_t)v[j + 1];
+        if (MODE == 1) {
+            a0 -= col_zero * rs[j];
+            a1 -= col_zero * rs[j + 1];
+        }
+        const float y0 = __fmul_rn(__int2float_rn(a0), __fmul_rn(scale[j], col_scale));
+        const float y1 = __fmul_rn(__int2float_rn(a1), __fmul_rn(scale[j + 1], col_scale));
+        const __half2 h = __floats2half2_rn(y0, y1);
+        pk[j / 2] = *reinterpret_cast<const uint32_t *>(&h);
+    }
+}
+
+// The same store for 16 tokens already converted: pk[t] holds this lane's
+// weight row at tokens 2t (low half) and 2t + 1 (high half).
+__device__ __forceinline__ void store_packed_fp16(const CUtensorMap *tmap_y, const uint32_t *pk, int64_t m_first,
+                                                  int n_warp, int lane, __half *stage) {
+    if (lane == 0) bulk_wait_group_read<1>();
+    __syncwarp();
+    unsigned short *st = reinterpret_cast<unsigned short *>(stage);
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+        st[(2 * t) * 32 + lane] = (unsigned short)(pk[t] & 0xFFFFu);
+        st[(2 * t + 1) * 32 + lane] = (unsigned short)(pk[t] >> 16);
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        tma_store_2d(tmap_y, stage, n_warp, (int)m_first);
+        bulk_commit_group();
+    }
+}
+
 // INT32 accumulators (after the per-channel zero-point term) of CH tokens.
 template <int CH, int MODE>
 __device__ __forceinline__ void store_outputs_i32(const GemmParams &p, const uint32_t (&v)[CH], int64_t m_first,
@@ -314,7 +375,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     qoq_gemm_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ CUtensorMap tmap_x,
                     const __grid_constant__ CUtensorMap tmap_y) {
     using C = GemmCfg<TOK, MODE>;
-    constexpr int CH = (TOK < 32 || C::kAlt) ? 16 : 32;   // epilogue TMEM chunk (16 when two accumulators are summed)
     constexpr int S = C::kStages;
     constexpr int KB = C::kKB;
     extern __shared__ uint8_t smem_raw[];
@@ -333,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&ctl->a_full[s], 4);   // the four warps of one dequant warpgroup
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&ctl->acc_full[b], kIssuers);
+            mbar_init(&ctl->acc_full[b], C::kHalves ? 1 : kIssuers);
             mbar_init(&ctl->acc_empty[b], 4);
         }
         mbar_init(&ctl->final_bar[0], 1);
@@ -350,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ctl->abort_flag = 1;   // reported on the status word after griddepcontrol.wait
     }
     if (warp == kWarpProducer && lane == 0) prefetch_tensormap(&tmap_x);
-    if (warp == kWarpEpilogue && lane == 0 && p.fp16_out) prefetch_tensormap(&tmap_y);
+    if (warp == C::kWarpEpi0 && lane == 0 && p.fp16_out) prefetch_tensormap(&tmap_y);
     if (warp == kWarpMma) {
         tmem_alloc(&ctl->tmem_base, C::kTmemCols);
         tmem_relinquish();
@@ -463,7 +523,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 while (ok && !cur.done()) {
                     const int buf = seg % C::kAccBufs;
                     const uint32_t aph = (uint32_t)(seg / C::kAccBufs) & 1u;
-                    ok = wait_bounded(&ctl->acc_empty[buf], aph ^ 1u, wd, kSiteMmaAccEmpty, seg);
+                    const int bi = C::kHalves ? k : buf;   // this issuer's accumulator barrier pair
+                    ok = wait_bounded(&ctl->acc_empty[bi], aph ^ 1u, wd, kSiteMmaAccEmpty, seg);
                     if (!ok) break;
                     const uint32_t d_tmem = tmem_base + (uint32_t)(buf * C::kAccCols + k * (ALT ? TOK : TOK / 2));
                     uint32_t acc = 0u;   // this issuer's first MMA of the segment overwrites its accumulator
@@ -502,7 +563,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         seg_done = cur.advance();
                     }
                     if (!ok) break;
-                    tc_commit(&ctl->acc_full[buf]);
+                    tc_commit(&ctl->acc_full[bi]);
                     ++seg;
                 }
                 // Every MMA must have completed before tensor memory is freed.
@@ -510,12 +571,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 wait_drain(&ctl->final_bar[k], 0, kDrainNs);
             }
             __syncwarp();
-        } else if (warp >= kWarpDequant0 && warp < kWarpEpilogue) {
+        } else if (warp >= kWarpDequant0 && warp < C::kWarpEpi0) {
             // ------------------------------------------------ dequant
-            // Warpgroup g takes the units i with i % 2 == g, i.e. (the stage
-            // count being even) always the same stages: it waits on every phase
-            // of those stage barriers and on no others, so parity waits cannot
-            // alias. Thread (quarter, lane) decodes weight row r of each k-tile.
+            // With two warpgroups, warpgroup g takes the units i with
+            // i % 2 == g, i.e. (the stage count being even) always the same
+            // stages: it waits on every phase of those stage barriers and on no
+            // others, so parity waits cannot alias. A single warpgroup takes
+            // every unit. Thread (quarter, lane) decodes weight row r of each
+            // k-tile.
             const int g = (warp - kWarpDequant0) >> 2;
             const int quarter = warp & 3;                    // TMEM lanes 32q .. 32q+31
             const int r = quarter * 32 + lane;               // weight row in the tile
@@ -531,7 +594,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     s = 0;
                     ph ^= 1u;
                 }
-                if ((i & 1) != g) continue;
+                if (C::kDqGroups == 2 && (i & 1) != g) continue;
                 // full[s] for this unit implies the producer saw freed[s] for
                 // the unit S earlier, i.e. TMEM A buffer s is no longer read.
                 const bool ok = __all_sync(0xffffffffu, wait_bounded(&ctl->full[unit_s], unit_ph, wd, kSiteDequantFull, i));
@@ -583,12 +646,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lane == 0) mbar_arrive(&ctl->a_full[unit_s]);
                 __syncwarp();
             }
-        } else if (warp >= kWarpEpilogue) {
+        } else if (warp >= C::kWarpEpi0) {
             // ------------------------------------------------ epilogue
+            // kEpiGroups warpgroups. Each reads its share of the accumulator's
+            // parts: with two (256-token tiles), warpgroup e takes issuer e's
+            // half of the token columns, waiting on acc_full[e] and handing it
+            // back on acc_empty[e]; with one, the whole buffer. Named barrier
+            // 1 + e syncs one warpgroup, barrier 3 all epilogue warps.
+            constexpr int NEPI = 128 * C::kEpiGroups;
+            constexpr int kBarAll = C::kEpiGroups == 2 ? 3 : 1;
+            const int e = (warp - C::kWarpEpi0) >> 2;
             const int quarter = warp & 3;
             const int r = quarter * 32 + lane;
+            const int te = threadIdx.x - (C::kWarpEpi0 + 4 * e) * 32;   // thread within the warpgroup
             const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-            const bool leader = (threadIdx.x == kWarpEpilogue * 32);
+            const bool leader = (threadIdx.x == C::kWarpEpi0 * 32);
+            const bool poller = (warp == C::kWarpEpi0);
             griddep_wait();   // outputs, scales, row sums and workspace belong to the previous kernel until now
             UnitCursor<KB> cur;
             cur.init(blockIdx.x, G, waves, b0, b1, KT, p.NT);
@@ -620,25 +693,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t c_first = blockIdx.x + 1;
                 const uint32_t c_last =
                     (!owner || kt_hi == KT) ? blockIdx.x : cta_of(tile_b + (uint32_t)KT - 1 - p.sk_base, BS, G);
-                constexpr int CO = 16;   // owner: token columns per step
+                constexpr int CO = 16;   // token columns per step
+                // The parts this warpgroup reads: [h_lo, h_hi) of NP, PART columns each.
+                constexpr int NP = C::kHalves ? 2 : 1;
+                constexpr int PART = TOK / NP;
+                const int h_lo = C::kEpiGroups == 2 ? e : 0, h_hi = C::kEpiGroups == 2 ? e + 1 : NP;
                 const bool polls = c_last >= c_first;
                 float col_scale = 0.0f;
                 int col_zero = 0;
                 if (owner) {
                     // Inputs that depend neither on the accumulator nor on the
                     // contributors, fetched first: the weight row's scale (and
-                    // zero point), and the tile's token scales (and row sums),
-                    // staged in shared memory once per tile. The previous
-                    // segment's readers have passed its closing barrier; the
-                    // barrier after the accumulator wait orders these stores
-                    // before every read. While contributors are polled, the
-                    // polling warp takes no part in the staging.
+                    // zero point), and the token scales (and row sums) of this
+                    // warpgroup's columns, staged in shared memory once per tile.
+                    // The previous segment's readers have passed its closing
+                    // barrier; the barrier after the accumulator wait orders
+                    // these stores before every read. While contributors are
+                    // polled, the polling warp takes no part in the staging.
                     col_scale = __half2float(reinterpret_cast<const __half *>(p.blob + p.off_scale)[n]);
                     if (MODE == 1)
                         col_zero = __half2int_rn(reinterpret_cast<const __half *>(p.blob + p.off_zero)[n]);
-                    if (!polls || warp != kWarpEpilogue) {
-                        const int t0 = threadIdx.x - kWarpEpilogue * 32;
-                        for (int j = polls ? t0 - 32 : t0; j < TOK; j += polls ? 96 : 128) {
+                    if (!polls || !poller) {
+                        const bool skip = polls && e == 0;   // warp 0 of this warpgroup polls
+                        const int jend = h_hi * PART;
+                        for (int j = h_lo * PART + (skip ? te - 32 : te); j < jend; j += skip ? 96 : 128) {
                             const int64_t m = m0 + j < p.M ? m0 + j : p.M - 1;
                             ctl->tok_scale[j] = p.fp16_out ? __half2float(p.s_x[m]) : 0.0f;
                             if (MODE == 1) ctl->tok_rowsum[j] = p.rowsum[m];
@@ -649,65 +727,99 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // Contributors reach their share of the tile first, so their
                     // flags are usually up before this CTA's own accumulator is:
                     // poll them now (lanes of the first epilogue warp in
-                    // parallel, acquire loads). The barrier orders everyone's
-                    // partial-sum reads after the polls.
+                    // parallel). The barrier orders everyone's partial-sum reads
+                    // after the polls.
                     bool got = true;
-                    if (warp == kWarpEpilogue) {
+                    if (poller) {
                         for (uint32_t c = c_first + (uint32_t)lane; c <= c_last && got; c += 32)
                             got = wait_flag_bounded(p.flags + c, wd, (int)c);
                         got = __all_sync(0xffffffffu, got);
                     }
-                    if (named_bar_any(1, 128, !got)) break;
+                    if (named_bar_any(kBarAll, NEPI, !got)) break;
                 }
-                // Every lane spins on its own; the vote reconverges the warp
-                // before the named barrier, and all four epilogue warps leave
-                // together (the shared-tile paths below meet at named barriers).
-                const bool ok = __all_sync(0xffffffffu, wait_bounded(&ctl->acc_full[buf], aph, wd, kSiteEpilogueAcc, seg));
-                if (named_bar_any(1, 128, !ok)) break;
-                tc_fence_after();
+                // Each part is handed back to its issuer right after its last
+                // TMEM load. Every lane spins on its own; the votes reconverge
+                // the warps before the named barriers, and all epilogue warps
+                // leave together.
+                const int live_end = (m_live + CO - 1) / CO * CO;   // token columns read and stored
                 const uint32_t acc_addr = tmem_base + lane_addr + (uint32_t)(buf * C::kAccCols + prim * TOK);
                 const uint32_t acc2_addr = tmem_base + lane_addr + (uint32_t)(buf * C::kAccCols + (prim ^ 1) * TOK);
-                if (!owner) {
-                    // Contributor: this tile's first k-tile belongs to an earlier
-                    // CTA. Store the partial sums in this CTA's slot, raise its flag.
-                    int32_t *part = p.partials + (long long)blockIdx.x * TOK * kTileN;
-#pragma unroll 1
-                    for (int c0 = 0; c0 < (m_live + CH - 1) / CH * CH; c0 += CH) {
-                        uint32_t v[CH];
-                        tmem_load<CH>(acc_addr + (uint32_t)c0, v);
-                        if (two) add_second<CH>(acc2_addr + (uint32_t)c0, v);
-#pragma unroll
-                        for (int j = 0; j < CH; ++j)
-                            if (c0 + j < m_live) part[(c0 + j) * kTileN + r] = (int32_t)v[j];
+                int32_t *slot = p.partials + (long long)blockIdx.x * TOK * kTileN;   // a contributor's partial tile
+                bool fail = false;
+                for (int h = h_lo; h < h_hi && !fail; ++h) {
+                    const int bi = C::kHalves ? h : buf;
+                    const uint32_t fph = C::kHalves ? (uint32_t)(seg & 1) : aph;
+                    const bool ok =
+                        __all_sync(0xffffffffu, wait_bounded(&ctl->acc_full[bi], fph, wd, kSiteEpilogueAcc, seg));
+                    if (named_bar_any(1 + e, 128, !ok)) {
+                        fail = true;
+                        break;
                     }
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&ctl->acc_empty[buf]);
-                    // The barrier orders every thread's partial-sum stores
-                    // before the leader's release store of the flag (release is
-                    // cumulative), so the owner's acquire load sees them all.
-                    named_bar_sync(1, 128);
-                    if (leader) st_release_gpu(p.flags + blockIdx.x, 1);
-                    __syncwarp();
-                } else {
-                    // Owner: add the contributors' partial sums, run the
-                    // epilogue, clear their flags.
-                    const int c_end = (m_live + CO - 1) / CO * CO;
+                    tc_fence_after();
+                    const int c_lo = h * PART;
+                    const int c_hi = live_end < c_lo + PART ? live_end : c_lo + PART;
+                    if (c_hi <= c_lo) {   // no token in this part: hand it back at once
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&ctl->acc_empty[bi]);
+                        continue;
+                    }
+                    if (C::kHalves && owner && !polls && p.fp16_out) {
+                        // A whole tile of this CTA (no partial sums): convert the
+                        // part to FP16 in registers, hand the accumulator back,
+                        // then store while the issuer runs the next tile.
+                        constexpr int NS = PART / CO;
+                        uint32_t pk[NS][CO / 2];
+#pragma unroll
+                        for (int q = 0; q < NS; ++q) {
+                            const int c0 = c_lo + q * CO;
+                            if (c0 < c_hi) {
+                                uint32_t v[CO];
+                                tmem_load<CO>(acc_addr + (uint32_t)c0, v);
+                                if (c0 + CO >= c_hi) {
+                                    tc_fence_before();
+                                    __syncwarp();
+                                    if (lane == 0) mbar_arrive(&ctl->acc_empty[bi]);
+                                }
+                                convert_fp16<CO, MODE>(v, pk[q], col_scale, col_zero, ctl->tok_scale + c0,
+                                                       ctl->tok_rowsum + c0);
+                            }
+                        }
+#pragma unroll
+                        for (int q = 0; q < NS; ++q) {
+                            const int c0 = c_lo + q * CO;
+                            if (c0 < c_hi) {
+                                store_packed_fp16(&tmap_y, pk[q], m0 + c0, n - lane, lane,
+                                                  ctl->out_stage[warp - C::kWarpEpi0][obuf]);
+                                obuf ^= 1;
+                            }
+                        }
+                        continue;
+                    }
 #pragma unroll 1
-                    for (int c0 = 0; c0 < c_end; c0 += CO) {
+                    for (int c0 = c_lo; c0 < c_hi; c0 += CO) {
                         uint32_t v[CO];
                         tmem_load<CO>(acc_addr + (uint32_t)c0, v);
                         if (two) add_second<CO>(acc2_addr + (uint32_t)c0, v);
-                        if (c0 + CO >= c_end) {
+                        if (c0 + CO >= c_hi) {
                             tc_fence_before();
                             __syncwarp();
-                            if (lane == 0) mbar_arrive(&ctl->acc_empty[buf]);
+                            if (lane == 0) mbar_arrive(&ctl->acc_empty[bi]);
                         }
-                        // Contributors' partial sums: eight contributors per L2
-                        // round trip when at most four columns hold tokens, four
-                        // otherwise. Columns past the live ones hold stale values
-                        // (contributors store only the live ones); they belong to
-                        // no token and are never stored.
+                        if (!owner) {
+                            // Contributor: the live token columns of the partial
+                            // sums go to this CTA's slot.
+#pragma unroll
+                            for (int j = 0; j < CO; ++j)
+                                if (c0 + j < m_live) slot[(c0 + j) * kTileN + r] = (int32_t)v[j];
+                            continue;
+                        }
+                        // Owner: add the contributors' partial sums: eight
+                        // contributors per L2 round trip when at most four
+                        // columns hold tokens, four otherwise. Columns past the
+                        // live ones hold stale values (contributors store only
+                        // the live ones); they belong to no token and are never
+                        // stored.
                         if (m_live <= 4) {
 #pragma unroll 1
                             for (uint32_t c = c_first; c <= c_last; c += 8) {
@@ -746,20 +858,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (p.fp16_out) {
                             store_outputs_fp16<CO, MODE>(&tmap_y, v, m0 + c0, n - lane, lane, col_scale, col_zero,
                                                          ctl->tok_scale + c0, ctl->tok_rowsum + c0,
-                                                         ctl->out_stage[quarter][obuf]);
+                                                         ctl->out_stage[warp - C::kWarpEpi0][obuf]);
                             obuf ^= 1;
                         } else {
                             store_outputs_i32<CO, MODE>(p, v, m0 + c0, n, col_zero, ctl->tok_rowsum + c0);
                         }
                     }
-                    // Closing barrier: every read of the staged scales (and of
-                    // the contributors' partial sums) is done.
-                    named_bar_sync(1, 128);
-                    if (c_last >= c_first) {
-                        if (warp == kWarpEpilogue)
-                            for (uint32_t c = c_first + (uint32_t)lane; c <= c_last; c += 32) p.flags[c] = 0;
-                        __syncwarp();
-                    }
+                }
+                // Closing barrier of the segment (all epilogue warps): every
+                // read of the staged scales and of the contributors' partial
+                // sums is done, and (contributor) every partial-sum store comes
+                // before the leader's release store of the flag (release is
+                // cumulative, so the owner's acquire sees them all). It also
+                // carries the failure vote, so that all warps leave together.
+                if (named_bar_any(kBarAll, NEPI, fail)) break;
+                if (!owner) {
+                    if (leader) st_release_gpu(p.flags + blockIdx.x, 1);
+                    __syncwarp();
+                } else if (polls && poller) {
+                    for (uint32_t c = c_first + (uint32_t)lane; c <= c_last; c += 32) p.flags[c] = 0;
+                    __syncwarp();
                 }
                 ++seg;
             }
