@@ -101,10 +101,10 @@ struct GemmCfg {
     static constexpr int kStagesSmem = (kSmemLimit - kReserve) / kStageBytes;
     static constexpr int kStagesTmem = (kTmemCols - kACol0) / (kKB * 32);
     static constexpr int kStagesMin = kStagesSmem < kStagesTmem ? kStagesSmem : kStagesTmem;
-    // Even, so that stage s is always dequantised by warpgroup s % 2 (the two
-    // warpgroups take alternate units); each warpgroup then waits on every
-    // phase of the stages it reads.
-    static constexpr int kStages = (kStagesMin > 16 ? 16 : kStagesMin) & ~1;
+    // With two dequant warpgroups even, so that stage s is always dequantised
+    // by warpgroup s % 2 (they take alternate units); each warpgroup then waits
+    // on every phase of the stages it reads. One warpgroup takes every stage.
+    static constexpr int kStages = (kStagesMin > 16 ? 16 : kStagesMin) & (kHalves ? ~0 : ~1);
     static constexpr int kSmemBytes = kStages * kStageBytes + kReserve;
     static_assert(kStages >= 4, "pipeline too shallow");
     static_assert(kACol0 + kStages * kKB * 32 <= kTmemCols, "TMEM over-subscribed");
@@ -122,6 +122,7 @@ struct GemmParams {
     int32_t *partials;      // [grid][TOK][128]: contributor c's partial sums
     int M, N, K, group;
     int NT, KT, MT;
+    int GM;                 // token tiles per group of the tile order
     int grid;
     uint32_t total_blocks;  // MT * NT * KT (k-tile blocks)
     uint32_t dp_tiles;      // tiles 0 .. dp_tiles-1 go whole to CTAs in data-parallel waves
@@ -158,23 +159,29 @@ __device__ __forceinline__ uint32_t cta_of(uint32_t b, uint32_t B, uint32_t G) {
 // k-tiles of one tile, never crossing a tile boundary. The schedule has two
 // phases. Data-parallel waves: CTA c takes whole tiles c, c + G, c + 2G, ...
 // (`waves` of them), so the G tiles in flight at a time are consecutive in
-// (token tile, n-tile) order and share activation and weight tiles in L2.
-// Stream-K tail: the remaining tiles' k-tile blocks [sk_base, B) are split
-// evenly over the G CTAs, CTA c taking blocks [sk_b0, sk_b1). Blocks are
-// numbered tile * KT + k-tile in both phases. No division per unit.
+// tile order and share activation and weight tiles in L2. Stream-K tail: the
+// remaining tiles' k-tile blocks [sk_base, B) are split evenly over the G
+// CTAs, CTA c taking blocks [sk_b0, sk_b1). Blocks are numbered
+// tile * KT + k-tile in both phases. Tile order: groups of GM token tiles;
+// inside a group the token tile runs fastest, then the n-tile, so that the G
+// tiles in flight cover about GM token tiles x G/GM n-tiles, and each weight
+// tile is read by GM CTAs at about the same time (one DRAM read, the rest L2
+// hits) while the group's activations stay in L2. No division per unit.
 template <int KB>
 struct UnitCursor {
     uint32_t b, b1, seg_end;   // current block, end of the current range, end of the current segment
-    int KT, NT;
+    int KT, NT, MT, GM;
     int kt, nk, nt, mt;
     uint32_t tile, G;          // data-parallel phase: current tile, tile stride
     int waves_left;            // data-parallel tiles after the current one
     bool dp;
     uint32_t sk_b0, sk_b1;
     __device__ __forceinline__ void init(uint32_t c, uint32_t G_, int waves, uint32_t sk_b0_, uint32_t sk_b1_,
-                                         int KT_, int NT_) {
+                                         int KT_, int NT_, int MT_, int GM_) {
         KT = KT_;
         NT = NT_;
+        MT = MT_;
+        GM = GM_;
         G = G_;
         sk_b0 = sk_b0_;
         sk_b1 = sk_b1_;
@@ -189,21 +196,31 @@ struct UnitCursor {
             start_range();
         }
     }
+    // (mt, nt) of `tile` in the grouped order.
+    __device__ __forceinline__ void coords() {
+        const uint32_t span = (uint32_t)GM * (uint32_t)NT;
+        const uint32_t grp = tile / span;
+        const uint32_t idx = tile - grp * span;
+        const uint32_t m_base = grp * (uint32_t)GM;
+        uint32_t gm = (uint32_t)MT - m_base < (uint32_t)GM ? (uint32_t)MT - m_base : (uint32_t)GM;
+        if (gm == 0) gm = 1;   // only past the last tile (an empty range), never used
+        const uint32_t q = idx / gm;
+        nt = (int)q;
+        mt = (int)(m_base + idx - q * gm);
+    }
     __device__ __forceinline__ void start_tile() {
         b = tile * (uint32_t)KT;
         b1 = b + (uint32_t)KT;
         kt = 0;
-        mt = (int)(tile / (uint32_t)NT);
-        nt = (int)(tile - (uint32_t)mt * (uint32_t)NT);
+        coords();
         set_segment();
     }
     __device__ __forceinline__ void start_range() {
         b = sk_b0;
         b1 = sk_b1;
-        const uint32_t t = b / (uint32_t)KT;
-        kt = (int)(b - t * (uint32_t)KT);
-        mt = (int)(t / (uint32_t)NT);
-        nt = (int)(t - (uint32_t)mt * (uint32_t)NT);
+        tile = b / (uint32_t)KT;
+        kt = (int)(b - tile * (uint32_t)KT);
+        coords();   // unused when the range is empty
         set_segment();
     }
     __device__ __forceinline__ void set_segment() {
@@ -226,10 +243,8 @@ struct UnitCursor {
         }
         if (b < b1) {   // the stream-K range goes on with the next tile
             kt = 0;
-            if (++nt == NT) {
-                nt = 0;
-                ++mt;
-            }
+            ++tile;
+            coords();
             set_segment();
             return true;
         }
@@ -446,7 +461,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t pol_w = policy_evict_first();   // weights: streamed once
             const uint64_t pol_x = policy_evict_last();    // activations: reused by every n-tile
             UnitCursor<KB> cur;
-            cur.init(blockIdx.x, G, waves, b0, b1, KT, p.NT);
+            cur.init(blockIdx.x, G, waves, b0, b1, KT, p.NT, p.MT, p.GM);
             auto issue_w = [&](int s, const UnitCursor<KB> &c) {
                 mbar_arrive_expect_tx(&ctl->full[s], (uint32_t)(c.nk * (C::kWTile + C::kXTile)));
                 const uint8_t *wsrc = p.blob + p.off_codes + ((long long)c.nt * KT + c.kt) * C::kWTile;
@@ -516,7 +531,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 constexpr bool ALT = C::kAlt;
                 constexpr uint32_t idesc = idesc_i8(128, ALT ? TOK : TOK / 2, true, true);
                 UnitCursor<KB> cur;
-                cur.init(blockIdx.x, G, waves, b0, b1, KT, p.NT);
+                cur.init(blockIdx.x, G, waves, b0, b1, KT, p.NT, p.MT, p.GM);
                 int s = 0, seg = 0, unit = 0;
                 uint32_t ph = 0;
                 bool ok = true;
@@ -584,7 +599,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int r = quarter * 32 + lane;               // weight row in the tile
             const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
             UnitCursor<KB> cur;
-            cur.init(blockIdx.x, G, waves, b0, b1, KT, p.NT);
+            cur.init(blockIdx.x, G, waves, b0, b1, KT, p.NT, p.MT, p.GM);
             int s = 0;
             uint32_t ph = 0;
             for (int i = 0; !cur.done(); ++i, cur.advance()) {
@@ -664,7 +679,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool poller = (warp == C::kWarpEpi0);
             griddep_wait();   // outputs, scales, row sums and workspace belong to the previous kernel until now
             UnitCursor<KB> cur;
-            cur.init(blockIdx.x, G, waves, b0, b1, KT, p.NT);
+            cur.init(blockIdx.x, G, waves, b0, b1, KT, p.NT, p.MT, p.GM);
             int seg = 0, ubase = 0;
             int obuf = 0;   // this warp's next output stage block
             while (!cur.done()) {
@@ -992,6 +1007,7 @@ static qoq_status launch_gemm_t(const GemmArgs &a, cudaStream_t stream) {
     p.NT = (int)(a.N / kTileN);
     p.KT = (int)(a.K / kTileK);
     p.MT = (int)((a.M + TOK - 1) / TOK);
+    p.GM = p.MT < kTileGroup ? p.MT : kTileGroup;
     const long long blocks = (long long)p.MT * p.NT * p.KT;
     if (blocks >= (1ll << 31)) return QOQ_ERR_UNSUPPORTED;
     p.total_blocks = (uint32_t)blocks;

@@ -14,6 +14,7 @@ constexpr int kTileK = 128;        // K per tile = one quantisation group
 constexpr int kGroup = 128;
 constexpr int kMaxK = 65536;
 constexpr int kMaxGrid = 256;      // upper bound of the persistent grid (>= SM count)
+constexpr int kTileGroup = 8;      // token tiles per group of the GEMM's tile order
 
 // Programmatic dependent launch (griddepcontrol) between the activation
 // quantiser and the GEMM: each kernel releases its successor right after its
