@@ -45,6 +45,19 @@ def test_ragged_tokens_per_channel(M):
     check_full(X, W, 0, "per-channel M=%d" % M)
 
 
+@pytest.mark.parametrize("M", [513, 600, 700, 1000])
+def test_paired_ctas_ragged_tokens(M):
+    """Above 512 tokens the GEMM runs 256-token tiles on CTA pairs (one
+    256-row MMA across two SMs, each SM staging half of the token tile) when
+    the n-tiles pair up (N/128 even). Ragged last tiles whose second half is
+    empty (M=513, 600), partly live (700) or nearly full (1000), both
+    quantisation modes."""
+    X = inputs.make_activations(M, 640, seed=200 + M)
+    W = inputs.make_weights(512, 640, seed=200 + M)
+    check_full(X, W, 128, "pairs M=%d" % M)
+    check_full(X, W, 0, "pairs per-channel M=%d" % M)
+
+
 @pytest.mark.parametrize("N,K", [(128, 128), (128, 1152), (1152, 128), (896, 2176)])
 def test_tile_shapes(N, K):
     X = inputs.make_activations(24, K, seed=N + K)

@@ -58,13 +58,19 @@ constexpr int kIssuers = 2;
 constexpr int kWarpDequant0 = 4;         // warps 4..: the dequant warpgroups, then the epilogue warpgroups
 constexpr uint64_t kDrainNs = 100ull * 1000ull * 1000ull;   // 100 ms
 
-template <int TOK, int MODE>
+template <int TOK, int MODE, bool PAIR = false>
 struct GemmCfg {
+    // PAIR: a cluster of two CTAs runs one 256-row MMA (tcgen05.mma.cta_group::2):
+    // each CTA dequantises its own 128 weight rows into its own tensor memory
+    // and stages half of the token tile (tokens rank*TOK/2 ..), so per SM the
+    // token-tile bytes per MAC halve; the leader CTA issues the MMAs.
+    static_assert(!PAIR || TOK == 256, "paired CTAs are built for 256-token tiles");
+    static constexpr int kXRows = PAIR ? TOK / 2 : TOK;        // token rows staged by this CTA
     // KB = k-tiles per pipeline unit: two up to 128-token tiles (halves the
     // barrier and issue work per weight byte), one for 256-token tiles
     // (shared memory holds only two two-k-tile stages of those).
     static constexpr int kKB = TOK <= 128 ? 2 : 1;
-    static constexpr int kXTile = TOK * 128;                    // token tile, 128 k
+    static constexpr int kXTile = kXRows * 128;                 // this CTA's token rows, 128 k
     static constexpr int kWTile = MODE == 0 ? 8448 : 8192;      // codes (+ s, z*s) per k-tile
     static constexpr int kXBytes = kKB * kXTile;
     static constexpr int kWBytes = kKB * kWTile;
@@ -122,6 +128,7 @@ struct GemmParams {
     int32_t *partials;      // [grid][TOK][128]: contributor c's partial sums
     int M, N, K, group;
     int NT, KT, MT;
+    int NTw;                // n-tiles of the schedule: NT, or NT / 2 CTA pairs' 256-row tiles
     int GM;                 // token tiles per group of the tile order
     int grid;
     uint32_t total_blocks;  // MT * NT * KT (k-tile blocks)
@@ -385,11 +392,11 @@ __device__ __forceinline__ void add_second(uint32_t taddr, uint32_t (&v)[CH]) {
     for (int j = 0; j < CH; ++j) v[j] = (uint32_t)((int32_t)v[j] + (int32_t)w[j]);
 }
 
-template <int TOK, int MODE>
+template <int TOK, int MODE, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     qoq_gemm_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ CUtensorMap tmap_x,
                     const __grid_constant__ CUtensorMap tmap_y) {
-    using C = GemmCfg<TOK, MODE>;
+    using C = GemmCfg<TOK, MODE, PAIR>;
     constexpr int S = C::kStages;
     constexpr int KB = C::kKB;
     extern __shared__ uint8_t smem_raw[];
@@ -398,18 +405,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const Watchdog wd{&ctl->abort_flag, p.status};
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;   // 0: the pair's leader (MMA issue)
 
     // ------------------------------------------------------------ set-up
     if (threadIdx.x == 0) {
         ctl->abort_flag = 0;
         for (int s = 0; s < S; ++s) {
             mbar_init(&ctl->full[s], 1);
-            mbar_init(&ctl->freed[s], C::kAlt ? 1 : kIssuers);
-            mbar_init(&ctl->a_full[s], 4);   // the four warps of one dequant warpgroup
+            mbar_init(&ctl->freed[s], (C::kAlt || PAIR) ? 1 : kIssuers);
+            // the four warps of one dequant warpgroup (of each CTA of a pair)
+            mbar_init(&ctl->a_full[s], PAIR ? 8 : 4);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&ctl->acc_full[b], C::kHalves ? 1 : kIssuers);
-            mbar_init(&ctl->acc_empty[b], 4);
+            mbar_init(&ctl->acc_empty[b], PAIR ? 8 : 4);
         }
         mbar_init(&ctl->final_bar[0], 1);
         mbar_init(&ctl->final_bar[1], 1);
@@ -427,11 +436,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kWarpProducer && lane == 0) prefetch_tensormap(&tmap_x);
     if (warp == C::kWarpEpi0 && lane == 0 && p.fp16_out) prefetch_tensormap(&tmap_y);
     if (warp == kWarpMma) {
-        tmem_alloc(&ctl->tmem_base, C::kTmemCols);
-        tmem_relinquish();
+        if (PAIR) {
+            tmem_alloc_pair(&ctl->tmem_base, C::kTmemCols);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(&ctl->tmem_base, C::kTmemCols);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
     __syncthreads();
+    // A pair's CTAs arrive on the leader's barriers and the leader's MMAs
+    // write both CTAs' tensor memory: both set-ups complete first.
+    if (PAIR) cluster_sync_all();
     tc_fence_after();
     const uint32_t tmem_base = ctl->tmem_base;
     griddep_launch_dependents();   // the next kernel may start its own set-up
@@ -445,11 +462,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     // p.dp_tiles (`waves` of them), then its stream-K share [b0, b1) of the
     // tail blocks [sk_base, total) in (token tile, n-tile, k-tile) order,
     // k-tile fastest.
+    // With CTA pairs the schedule's unit is the pair (both CTAs walk the same
+    // blocks, each for its own n-tile 2 * nt + rank).
+    const uint32_t me = PAIR ? (blockIdx.x >> 1) : blockIdx.x;
     const uint32_t G = (uint32_t)p.grid;
-    const int waves = p.dp_tiles > blockIdx.x ? (int)((p.dp_tiles - blockIdx.x + G - 1) / G) : 0;
+    const int waves = p.dp_tiles > me ? (int)((p.dp_tiles - me + G - 1) / G) : 0;
     const uint32_t BS = p.total_blocks - p.sk_base;   // stream-K tail blocks
-    const uint32_t b0 = p.sk_base + cta_begin(blockIdx.x, BS, G);
-    const uint32_t b1 = p.sk_base + cta_begin(blockIdx.x + 1, BS, G);
+    const uint32_t b0 = p.sk_base + cta_begin(me, BS, G);
+    const uint32_t b1 = p.sk_base + cta_begin(me + 1, BS, G);
     const int KT = p.KT;
 
     auto stage_x = [&](int s) { return smem + s * C::kStageBytes; };
@@ -461,16 +481,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t pol_w = policy_evict_first();   // weights: streamed once
             const uint64_t pol_x = policy_evict_last();    // activations: reused by every n-tile
             UnitCursor<KB> cur;
-            cur.init(blockIdx.x, G, waves, b0, b1, KT, p.NT, p.MT, p.GM);
+            cur.init(me, G, waves, b0, b1, KT, p.NTw, p.MT, p.GM);
             auto issue_w = [&](int s, const UnitCursor<KB> &c) {
                 mbar_arrive_expect_tx(&ctl->full[s], (uint32_t)(c.nk * (C::kWTile + C::kXTile)));
-                const uint8_t *wsrc = p.blob + p.off_codes + ((long long)c.nt * KT + c.kt) * C::kWTile;
+                const int nt_cta = PAIR ? 2 * c.nt + (int)rank : c.nt;
+                const uint8_t *wsrc = p.blob + p.off_codes + ((long long)nt_cta * KT + c.kt) * C::kWTile;
                 bulk_load(stage_w(s), wsrc, (uint32_t)(c.nk * C::kWTile), &ctl->full[s], pol_w);
             };
             auto issue_x = [&](int s, const UnitCursor<KB> &c) {
                 for (int j = 0; j < c.nk; ++j)
                     tma_load_2d(stage_x(s) + j * C::kXTile, &tmap_x, &ctl->full[s], (c.kt + j) * kTileK,
-                                c.mt * TOK, pol_x);
+                                c.mt * TOK + (int)rank * C::kXRows, pol_x);
             };
             // The first S units need no free stage: start their weight copies
             // before waiting for the previous kernel, then their token tiles.
@@ -526,12 +547,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             // waits on) into its own accumulator and commits their freed[s].
             // Wider tiles: both issuers take every unit, each half of the
             // token columns, and both commit freed[s]. Both commit acc_full.
+            // A pair has one issuer, lane 0 of the leader's first issuer warp:
+            // one M = 256, N = TOK MMA per K = 32 step covers both CTAs.
             const int k = warp - kWarpMma;
-            if (lane == 0) {
+            if (lane == 0 && (!PAIR || (rank == 0 && k == 0))) {
                 constexpr bool ALT = C::kAlt;
-                constexpr uint32_t idesc = idesc_i8(128, ALT ? TOK : TOK / 2, true, true);
+                constexpr uint32_t idesc = idesc_i8(PAIR ? 256 : 128, (ALT || PAIR) ? TOK : TOK / 2, true, true);
                 UnitCursor<KB> cur;
-                cur.init(blockIdx.x, G, waves, b0, b1, KT, p.NT, p.MT, p.GM);
+                cur.init(me, G, waves, b0, b1, KT, p.NTw, p.MT, p.GM);
                 int s = 0, seg = 0, unit = 0;
                 uint32_t ph = 0;
                 bool ok = true;
@@ -539,7 +562,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int buf = seg % C::kAccBufs;
                     const uint32_t aph = (uint32_t)(seg / C::kAccBufs) & 1u;
                     const int bi = C::kHalves ? k : buf;   // this issuer's accumulator barrier pair
-                    ok = wait_bounded(&ctl->acc_empty[bi], aph ^ 1u, wd, kSiteMmaAccEmpty, seg);
+                    if (PAIR)   // both halves, released by the epilogues of both CTAs
+                        ok = wait_bounded_cluster(&ctl->acc_empty[0], aph ^ 1u, wd, kSiteMmaAccEmpty, seg) &&
+                             wait_bounded_cluster(&ctl->acc_empty[1], aph ^ 1u, wd, kSiteMmaAccEmpty, seg);
+                    else
+                        ok = wait_bounded(&ctl->acc_empty[bi], aph ^ 1u, wd, kSiteMmaAccEmpty, seg);
                     if (!ok) break;
                     const uint32_t d_tmem = tmem_base + (uint32_t)(buf * C::kAccCols + k * (ALT ? TOK : TOK / 2));
                     uint32_t acc = 0u;   // this issuer's first MMA of the segment overwrites its accumulator
@@ -554,7 +581,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                             // before this thread's MMAs. Each wait of an
                             // issuing thread costs it hundreds of cycles, so
                             // the issuer waits once per unit.
-                            ok = wait_bounded(&ctl->a_full[s], ph, wd, kSiteMmaOperands, unit);
+                            ok = PAIR ? wait_bounded_cluster(&ctl->a_full[s], ph, wd, kSiteMmaOperands, unit)
+                                      : wait_bounded(&ctl->a_full[s], ph, wd, kSiteMmaOperands, unit);
                             if (!ok) break;
                             tc_fence_after();
                             const uint32_t a_tmem = tmem_base + (uint32_t)(C::kACol0 + s * KB * 32);
@@ -564,11 +592,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                             // and (N split) issuer k's token rows k*TOK/2 ..
                             // another (TOK/2) x 128 bytes on.
                             const uint64_t bk = bdesc + (uint64_t)(ALT ? 0 : k * (TOK / 2) * 128 / 16);
-                            mma4_i8_ts(d_tmem, a_tmem, bk, idesc, acc);
-                            if (KB == 2 && cur.nk == 2)
-                                mma4_i8_ts(d_tmem, a_tmem + 32u, bk + (uint64_t)(C::kXTile >> 4), idesc, 1u);
-                            acc = 1u;
-                            tc_commit(&ctl->freed[s]);
+                            if (PAIR) {
+                                mma4_i8_ts_pair(d_tmem, a_tmem, bk, idesc, acc);
+                                acc = 1u;
+                                tc_commit_pair_both(&ctl->freed[s]);
+                            } else {
+                                mma4_i8_ts(d_tmem, a_tmem, bk, idesc, acc);
+                                if (KB == 2 && cur.nk == 2)
+                                    mma4_i8_ts(d_tmem, a_tmem + 32u, bk + (uint64_t)(C::kXTile >> 4), idesc, 1u);
+                                acc = 1u;
+                                tc_commit(&ctl->freed[s]);
+                            }
                         }
                         ++unit;
                         if (++s == S) {
@@ -578,11 +612,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                         seg_done = cur.advance();
                     }
                     if (!ok) break;
-                    tc_commit(&ctl->acc_full[bi]);
+                    if (PAIR) {
+                        tc_commit_pair_both(&ctl->acc_full[0]);
+                        tc_commit_pair_both(&ctl->acc_full[1]);
+                    } else {
+                        tc_commit(&ctl->acc_full[bi]);
+                    }
                     ++seg;
                 }
                 // Every MMA must have completed before tensor memory is freed.
-                tc_commit(&ctl->final_bar[k]);
+                if (PAIR)
+                    tc_commit_pair(&ctl->final_bar[k]);
+                else
+                    tc_commit(&ctl->final_bar[k]);
                 wait_drain(&ctl->final_bar[k], 0, kDrainNs);
             }
             __syncwarp();
@@ -599,7 +641,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int r = quarter * 32 + lane;               // weight row in the tile
             const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
             UnitCursor<KB> cur;
-            cur.init(blockIdx.x, G, waves, b0, b1, KT, p.NT, p.MT, p.GM);
+            cur.init(me, G, waves, b0, b1, KT, p.NTw, p.MT, p.GM);
             int s = 0;
             uint32_t ph = 0;
             for (int i = 0; !cur.done(); ++i, cur.advance()) {
@@ -658,7 +700,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&ctl->a_full[unit_s]);
+                if (lane == 0) {
+                    if (PAIR)
+                        mbar_arrive_cluster(&ctl->a_full[unit_s], 0);   // the leader's barrier
+                    else
+                        mbar_arrive(&ctl->a_full[unit_s]);
+                }
                 __syncwarp();
             }
         } else if (warp >= C::kWarpEpi0) {
@@ -677,9 +724,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
             const bool leader = (threadIdx.x == C::kWarpEpi0 * 32);
             const bool poller = (warp == C::kWarpEpi0);
+            // A part of the accumulator goes back to the issuer's CTA.
+            auto acc_release = [&](uint64_t *bar) {
+                if (PAIR)
+                    mbar_arrive_cluster(bar, 0);
+                else
+                    mbar_arrive(bar);
+            };
+            // Flag and partial-sum slot of contributor c (a schedule unit).
+            auto fidx = [&](uint32_t c) { return PAIR ? 2u * c + rank : c; };
             griddep_wait();   // outputs, scales, row sums and workspace belong to the previous kernel until now
             UnitCursor<KB> cur;
-            cur.init(blockIdx.x, G, waves, b0, b1, KT, p.NT, p.MT, p.GM);
+            cur.init(me, G, waves, b0, b1, KT, p.NTw, p.MT, p.GM);
             int seg = 0, ubase = 0;
             int obuf = 0;   // this warp's next output stage block
             while (!cur.done()) {
@@ -696,7 +752,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ubase += nunits;
                 const int buf = seg % C::kAccBufs;
                 const uint32_t aph = (uint32_t)(seg / C::kAccBufs) & 1u;
-                const int n = nt * kTileN + r;
+                const int n = (PAIR ? 2 * nt + (int)rank : nt) * kTileN + r;
                 const int64_t m0 = (int64_t)mt * TOK;
                 const bool two = C::kAlt && nunits >= 2;
                 // Token columns of the tile that hold tokens (>= 1): the steps
@@ -705,9 +761,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // Owner (or sole computer) of a tile: the CTA holding its first
                 // k-tile. Contributors c_first .. c_last (none if c_last < c_first).
                 const bool owner = kt_lo == 0;
-                const uint32_t c_first = blockIdx.x + 1;
+                const uint32_t c_first = me + 1;
                 const uint32_t c_last =
-                    (!owner || kt_hi == KT) ? blockIdx.x : cta_of(tile_b + (uint32_t)KT - 1 - p.sk_base, BS, G);
+                    (!owner || kt_hi == KT) ? me : cta_of(tile_b + (uint32_t)KT - 1 - p.sk_base, BS, G);
                 constexpr int CO = 16;   // token columns per step
                 // The parts this warpgroup reads: [h_lo, h_hi) of NP, PART columns each.
                 constexpr int NP = C::kHalves ? 2 : 1;
@@ -747,7 +803,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     bool got = true;
                     if (poller) {
                         for (uint32_t c = c_first + (uint32_t)lane; c <= c_last && got; c += 32)
-                            got = wait_flag_bounded(p.flags + c, wd, (int)c);
+                            got = wait_flag_bounded(p.flags + fidx(c), wd, (int)c);
                         got = __all_sync(0xffffffffu, got);
                     }
                     if (named_bar_any(kBarAll, NEPI, !got)) break;
@@ -776,7 +832,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (c_hi <= c_lo) {   // no token in this part: hand it back at once
                         tc_fence_before();
                         __syncwarp();
-                        if (lane == 0) mbar_arrive(&ctl->acc_empty[bi]);
+                        if (lane == 0) acc_release(&ctl->acc_empty[bi]);
                         continue;
                     }
                     if (C::kHalves && owner && !polls && p.fp16_out) {
@@ -794,7 +850,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 if (c0 + CO >= c_hi) {
                                     tc_fence_before();
                                     __syncwarp();
-                                    if (lane == 0) mbar_arrive(&ctl->acc_empty[bi]);
+                                    if (lane == 0) acc_release(&ctl->acc_empty[bi]);
                                 }
                                 convert_fp16<CO, MODE>(v, pk[q], col_scale, col_zero, ctl->tok_scale + c0,
                                                        ctl->tok_rowsum + c0);
@@ -819,7 +875,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (c0 + CO >= c_hi) {
                             tc_fence_before();
                             __syncwarp();
-                            if (lane == 0) mbar_arrive(&ctl->acc_empty[bi]);
+                            if (lane == 0) acc_release(&ctl->acc_empty[bi]);
                         }
                         if (!owner) {
                             // Contributor: the live token columns of the partial
@@ -842,7 +898,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                                 for (int cc = 0; cc < 8; ++cc) {
                                     const int32_t *part =
-                                        p.partials + (long long)(c + cc) * TOK * kTileN + c0 * kTileN + r;
+                                        p.partials + (long long)fidx(c + cc) * TOK * kTileN + c0 * kTileN + r;
 #pragma unroll
                                     for (int j = 0; j < 4; ++j)
                                         t[cc][j] = (c + cc <= c_last) ? ld_cg_s32(part + j * kTileN) : 0;
@@ -859,7 +915,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                                 for (int cc = 0; cc < 4; ++cc) {
                                     const int32_t *part =
-                                        p.partials + (long long)(c + cc) * TOK * kTileN + c0 * kTileN + r;
+                                        p.partials + (long long)fidx(c + cc) * TOK * kTileN + c0 * kTileN + r;
 #pragma unroll
                                     for (int j = 0; j < CO; ++j)
                                         t[cc][j] = (c + cc <= c_last) ? ld_cg_s32(part + j * kTileN) : 0;
@@ -891,7 +947,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (leader) st_release_gpu(p.flags + blockIdx.x, 1);
                     __syncwarp();
                 } else if (polls && poller) {
-                    for (uint32_t c = c_first + (uint32_t)lane; c <= c_last; c += 32) p.flags[c] = 0;
+                    for (uint32_t c = c_first + (uint32_t)lane; c <= c_last; c += 32) p.flags[fidx(c)] = 0;
                     __syncwarp();
                 }
                 ++seg;
@@ -907,9 +963,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
     tc_fence_before();
     __syncthreads();
+    // The leader's MMAs (which write the peer's tensor memory) have completed
+    // and the peer's last arrivals on the leader's barriers are done before
+    // either CTA frees tensor memory or exits.
+    if (PAIR) cluster_sync_all();
     if (warp == kWarpMma) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, C::kTmemCols);
+        if (PAIR)
+            tmem_dealloc_pair(tmem_base, C::kTmemCols);
+        else
+            tmem_dealloc(tmem_base, C::kTmemCols);
     }
 }
 
@@ -965,25 +1028,55 @@ static bool encode_y_map(CUtensorMap *map, void *Y, int64_t M, int64_t N) {
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Number of two-CTA clusters of the paired kernel that can be resident at
+// once (clusters live inside one GPC, so this can be below SMs / 2); the
+// persistent schedule never launches more, so every cluster is resident and
+// stream-K partners can wait on one another. 0 when pairs cannot launch.
 template <int TOK, int MODE>
-static qoq_status launch_gemm_t(const GemmArgs &a, cudaStream_t stream) {
-    using C = GemmCfg<TOK, MODE>;
+static int pair_clusters_of(int dev) {
+    using C = GemmCfg<TOK, MODE, true>;
+    static std::once_flag once[64];
+    static int count[64];
+    std::call_once(once[dev], [&] {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = C::kSmemBytes;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaFuncSetAttribute(qoq_gemm_kernel<TOK, MODE, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::kSmemBytes) != cudaSuccess ||
+            cudaOccupancyMaxActiveClusters(&n, qoq_gemm_kernel<TOK, MODE, true>, &cfg) != cudaSuccess)
+            n = 0;
+        (void)cudaGetLastError();
+        count[dev] = n;
+    });
+    return count[dev];
+}
+
+template <int TOK, int MODE, bool PAIR>
+static qoq_status launch_gemm_t(const GemmArgs &a, cudaStream_t stream, int units_max) {
+    using C = GemmCfg<TOK, MODE, PAIR>;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return QOQ_ERR_CUDA;
-    const int sms = sm_count_of(dev);
-    if (sms <= 0) return QOQ_ERR_CUDA;
 
     // Opt in to the large dynamic shared memory once per device.
     static std::once_flag attr_once[64];
     static cudaError_t attr_err[64];
     std::call_once(attr_once[dev], [&] {
-        attr_err[dev] = cudaFuncSetAttribute(qoq_gemm_kernel<TOK, MODE>,
+        attr_err[dev] = cudaFuncSetAttribute(qoq_gemm_kernel<TOK, MODE, PAIR>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     });
     if (attr_err[dev] != cudaSuccess) return QOQ_ERR_CUDA;
 
     CUtensorMap tmap, tmap_y;
-    if (!encode_x_map(&tmap, a.X8, a.M, a.K, TOK)) return QOQ_ERR_CUDA;
+    if (!encode_x_map(&tmap, a.X8, a.M, a.K, C::kXRows)) return QOQ_ERR_CUDA;
     if (a.fp16_out) {
         if (!encode_y_map(&tmap_y, a.out, a.M, a.N)) return QOQ_ERR_CUDA;
     } else {
@@ -1005,16 +1098,18 @@ static qoq_status launch_gemm_t(const GemmArgs &a, cudaStream_t stream) {
     p.K = (int)a.K;
     p.group = a.group;
     p.NT = (int)(a.N / kTileN);
+    p.NTw = PAIR ? p.NT / 2 : p.NT;
     p.KT = (int)(a.K / kTileK);
     p.MT = (int)((a.M + TOK - 1) / TOK);
     p.GM = p.MT < kTileGroup ? p.MT : kTileGroup;
-    const long long blocks = (long long)p.MT * p.NT * p.KT;
+    const long long blocks = (long long)p.MT * p.NTw * p.KT;
     if (blocks >= (1ll << 31)) return QOQ_ERR_UNSUPPORTED;
     p.total_blocks = (uint32_t)blocks;
-    p.grid = (int)std::min<long long>(std::min(sms, kMaxGrid), blocks);
+    // Schedule units (CTAs, or CTA pairs): at most one per SM (pair), all resident.
+    p.grid = (int)std::min<long long>(units_max, blocks);
     // Whole tiles in data-parallel waves while at least one to two waves of
     // tiles remain for the stream-K tail, which evens out the last wave.
-    const long long tiles = (long long)p.MT * p.NT;
+    const long long tiles = (long long)p.MT * p.NTw;
     const long long dp_tiles = tiles >= 2ll * p.grid ? (tiles / p.grid - 1) * p.grid : 0;
     p.dp_tiles = (uint32_t)dp_tiles;
     p.sk_base = (uint32_t)(dp_tiles * p.KT);
@@ -1024,27 +1119,49 @@ static qoq_status launch_gemm_t(const GemmArgs &a, cudaStream_t stream) {
     p.fp16_out = a.fp16_out ? 1 : 0;
 
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)p.grid);
+    cfg.gridDim = dim3((unsigned)(PAIR ? 2 * p.grid : p.grid));
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = C::kSmemBytes;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    if (kProgrammaticLaunch) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    if (PAIR) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = 2;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+    }
     cfg.attrs = attr;
-    cfg.numAttrs = kProgrammaticLaunch ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, qoq_gemm_kernel<TOK, MODE>, p, tmap, tmap_y) == cudaSuccess ? QOQ_OK
-                                                                                               : QOQ_ERR_CUDA;
+    cfg.numAttrs = na;
+    return cudaLaunchKernelEx(&cfg, qoq_gemm_kernel<TOK, MODE, PAIR>, p, tmap, tmap_y) == cudaSuccess
+               ? QOQ_OK
+               : QOQ_ERR_CUDA;
 }
 
 template <int MODE>
 static qoq_status launch_gemm_mode(const GemmArgs &a, cudaStream_t stream) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return QOQ_ERR_CUDA;
+    const int sms = sm_count_of(dev);
+    if (sms <= 0) return QOQ_ERR_CUDA;
+    const int ctas = std::min(sms, kMaxGrid);
     switch (token_tile_for(a.M, a.N, a.K)) {
-        case 16: return launch_gemm_t<16, MODE>(a, stream);
-        case 32: return launch_gemm_t<32, MODE>(a, stream);
-        case 64: return launch_gemm_t<64, MODE>(a, stream);
-        case 128: return launch_gemm_t<128, MODE>(a, stream);
-        default: return launch_gemm_t<256, MODE>(a, stream);
+        case 16: return launch_gemm_t<16, MODE, false>(a, stream, ctas);
+        case 32: return launch_gemm_t<32, MODE, false>(a, stream, ctas);
+        case 64: return launch_gemm_t<64, MODE, false>(a, stream, ctas);
+        case 128: return launch_gemm_t<128, MODE, false>(a, stream, ctas);
+        default: {
+            // 256-token tiles run on CTA pairs when the n-tiles pair up.
+            const int pairs = (a.N / kTileN) % 2 == 0 ? std::min(pair_clusters_of<256, MODE>(dev), kMaxGrid / 2) : 0;
+            if (pairs > 0) return launch_gemm_t<256, MODE, true>(a, stream, pairs);
+            return launch_gemm_t<256, MODE, false>(a, stream, ctas);
+        }
     }
 }
 

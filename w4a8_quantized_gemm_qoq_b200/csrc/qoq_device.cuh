@@ -303,6 +303,111 @@ __device__ __forceinline__ void tmem_st32_wait(uint32_t taddr, const uint32_t (&
         : "memory");
 }
 
+// ---------------------------------------------- CTA pairs (cta_group::2)
+// A kernel uses one cta_group for all its tcgen05 instructions; the paired
+// GEMM uses these forms. The pair is a cluster of two CTAs; rank 0 (the
+// leader) issues the MMAs, which read A from both CTAs' tensor memory and B
+// from both CTAs' shared memory (each holds half of the MMA's N), and write
+// each CTA's half of the M rows into its own tensor memory.
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// All threads of both CTAs; release/acquire at cluster scope.
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t *smem_result, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(smem_result)),
+                 "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// Arrive on this CTA's `bar` once the pair's tcgen05 operations issued so
+// far by this thread have completed.
+__device__ __forceinline__ void tc_commit_pair(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+// The same, arriving on the barrier at `bar`'s offset in both CTAs of the pair.
+__device__ __forceinline__ void tc_commit_pair_both(uint64_t *bar) {
+    asm volatile(
+        "{\n\t.reg .b16 m;\n\tmov.b16 m, 3;\n\t"
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n\t}" ::"r"(
+            smem_u32(bar))
+        : "memory");
+}
+
+// Four paired MMAs (K = 32 each) of one 128-wide k-tile, as mma4_i8_ts.
+__device__ __forceinline__ void mma4_i8_ts_pair(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::i8 [%0], [%1], %2, %3, p;\n\t"
+        "tcgen05.mma.cta_group::2.kind::i8 [%0], [%5], %6, %3, 1;\n\t"
+        "tcgen05.mma.cta_group::2.kind::i8 [%0], [%7], %8, %3, 1;\n\t"
+        "tcgen05.mma.cta_group::2.kind::i8 [%0], [%9], %10, %3, 1;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(a_tmem + 8u), "l"(b_desc + 2ull),
+        "r"(a_tmem + 16u), "l"(b_desc + 4ull), "r"(a_tmem + 24u), "l"(b_desc + 6ull)
+        : "memory");
+}
+
+// Arrive on the barrier at `bar`'s offset in CTA `rank` of the cluster
+// (this CTA included), with the instruction's default release semantics, the
+// form CUTLASS's 2-SM pipelines use for cross-CTA arrivals. (The .cluster
+// scope release costs the arriving thread about a microsecond on B200: it
+// waits for the SM's outstanding memory traffic.)
+__device__ __forceinline__ void mbar_arrive_cluster(uint64_t *bar, uint32_t rank) {
+    uint32_t ra;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(bar)), "r"(rank));
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(ra) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// wait_bounded for barriers that CTAs of the cluster arrive on (acquire at
+// cluster scope).
+__device__ __forceinline__ bool wait_bounded_cluster(uint64_t *bar, uint32_t parity, const Watchdog &wd, int site,
+                                                     int detail, uint64_t limit_ns = kWaitLimitNs) {
+    const uint32_t a = smem_u32(bar);
+    if (mbar_try_wait_cluster(a, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait_cluster(a, parity)) return true;
+        if ((it & 31u) == 0) {
+            if (wd.aborted()) return false;
+            if (globaltimer_ns() - t0 > limit_ns) {
+                wd.fail(QOQ_ERR_TIMEOUT, site, detail);
+                return false;
+            }
+        }
+    }
+}
+
 // ------------------------------------------- programmatic dependent launch
 
 // Block until the grids this one depends on have completed and their memory
