@@ -76,7 +76,10 @@ struct GemmCfg {
     static constexpr int kWBytes = kKB * kWTile;
     static constexpr int kStageBytes = (kXBytes + kWBytes + 1023) / 1024 * 1024;
     static constexpr int kSmemLimit = 232448;                   // 227 KB per CTA
-    static constexpr int kReserve = 20480;                      // alignment slack + control block
+    // After the stages: 1 KB alignment slack, the control block (3 KB) and
+    // the epilogue warps' output staging (two 1 KB blocks per warp).
+    static constexpr int kCtlBytes = 3072;
+    static constexpr int kReserve = 1024 + kCtlBytes + (TOK == 256 ? 8 : 4) * 2048;
     // Two MMA issuers. Up to 64-token tiles (kAlt), issuer j takes the units
     // of index parity j (those its dequant warpgroup serves) into its own
     // accumulator, and the epilogue adds the two; wider tiles have no TMEM for
@@ -148,11 +151,8 @@ struct SharedCtl {
     // tile: FP32(s_x) and (per-channel variant) the row sums.
     alignas(16) float tok_scale[256];
     int32_t tok_rowsum[256];
-    // Per epilogue warp, two alternating blocks of one step's FP16 outputs
-    // (16 tokens x 32 weight rows), the source of the TMA output stores.
-    alignas(128) __half out_stage[8][2][16 * 32];
 };
-static_assert(sizeof(SharedCtl) + 1023 <= GemmCfg<16, 0>::kReserve, "control block outgrows the reserve");
+static_assert(sizeof(SharedCtl) <= GemmCfg<16, 0>::kCtlBytes, "control block outgrows its reserve");
 
 // First k-tile block of CTA c (the stream-K split), and the CTA holding block b.
 __device__ __forceinline__ uint32_t cta_begin(uint32_t c, uint32_t B, uint32_t G) {
@@ -402,6 +402,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     SharedCtl *ctl = reinterpret_cast<SharedCtl *>(smem + S * C::kStageBytes);
+    // Per epilogue warp, two alternating blocks of one step's FP16 outputs
+    // (16 tokens x 32 weight rows), the source of the TMA output stores.
+    __half *out_stage = reinterpret_cast<__half *>(smem + S * C::kStageBytes + C::kCtlBytes);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const Watchdog wd{&ctl->abort_flag, p.status};
@@ -861,7 +864,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const int c0 = c_lo + q * CO;
                             if (c0 < c_hi) {
                                 store_packed_fp16(&tmap_y, pk[q], m0 + c0, n - lane, lane,
-                                                  ctl->out_stage[warp - C::kWarpEpi0][obuf]);
+                                                  out_stage + ((warp - C::kWarpEpi0) * 2 + obuf) * (16 * 32));
                                 obuf ^= 1;
                             }
                         }
@@ -929,7 +932,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (p.fp16_out) {
                             store_outputs_fp16<CO, MODE>(&tmap_y, v, m0 + c0, n - lane, lane, col_scale, col_zero,
                                                          ctl->tok_scale + c0, ctl->tok_rowsum + c0,
-                                                         ctl->out_stage[warp - C::kWarpEpi0][obuf]);
+                                                         out_stage + ((warp - C::kWarpEpi0) * 2 + obuf) * (16 * 32));
                             obuf ^= 1;
                         } else {
                             store_outputs_i32<CO, MODE>(p, v, m0 + c0, n, col_zero, ctl->tok_rowsum + c0);
