@@ -23,9 +23,13 @@
 //     scalar. 8 nibbles per 32-bit word decode with and/shift, one 32-bit
 //     multiply-add (q*s <= 240 and q*s + 128 - z*s in [7, 249] never carry
 //     between bytes) and one xor that turns excess-128 bytes into int8.
-//   * warp roles: 1 TMA producer warp, 2 MMA issuer warps (lane 0 each), two
-//     dequant warpgroups that take alternate pipeline units, one epilogue
-//     warpgroup.
+//   * warp roles: 1 TMA producer warp, 2 MMA issuer warps (lane 0 each), and
+//     either two dequant warpgroups that take alternate pipeline units and one
+//     epilogue warpgroup (up to 128-token tiles), or one dequant warpgroup and
+//     two epilogue warpgroups, one per accumulator half (256-token tiles).
+//   * 256-token tiles run on CTA pairs where the n-tiles pair up: one
+//     tcgen05.mma.cta_group::2 with M = 256 (each CTA's 128 weight rows in its
+//     own tensor memory) and each CTA staging half of the token tile.
 //   * a pipeline unit is up to KB consecutive k-tiles of one n-tile: one bulk
 //     copy of the packed weights, one TMA per token tile, one TMEM A buffer,
 //     one commit that frees both the shared-memory stage and the TMEM buffer.
@@ -34,7 +38,8 @@
 //     kernel may write (activations, scales, outputs, workspace) is touched
 //     only after griddepcontrol.wait.
 //   * persistent stream-K at k-tile granularity: the (token tile, n-tile,
-//     k-tile) blocks are split evenly over at most one CTA per SM. A tile cut
+//     k-tile) blocks, tiles in groups of up to 8 token tiles with the token
+//     tile fastest, are split evenly over at most one CTA (pair) per SM (pair). A tile cut
 //     between CTAs is finished by its owner -- the CTA holding the tile's
 //     first k-tile, which it reaches last -- after the other contributors
 //     (which reach their share of the tile first) have stored their INT32
