@@ -399,6 +399,7 @@ def run_gpu(args, rank, world, local_rank):
     e2e = run_e2e(args, probs, qoq, stream) if rank == 0 else None
     w8a8 = run_w8a8(probs, stream, gemm_only_us, max(K, 10)) if rank == 0 else None
     producers = run_producers(stream, peaks) if rank == 0 and not args.no_context else None
+    saturation = run_saturation(stream) if rank == 0 and args.saturation else None
     res = {
         "metric": METRIC, "value": round(world * ops_step / (step_ms * 1e-3) / 1e12, 3), "unit": "TOPS",
         "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup),
@@ -418,6 +419,7 @@ def run_gpu(args, rank, world, local_rank):
         "per_gemm": per,
         "w8a8_context": w8a8,
         "producers_context": producers,
+        "saturation_context": saturation,
     }
     return res
 
@@ -466,6 +468,61 @@ def run_shape(args):
     return {"shape": [M, N, K], "launches": args.steps, "us_per_launch": round(us, 3),
             "how": "one CUDA graph of back-to-back launches, replayed",
             "GBps": round(gemm_bytes(M, N, K) / us / 1e3, 1), "TOPS": round(gemm_ops(M, N, K) / us / 1e6, 2)}
+
+
+def run_saturation(stream, reps=20):
+    """Context, not the product: the protective range's point on this GPU.
+    The same GEMM with the excess-128 decode (protective range: no saturation
+    can occur) and with a decode that saturates every byte (what a kernel
+    without the protective range must do), on the gate_up projection at decode
+    (M = 16) and prefill (M = 2048) sizes: one graph of back-to-back launches,
+    each launch its own weight copy (more than L2 together), events around the
+    replays. The two outputs are bit-identical (GPU test)."""
+    import torch
+    from w4a8_quantized_gemm_qoq_b200 import qoq
+    dev = torch.device("cuda", torch.cuda.current_device())
+    out = []
+    K, N = 4096, 28672
+    W = torch.from_numpy(inputs.make_weights(N, K, seed=5)).to(dev)
+    blob = qoq.quantize_weights(W, GROUP)
+    del W
+    blobs = [blob] + [blob.clone() for _ in range(int(300e6 // blob.numel()))]
+    for M in (16, 2048):
+        X = torch.from_numpy(inputs.make_activations(M, K, seed=5)).to(dev)
+        X8, s_x, rs = qoq.quantize_act_per_token(X)
+        ws = qoq.Workspace.for_shape(M, N, K, GROUP, dev)
+        Y = torch.empty((M, N), dtype=torch.float16, device=dev)
+        res = {"M": M, "N": N, "K": K}
+        for key, fn in (("protective_us", lambda b: qoq.gemm_fp16_out(X8, s_x, b, N, K, GROUP, rowsum=rs, ws=ws,
+                                                                      Y=Y, stream=stream)),
+                        ("saturating_us", lambda b: qoq.gemm_fp16_out_saturating(X8, s_x, b, N, K, ws=ws, Y=Y,
+                                                                                 stream=stream))):
+            stream.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(stream):
+                for i in range(3):
+                    fn(blobs[i % len(blobs)])
+            stream.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(reps):
+                    fn(blobs[i % len(blobs)])
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                g.replay()
+                e0.record(stream)
+                g.replay()
+                e1.record(stream)
+            stream.synchronize()
+            assert ws.status() == 0, "device status %d" % ws.status()
+            del g
+            res[key] = round(1000.0 * e0.elapsed_time(e1) / reps, 3)
+        res["saturating_slowdown"] = round(res["saturating_us"] / res["protective_us"], 3)
+        out.append(res)
+        del X, X8, s_x, rs, ws, Y
+    del blobs, blob
+    torch.cuda.empty_cache()
+    return {"shapes": out, "how": "qoq_gemm_fp16_out vs qoq_gemm_fp16_out_saturating, gate_up 4096->28672; one "
+                                  "graph of %d back-to-back launches per variant, own weight copies" % reps}
 
 
 def run_producers(stream, peaks, reps=20):
@@ -699,6 +756,8 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--saturation", action="store_true",
+                    help="also time the protective-range ablation (saturating weight decode) as context")
     ap.add_argument("--no-context", action="store_true",
                     help="skip the fused-producer context measurements (not part of the timed step)")
     ap.add_argument("--shape", default=None,

@@ -191,6 +191,26 @@ qoq_status qoq_gemm_fp16_out(const int8_t *X8, const void *s_x_fp16, const int32
                              void *stream);
 
 /*
+ * Ablation of the protective range: qoq_gemm_fp16_out with a weight decode
+ * that saturates every dequantised byte to [-128, 127], as a kernel must when
+ * dequantised weights can leave the INT8 range. (paperlayer.ai summary,
+ * section 4 "Progressive Group Quantization": the range is shrunk to
+ * [-119, 119] so that the intermediate weights never overflow INT8, because
+ * saturation would otherwise cost up to 67% of the GEMM's throughput.)
+ *
+ * With blobs from qoq_quantize_weights (protective range) the saturation
+ * never acts, so the result is bit-identical to qoq_gemm_fp16_out; the call
+ * exists to measure what the saturating decode costs on this GPU. Arguments,
+ * workspace and status word as for qoq_gemm_fp16_out. Built for
+ * group_size 128 and two token tiles: M <= 16 (decode) and M > 512 on CTA
+ * pairs (N / 128 even); other sizes return QOQ_ERR_UNSUPPORTED without a
+ * launch.
+ */
+qoq_status qoq_gemm_fp16_out_saturating(const int8_t *X8, const void *s_x_fp16, const void *blob, int64_t M,
+                                        int64_t N, int64_t K, int group_size, void *Y_fp16, void *workspace,
+                                        size_t *workspace_bytes, void *stream);
+
+/*
  * W4A8 GEMM with the fused FP16 epilogue, for callers that cannot allocate
  * device memory (a pre-planned memory arena, a thread that must not touch the
  * device allocator while other work owns it, a runtime that forbids cudaMalloc

@@ -101,6 +101,14 @@ def test_argument_validation_without_launch(L):
     assert L.qoq_silu_mul_quant(dummy, 4, 14336, ctypes.c_void_p(16 * 1024 + 4), dummy, None, None) == 3
     assert L.qoq_silu_mul_quant(dummy, 4, 14336, dummy, ctypes.c_void_p(16 * 1024 + 1), None, None) == 3
     assert L.qoq_silu_mul_quant(None, 0, 14336, None, None, None, None) == 0
+    # saturating-decode ablation: group 128 only; M <= 16, or M > 512 on paired n-tiles
+    S = L.qoq_gemm_fp16_out_saturating
+    assert S(dummy, dummy, dummy, 4, 256, 512, 0, dummy, dummy, ws, None) == 2      # per-channel
+    assert S(dummy, dummy, dummy, 64, 256, 512, 128, dummy, dummy, ws, None) == 2   # 16 < M <= 512
+    assert S(dummy, dummy, dummy, 600, 384, 512, 128, dummy, dummy, ws, None) == 2  # N / 128 odd
+    assert S(dummy, dummy, dummy, 4, 256, 512, 128, dummy, dummy, _sz(8), None) == 4
+    assert S(dummy, None, dummy, 4, 256, 512, 128, dummy, dummy, ws, None) == 1     # s_x needed
+    assert S(None, None, None, 0, 256, 512, 128, None, dummy, ws, None) == 0        # M = 0
 
 
 def test_watchdog_selftest_validation_without_launch(L):

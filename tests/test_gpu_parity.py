@@ -58,6 +58,25 @@ def test_paired_ctas_ragged_tokens(M):
     check_full(X, W, 0, "pairs per-channel M=%d" % M)
 
 
+@pytest.mark.parametrize("M,N,K", [(1, 256, 512), (16, 1024, 1280), (600, 512, 640), (2048, 28672, 4096)])
+def test_saturating_decode_ablation_is_bit_identical(M, N, K):
+    """The protective-range ablation decodes the weights with per-byte
+    saturation. On blobs with the protective range the clamp never acts, so
+    the outputs equal the excess-128 decode's bit for bit (both token tiles it
+    is built for: 16, and 256 on CTA pairs)."""
+    X = inputs.make_activations(M, K, seed=300 + M)
+    W = inputs.make_weights(N, K, seed=300 + N)
+    blob = qoq.quantize_weights(dev(W), 128)
+    X8, s_x, rs = qoq.quantize_act_per_token(dev(X))
+    ws = qoq.Workspace.for_shape(M, N, K, 128)
+    y = qoq.gemm_fp16_out(X8, s_x, blob, N, K, 128, rowsum=rs, ws=ws)
+    y_sat = qoq.gemm_fp16_out_saturating(X8, s_x, blob, N, K, ws=ws)
+    torch().cuda.synchronize()
+    assert ws.status() == 0
+    assert np.array_equal(host(y).view(np.uint16), host(y_sat).view(np.uint16))
+    assert ws.control_clear()
+
+
 @pytest.mark.parametrize("N,K", [(128, 128), (128, 1152), (1152, 128), (896, 2176)])
 def test_tile_shapes(N, K):
     X = inputs.make_activations(24, K, seed=N + K)

@@ -397,7 +397,23 @@ __device__ __forceinline__ void add_second(uint32_t taddr, uint32_t (&v)[CH]) {
     for (int j = 0; j < CH; ++j) v[j] = (uint32_t)((int32_t)v[j] + (int32_t)w[j]);
 }
 
-template <int TOK, int MODE, bool PAIR>
+// Four codes (bytes of b4, each 0..15) to int8 q*s - z*s, saturated to
+// [-128, 127] per byte: the decode a kernel needs when dequantised weights can
+// leave the INT8 range (no protective range). Each pair of codes is widened to
+// 16-bit lanes, multiplied, shifted by z*s, clamped and narrowed again. With
+// the protective range the clamp never acts, so the bytes equal the
+// excess-128 decode's.
+__device__ __forceinline__ uint32_t decode4_saturating(uint32_t b4, uint32_t s, uint32_t zs2) {
+    uint32_t a = __byte_perm(b4, 0u, 0x4140) * s;   // codes 0, 1 in 16-bit lanes
+    uint32_t b = __byte_perm(b4, 0u, 0x4342) * s;   // codes 2, 3
+    a = __vsub2(a, zs2);
+    b = __vsub2(b, zs2);
+    a = __vmaxs2(__vmins2(a, 0x007F007Fu), 0xFF80FF80u);
+    b = __vmaxs2(__vmins2(b, 0x007F007Fu), 0xFF80FF80u);
+    return __byte_perm(a, b, 0x6420);
+}
+
+template <int TOK, int MODE, bool PAIR, bool SAT>
 __global__ void __launch_bounds__(kThreads, 1)
     qoq_gemm_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ CUtensorMap tmap_x,
                     const __grid_constant__ CUtensorMap tmap_y) {
@@ -686,6 +702,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (j < nk) {
                         const uint32_t sc = sz[j] & 0xFFu;
                         const uint32_t c4 = (uint32_t)(128 - (int)(int8_t)(sz[j] >> 8)) * 0x01010101u;
+                        const uint32_t zs2 = ((uint32_t)(int32_t)(int8_t)(sz[j] >> 8) & 0xFFFFu) * 0x00010001u;
                         uint32_t o[32];
 #pragma unroll
                         for (int c = 0; c < 4; ++c) {
@@ -694,7 +711,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                             for (int q = 0; q < 4; ++q) {
                                 const uint32_t lo = w[q] & 0x0F0F0F0Fu;
                                 const uint32_t hi = (w[q] >> 4) & 0x0F0F0F0Fu;
-                                if (MODE == 0) {
+                                if (MODE == 0 && SAT) {
+                                    o[8 * c + 2 * q] = decode4_saturating(lo, sc, zs2);
+                                    o[8 * c + 2 * q + 1] = decode4_saturating(hi, sc, zs2);
+                                } else if (MODE == 0) {
                                     o[8 * c + 2 * q] = (lo * sc + c4) ^ 0x80808080u;
                                     o[8 * c + 2 * q + 1] = (hi * sc + c4) ^ 0x80808080u;
                                 } else {
@@ -1040,7 +1060,7 @@ static bool encode_y_map(CUtensorMap *map, void *Y, int64_t M, int64_t N) {
 // once (clusters live inside one GPC, so this can be below SMs / 2); the
 // persistent schedule never launches more, so every cluster is resident and
 // stream-K partners can wait on one another. 0 when pairs cannot launch.
-template <int TOK, int MODE>
+template <int TOK, int MODE, bool SAT>
 static int pair_clusters_of(int dev) {
     using C = GemmCfg<TOK, MODE, true>;
     static std::once_flag once[64];
@@ -1058,9 +1078,9 @@ static int pair_clusters_of(int dev) {
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int n = 0;
-        if (cudaFuncSetAttribute(qoq_gemm_kernel<TOK, MODE, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(qoq_gemm_kernel<TOK, MODE, true, SAT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  C::kSmemBytes) != cudaSuccess ||
-            cudaOccupancyMaxActiveClusters(&n, qoq_gemm_kernel<TOK, MODE, true>, &cfg) != cudaSuccess)
+            cudaOccupancyMaxActiveClusters(&n, qoq_gemm_kernel<TOK, MODE, true, SAT>, &cfg) != cudaSuccess)
             n = 0;
         (void)cudaGetLastError();
         count[dev] = n;
@@ -1068,7 +1088,7 @@ static int pair_clusters_of(int dev) {
     return count[dev];
 }
 
-template <int TOK, int MODE, bool PAIR>
+template <int TOK, int MODE, bool PAIR, bool SAT = false>
 static qoq_status launch_gemm_t(const GemmArgs &a, cudaStream_t stream, int units_max) {
     using C = GemmCfg<TOK, MODE, PAIR>;
     int dev = 0;
@@ -1078,7 +1098,7 @@ static qoq_status launch_gemm_t(const GemmArgs &a, cudaStream_t stream, int unit
     static std::once_flag attr_once[64];
     static cudaError_t attr_err[64];
     std::call_once(attr_once[dev], [&] {
-        attr_err[dev] = cudaFuncSetAttribute(qoq_gemm_kernel<TOK, MODE, PAIR>,
+        attr_err[dev] = cudaFuncSetAttribute(qoq_gemm_kernel<TOK, MODE, PAIR, SAT>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     });
     if (attr_err[dev] != cudaSuccess) return QOQ_ERR_CUDA;
@@ -1147,7 +1167,7 @@ static qoq_status launch_gemm_t(const GemmArgs &a, cudaStream_t stream, int unit
     }
     cfg.attrs = attr;
     cfg.numAttrs = na;
-    return cudaLaunchKernelEx(&cfg, qoq_gemm_kernel<TOK, MODE, PAIR>, p, tmap, tmap_y) == cudaSuccess
+    return cudaLaunchKernelEx(&cfg, qoq_gemm_kernel<TOK, MODE, PAIR, SAT>, p, tmap, tmap_y) == cudaSuccess
                ? QOQ_OK
                : QOQ_ERR_CUDA;
 }
@@ -1166,14 +1186,35 @@ static qoq_status launch_gemm_mode(const GemmArgs &a, cudaStream_t stream) {
         case 128: return launch_gemm_t<128, MODE, false>(a, stream, ctas);
         default: {
             // 256-token tiles run on CTA pairs when the n-tiles pair up.
-            const int pairs = (a.N / kTileN) % 2 == 0 ? std::min(pair_clusters_of<256, MODE>(dev), kMaxGrid / 2) : 0;
+            const int pairs =
+                (a.N / kTileN) % 2 == 0 ? std::min(pair_clusters_of<256, MODE, false>(dev), kMaxGrid / 2) : 0;
             if (pairs > 0) return launch_gemm_t<256, MODE, true>(a, stream, pairs);
             return launch_gemm_t<256, MODE, false>(a, stream, ctas);
         }
     }
 }
 
+// The saturating-decode ablation is built for two token tiles: 16 (decode)
+// and 256 on CTA pairs (prefill).
+static qoq_status launch_gemm_saturating(const GemmArgs &a, cudaStream_t stream) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return QOQ_ERR_CUDA;
+    const int sms = sm_count_of(dev);
+    if (sms <= 0) return QOQ_ERR_CUDA;
+    switch (token_tile_for(a.M, a.N, a.K)) {
+        case 16: return launch_gemm_t<16, 0, false, true>(a, stream, std::min(sms, kMaxGrid));
+        case 256: {
+            const int pairs =
+                (a.N / kTileN) % 2 == 0 ? std::min(pair_clusters_of<256, 0, true>(dev), kMaxGrid / 2) : 0;
+            if (pairs > 0) return launch_gemm_t<256, 0, true, true>(a, stream, pairs);
+            return QOQ_ERR_UNSUPPORTED;
+        }
+        default: return QOQ_ERR_UNSUPPORTED;
+    }
+}
+
 qoq_status launch_gemm(const GemmArgs &a, cudaStream_t stream) {
+    if (a.saturating) return a.group ? launch_gemm_saturating(a, stream) : QOQ_ERR_UNSUPPORTED;
     return a.group ? launch_gemm_mode<0>(a, stream) : launch_gemm_mode<1>(a, stream);
 }
 

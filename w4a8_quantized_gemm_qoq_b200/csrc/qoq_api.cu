@@ -25,7 +25,7 @@ qoq_status check_group(int group) {
 
 qoq_status gemm_common(const int8_t *X8, const void *s_x, const int32_t *rowsum, const void *blob, int64_t M,
                        int64_t N, int64_t K, int group, void *out, bool fp16_out, void *ws, size_t *ws_bytes,
-                       void *stream) {
+                       void *stream, bool saturating = false) {
     if (ws_bytes == nullptr) return QOQ_ERR_INVALID_ARG;
     if (M < 0 || M > INT32_MAX) return QOQ_ERR_INVALID_ARG;
     qoq_status st = check_nk(N, K);
@@ -56,6 +56,7 @@ qoq_status gemm_common(const int8_t *X8, const void *s_x, const int32_t *rowsum,
     a.out = out;
     a.fp16_out = fp16_out;
     a.ws = ws;
+    a.saturating = saturating;
     return launch_gemm(a, static_cast<cudaStream_t>(stream));
 }
 
@@ -139,6 +140,17 @@ qoq_status qoq_gemm_fp16_out(const int8_t *X8, const void *s_x_fp16, const int32
                              size_t *workspace_bytes, void *stream) {
     return gemm_common(X8, s_x_fp16, rowsum, blob, M, N, K, group_size, Y_fp16, true, workspace,
                        workspace_bytes, stream);
+}
+
+qoq_status qoq_gemm_fp16_out_saturating(const int8_t *X8, const void *s_x_fp16, const void *blob, int64_t M,
+                                        int64_t N, int64_t K, int group_size, void *Y_fp16, void *workspace,
+                                        size_t *workspace_bytes, void *stream) {
+    // Built for group_size 128 and two token tiles: M <= 16, and M > 512 on
+    // CTA pairs (N / 128 even).
+    if (group_size != kGroup) return QOQ_ERR_UNSUPPORTED;
+    if (M > 16 && (M <= 512 || token_tile_for(M, N, K) != 256 || (N / kTileN) % 2 != 0)) return QOQ_ERR_UNSUPPORTED;
+    return gemm_common(X8, s_x_fp16, nullptr, blob, M, N, K, group_size, Y_fp16, true, workspace, workspace_bytes,
+                       stream, true);
 }
 
 const char *qoq_status_string(qoq_status status) {

@@ -105,6 +105,10 @@ struct GemmArgs {
     void *out;          // int32 [M][N] or fp16 [M][N]
     bool fp16_out;
     void *ws;
+    // Ablation only (qoq_gemm_fp16_out_saturating): decode the weights with
+    // per-byte saturation to [-128, 127], as a kernel without the protective
+    // range would have to.
+    bool saturating = false;
 };
 qoq_status launch_gemm(const GemmArgs &a, cudaStream_t stream);
 

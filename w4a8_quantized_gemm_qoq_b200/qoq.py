@@ -45,6 +45,8 @@ def lib() -> ctypes.CDLL:
         L.qoq_silu_mul_quant.argtypes = [vp, i64, i64, vp, vp, vp, vp]
         L.qoq_w4a8_gemm.argtypes = [vp, vp, vp, i64, i64, i64, i32, vp, vp, sz, vp]
         L.qoq_gemm_fp16_out.argtypes = [vp, vp, vp, vp, i64, i64, i64, i32, vp, vp, sz, vp]
+        L.qoq_gemm_fp16_out_saturating.argtypes = [vp, vp, vp, i64, i64, i64, i32, vp, vp, sz, vp]
+        L.qoq_gemm_fp16_out_saturating.restype = ctypes.c_int
         L.qoq_watchdog_selftest.argtypes = [vp, i64, vp]
         L.qoq_watchdog_selftest.restype = ctypes.c_int
         L.qoq_status_string.argtypes = [ctypes.c_int]
@@ -221,6 +223,21 @@ def gemm_fp16_out(X8, s_x, blob, N, K, group_size=GROUP, rowsum=None, ws=None, Y
     _check("qoq_gemm_fp16_out", lib().qoq_gemm_fp16_out(_ptr(X8), _ptr(s_x), _ptr(rowsum), _ptr(blob), M, N, K,
                                                         group_size, _ptr(Y), _ptr(ws.buf), ctypes.byref(n),
                                                         _stream(stream)))
+    return Y
+
+
+def gemm_fp16_out_saturating(X8, s_x, blob, N, K, ws=None, Y=None, stream=None):
+    """The same GEMM with a saturating weight decode (the protective-range
+    ablation; group_size 128; M <= 16, or M > 512 with N / 128 even)."""
+    import torch
+    X8 = _cuda_tensor(X8, torch.int8, "X8")
+    M = X8.shape[0]
+    ws = ws or Workspace.for_shape(M, N, K, GROUP, X8.device)
+    Y = torch.empty((M, N), dtype=torch.float16, device=X8.device) if Y is None else Y
+    n = ctypes.c_size_t(ws.buf.numel())
+    _check("qoq_gemm_fp16_out_saturating",
+           lib().qoq_gemm_fp16_out_saturating(_ptr(X8), _ptr(s_x), _ptr(blob), M, N, K, GROUP, _ptr(Y),
+                                              _ptr(ws.buf), ctypes.byref(n), _stream(stream)))
     return Y
 
 
