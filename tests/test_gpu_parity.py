@@ -58,6 +58,17 @@ def test_paired_ctas_ragged_tokens(M):
     check_full(X, W, 0, "pairs per-channel M=%d" % M)
 
 
+@pytest.mark.parametrize("M", [600, 1000])
+def test_unpaired_wide_tiles_odd_ntiles(M):
+    """256-token tiles whose n-tiles do not pair up (N/128 odd) run on single
+    CTAs: two issuers on the two token halves, one dequant and two epilogue
+    warpgroups; both quantisation modes."""
+    X = inputs.make_activations(M, 640, seed=400 + M)
+    W = inputs.make_weights(384, 640, seed=400 + M)
+    check_full(X, W, 128, "unpaired M=%d" % M)
+    check_full(X, W, 0, "unpaired per-channel M=%d" % M)
+
+
 @pytest.mark.parametrize("M,N,K", [(1, 256, 512), (16, 1024, 1280), (600, 512, 640), (2048, 28672, 4096)])
 def test_saturating_decode_ablation_is_bit_identical(M, N, K):
     """The protective-range ablation decodes the weights with per-byte
