@@ -12,6 +12,9 @@ Contents
   producers.py the fused activation producers (RMSNorm or SiLU-gated product,
                then per-token INT8 quantisation) in plain numpy and Python
                integers.
+  kv4.py       KV4 decode attention (per-head dynamic asymmetric INT4 K/V,
+               grouped-query softmax attention) in plain numpy; no kernel
+               implements it yet.
 
 Pinning: every function here is checked in ``tests/test_oracle_*.py`` against
 something other than itself -- exact rational arithmetic (``fractions``),
@@ -22,3 +25,4 @@ from a printed value.
 """
 from .qoq_ref import *  # noqa: F401,F403
 from . import producers  # noqa: F401
+from . import kv4  # noqa: F401

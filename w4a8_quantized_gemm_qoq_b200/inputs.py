@@ -18,9 +18,14 @@ activations are not available here, so these stand in for them):
   * GU (merged gate/up projection output, FP16, [M][2I]): gate half
     N(0, 2^2) so that SiLU sees both its negative tail and its linear part,
     up half N(0, 1); 4 outlier columns x20 in each half.
+  * decode attention (GQA, one query token per sequence): q [B][Hq][D],
+    K and V [B][Hkv][T][D], FP16, i.i.d. N(0, 1); in K, 2 channels per KV
+    head (drawn first) are multiplied by 8, the outlier Key channels the
+    pages describe.
 Streams: numpy ``Generator(PCG64([seed, 1]))`` for W,
-``Generator(PCG64([seed, 2]))`` for X, ``[seed, 4]`` for gamma and
-``[seed, 5]`` for GU, so each can be drawn independently.
+``Generator(PCG64([seed, 2]))`` for X, ``[seed, 4]`` for gamma,
+``[seed, 5]`` for GU and ``[seed, 6]`` for the attention inputs, so each can
+be drawn independently.
 """
 from __future__ import annotations
 
@@ -109,3 +114,21 @@ def make_gate_up(M: int, I: int, seed: int = 0) -> np.ndarray:
         cols = half * I + rng.choice(I, size=min(N_OUTLIERS, I), replace=False)
         gu[:, cols] *= np.float32(OUTLIER_GAIN)
     return gu.astype(np.float16)
+
+
+LLAMA3_8B_ATTN = dict(Hq=32, Hkv=8, D=128)   # Llama-3-8B attention heads (GQA 4:1)
+N_KEY_OUTLIERS = 2
+KEY_OUTLIER_GAIN = 8.0
+
+
+def make_decode_attention(B: int, T: int, Hq: int, Hkv: int, D: int, seed: int = 0):
+    """FP16 (q [B][Hq][D], K [B][Hkv][T][D], V [B][Hkv][T][D]) ~ N(0, 1), with
+    2 outlier channels x8 per KV head in K."""
+    rng = _rng(seed, 6)
+    cols = np.stack([rng.choice(D, size=min(N_KEY_OUTLIERS, D), replace=False) for _ in range(Hkv)])
+    q = rng.standard_normal((B, Hq, D), dtype=np.float32)
+    K = rng.standard_normal((B, Hkv, T, D), dtype=np.float32)
+    V = rng.standard_normal((B, Hkv, T, D), dtype=np.float32)
+    for h in range(Hkv):
+        K[:, h, :, cols[h]] *= np.float32(KEY_OUTLIER_GAIN)
+    return q.astype(np.float16), K.astype(np.float16), V.astype(np.float16)
