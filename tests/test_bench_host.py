@@ -19,9 +19,8 @@ def test_reference_arm_json_line():
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
                           "--warmup", "1"], cwd=ROOT, capture_output=True, text=True, timeout=300, check=True)
     d = json.loads(out.stdout.strip().splitlines()[-1])
-    with open(os.path.join(ROOT, "BASELINE.json")) as f:
-        metric = json.load(f)["metric"]
-    assert d["impl"] == "reference" and d["metric"] == metric
+    import bench
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC
     for k in ("value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
               "vs_baseline", "dtype", "data", "config"):
         assert k in d, k
