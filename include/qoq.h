@@ -220,9 +220,12 @@ qoq_status qoq_gemm_fp16_out_saturating(const int8_t *X8, const void *s_x_fp16, 
  * Same computation and arguments as qoq_gemm_fp16_out, except that the
  * stream-K scratch lives in one fixed 8 MiB device array inside the library,
  * which every GPU that loads the library keeps until the process exits. That
- * bounds the problem: it needs 1280 + (SM count) * T * 512 bytes, T being the
- * token tile the library picks for (M, N, K) (16 for M <= 16, 32 for M <= 32,
- * 32 or 64 for M <= 64), so M <= 64 on a 148-SM B200; larger problems return
+ * bounds the problem: the call needs 1280 + C * T * 512 bytes, where T is the
+ * token tile the library picks for (M, N, K) and C the CTAs of the launch
+ * (min(SM count, 256, token tiles * N/128 * K/128); twice the CTA pairs for
+ * 256-token tiles). On a 148-SM B200 every problem whose token tile is at
+ * most 64 fits: all M <= 64, and M up to 256 where few weight tiles make the
+ * library keep 64-token tiles (e.g. N = K = 4096). Larger problems return
  * QOQ_ERR_WORKSPACE and launch nothing.
  *
  * status: optional device int32; when non-NULL the call copies the device

@@ -409,6 +409,42 @@ def w4a8_gemm_per_channel(X8, rowsum, q, z) -> np.ndarray:
     return per_channel_correct(accq, rowsum, z)
 
 
+# ---------------------------------------------------------------------------
+# Saturating weight decode: what a kernel without the protective range does
+# [P3-4]
+# ---------------------------------------------------------------------------
+
+
+def dequantize_saturating(q: np.ndarray, s: np.ndarray, zs: np.ndarray, g: int = GROUP) -> np.ndarray:
+    """Second-level decode clamped to INT8, for codes that may leave it.
+
+    Wsat[n,k] = clamp(q[n,k] * s[n,j] - zs[n,j], -128, 127),  j = k // g
+
+    with q the UINT4 codes [N][K], s the integer group scales (uint8)
+    [N][K/g] and zs = z*s (int8) [N][K/g]. The products are exact integers.
+
+    reading: [P3-4] shrinks the first level to [-119, 119] so that the
+    dequantised value q*s - z*s never leaves INT8; without that range the
+    main loop must saturate, which the pages say costs up to 67% of the
+    GEMM's throughput. Saturation is read as the usual clamp of the exact
+    integer to the INT8 range. On protective-range groups the clamp never
+    acts and Wsat equals the level-2 Wint.
+    """
+    q = np.asarray(q, dtype=np.uint8).astype(np.int64)
+    N, K = q.shape
+    s = np.asarray(s, dtype=np.uint8).astype(np.int64)
+    zs = np.asarray(zs, dtype=np.int8).astype(np.int64)
+    assert s.shape == (N, K // g) and zs.shape == (N, K // g)
+    raw = q.reshape(N, K // g, g) * s[:, :, None] - zs[:, :, None]
+    return np.clip(raw, -128, 127).reshape(N, K).astype(np.int8)
+
+
+def gemm_fp16_saturating(X8: np.ndarray, s_x: np.ndarray, q, s, zs, s_w) -> np.ndarray:
+    """FP16 output of the GEMM whose weights are decoded with saturation:
+    the exact INT32 product with Wsat, then the epilogue."""
+    return epilogue_fp16(gemm_int(X8, dequantize_saturating(q, s, zs)), s_x, s_w)
+
+
 def reference_forward(X: np.ndarray, W: np.ndarray, group: int = GROUP) -> dict:
     """Whole path on FP16 inputs: act quant, weight quant + pack, GEMM, epilogue."""
     X8, s_x, rowsum = quantize_act_per_token(X)

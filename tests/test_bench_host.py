@@ -20,7 +20,11 @@ def test_reference_arm_json_line():
                           "--warmup", "1"], cwd=ROOT, capture_output=True, text=True, timeout=300, check=True)
     d = json.loads(out.stdout.strip().splitlines()[-1])
     import bench
-    assert d["impl"] == "reference" and d["metric"] == bench.METRIC
+    # The contract's metric string, spelled out here independently of the
+    # constant bench.py prints, so that a drift in either is caught.
+    contract = "W4A8 GEMM TOPS and % of roofline vs M on Llama-3-8B linear shapes (1 B200)"
+    assert bench.METRIC == contract
+    assert d["impl"] == "reference" and d["metric"] == contract
     for k in ("value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
               "vs_baseline", "dtype", "data", "config"):
         assert k in d, k

@@ -164,29 +164,74 @@ def test_bad_blob_header_reported_on_device():
 
 
 # ------------------------------------------------------- full sizes, sampled oracle
+# Every (shape, M) of the four full-size configurations. The stream-K split
+# (data-parallel waves, tail boundaries, owner and contributor sets) changes
+# with every (M, N, K), so no grid point stands in for another. The M values
+# of one shape share its weights (seeded per shape).
 
-@pytest.mark.parametrize("K,N", [(4096, 6144), (4096, 4096), (4096, 28672), (14336, 4096)])
-@pytest.mark.parametrize("M", [1, 4, 16, 64, 256])
+_L3 = [(K, N) for (K, N, _) in inputs.LLAMA3_8B]
+_QW = [(K, N) for (K, N, _) in inputs.QWEN15_72B]
+_L2 = [(K, N) for (K, N, _) in inputs.LLAMA2_7B]
+
+
+@pytest.mark.parametrize("K,N,M", [(K, N, M) for (K, N) in _L3 for M in inputs.DECODE_M])
 def test_llama3_8b_decode_shapes(M, K, N):
-    check_sampled(M, N, K, 128, seed=M + N)
+    check_sampled(M, N, K, 128, seed=M + N, wseed=N + K)
 
 
-@pytest.mark.parametrize("K,N", [(4096, 28672), (14336, 4096)])
-@pytest.mark.parametrize("M", [2048, 16384])
+@pytest.mark.parametrize("K,N,M", [(K, N, M) for (K, N) in _L3 for M in inputs.PREFILL_M])
 def test_llama3_8b_prefill_shapes(M, K, N):
-    check_sampled(M, N, K, 128, seed=M + K, token_scale_span=(-3, 1), rows=12)
+    check_sampled(M, N, K, 128, seed=M + K, wseed=N + K, token_scale_span=(-3, 1), rows=12)
 
 
-@pytest.mark.parametrize("K,N,M", [(8192, 24576, 1), (8192, 8192, 16), (8192, 49152, 128), (24576, 8192, 512),
-                                   (8192, 8192, 4096)])
+@pytest.mark.parametrize("K,N,M", [(K, N, M) for (K, N) in _QW for M in inputs.QWEN_M])
 def test_qwen15_72b_shapes(M, K, N):
-    check_sampled(M, N, K, 128, seed=N + M, std=0.01, rows=12)
+    check_sampled(M, N, K, 128, seed=N + M, wseed=N + K, std=0.01, rows=12)
 
 
-@pytest.mark.parametrize("K,N", [(4096, 12288), (4096, 4096), (4096, 22016), (11008, 4096)])
-@pytest.mark.parametrize("M", [1, 8, 64, 1024])
+@pytest.mark.parametrize("K,N,M", [(K, N, M) for (K, N) in _L2 for M in inputs.PER_CHANNEL_M])
 def test_llama2_7b_per_channel_shapes(M, K, N):
-    check_sampled(M, N, K, 0, seed=K + M, rows=12)
+    check_sampled(M, N, K, 0, seed=K + M, wseed=N + K, rows=12)
+
+
+# ------------------------------------- saturating decode where the clamp acts
+
+def _saturating_blob(N, K, seed):
+    """Codes, integer scales and zero terms drawn so that q*s - z*s leaves
+    INT8 in many places (scales up to 40, any int8 zero term), packed by the
+    oracle's packer; a quarter of the rows keep protective-range groups."""
+    rng = np.random.default_rng(seed)
+    q = rng.integers(0, 16, size=(N, K)).astype(np.uint8)
+    s = rng.integers(1, 41, size=(N, K // 128)).astype(np.uint8)
+    zs = rng.integers(-128, 128, size=(N, K // 128)).astype(np.int8)
+    prot = oracle.quantize_weights_group(inputs.make_weights(N // 4, K, seed=seed))
+    q[: N // 4], s[: N // 4], zs[: N // 4] = prot["q"], prot["s"], prot["zs"]
+    s_w = (rng.uniform(1e-3, 4e-3, size=N)).astype(np.float16)
+    raw = q.astype(np.int64).reshape(N, K // 128, 128) * s.astype(np.int64)[:, :, None] - \
+        zs.astype(np.int64)[:, :, None]
+    assert (raw > 127).mean() > 0.2, "the fixture must make the clamp act"
+    return q, s, zs, s_w, oracle.pack_blob_group(q, s, zs, s_w)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 256, 512), (16, 384, 640), (600, 512, 640), (1000, 768, 384)])
+def test_saturating_decode_matches_oracle_where_the_clamp_acts(M, N, K):
+    """The protective-range ablation on a blob whose dequantised weights
+    leave INT8: the saturating GEMM equals the oracle's clamp(q*s - z*s,
+    -128, 127) decode followed by the exact INT32 product and the epilogue,
+    bit for bit, on both token tiles it is built for (16, and 256 on CTA
+    pairs)."""
+    X = inputs.make_activations(M, K, seed=500 + M)
+    q, s, zs, s_w, blob_h = _saturating_blob(N, K, seed=M + N)
+    X8o, s_xo, _ = oracle.quantize_act_per_token(X)
+    want = oracle.gemm_fp16_saturating(X8o, s_xo, q, s, zs, s_w)
+    X8, s_x, rs = qoq.quantize_act_per_token(dev(X))
+    ws = qoq.Workspace.for_shape(M, N, K, 128)
+    y = qoq.gemm_fp16_out_saturating(X8, s_x, dev(blob_h), N, K, ws=ws)
+    torch().cuda.synchronize()
+    assert ws.status() == 0
+    assert np.array_equal(host(X8), X8o)
+    assert np.array_equal(host(y).view(np.uint16), want.view(np.uint16))
+    assert ws.control_clear()
 
 
 # ------------------------------------------ back-to-back graph replays

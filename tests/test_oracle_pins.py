@@ -261,6 +261,85 @@ def test_level2_grid_groups_roundtrip():
     assert np.array_equal(Wint.astype(np.int64), Q8)
 
 
+# ------------------------------------------- saturating decode (no protective range)
+
+def _saturating_golden_rows(golden_dir):
+    return [tuple(int(t) for t in row.split()) for row in _golden(golden_dir, "saturating_decode.txt")]
+
+
+def _check_saturating_golden(fn, rows):
+    """Each hand-worked (q, s, zs) -> Wsat row sits in its own group of a
+    two-group row: group 0 holds row i's code at column i, group 1 row
+    (i + 1)'s code at column 128 + i; the other codes are 0."""
+    n = len(rows)
+    q = np.zeros((n, 256), dtype=np.uint8)
+    s = np.zeros((n, 2), dtype=np.uint8)
+    zs = np.zeros((n, 2), dtype=np.int8)
+    want = np.zeros((n, 2), dtype=np.int64)
+    for i in range(n):
+        a, b = rows[i], rows[(i + 1) % n]
+        q[i, i], s[i, 0], zs[i, 0], want[i, 0] = a
+        q[i, 128 + i], s[i, 1], zs[i, 1], want[i, 1] = b
+    got = fn(q, s, zs).astype(np.int64)
+    return all(got[i, i] == want[i, 0] and got[i, 128 + i] == want[i, 1] for i in range(n))
+
+
+def test_saturating_decode_golden(golden_dir):
+    rows = _saturating_golden_rows(golden_dir)
+    assert len(rows) >= 10
+    assert _check_saturating_golden(oracle.dequantize_saturating, rows)
+
+
+def test_saturating_decode_planted_mistakes_fail_the_golden(golden_dir):
+    """A top bound of 128 (a 16-bit clamp), an added instead of subtracted
+    zero term, and the group index taken modulo instead of divided each fail
+    the hand-worked rows."""
+    rows = _saturating_golden_rows(golden_dir)
+
+    def top128(q, s, zs):
+        raw = q.astype(np.int64).reshape(len(q), 2, 128) * s.astype(np.int64)[:, :, None] - \
+            zs.astype(np.int64)[:, :, None]
+        return np.clip(raw, -128, 128).reshape(len(q), 256)
+
+    def plus_zero(q, s, zs):
+        return oracle.dequantize_saturating(q, s, -zs.astype(np.int64).clip(-127, 127).astype(np.int8))
+
+    def group_mod(q, s, zs):
+        j = np.arange(256) % 2
+        raw = q.astype(np.int64) * s.astype(np.int64)[:, j] - zs.astype(np.int64)[:, j]
+        return np.clip(raw, -128, 127)
+
+    for bad in (top128, plus_zero, group_mod):
+        assert not _check_saturating_golden(bad, rows), bad.__name__
+
+
+def test_saturating_decode_reduces_to_level2_on_protective_groups():
+    """On groups from the protective range the clamp never acts: the
+    saturating decode equals the second level's own dequantised weights."""
+    rng = np.random.default_rng(21)
+    Q8 = rng.integers(-119, 120, size=(64, 1024)).astype(np.int8)
+    Q8[:8] = np.clip(rng.integers(-119, 120, size=(8, 1)) + rng.integers(-3, 4, size=(8, 1024)), -119, 119)
+    q, s, z, Wint = oracle.quantize_level2(Q8)
+    zs = (z.astype(np.int64) * s.astype(np.int64)).astype(np.int8)
+    assert np.array_equal(oracle.dequantize_saturating(q, s, zs), Wint)
+
+
+def test_saturating_decode_bounds_and_monotone():
+    """Over random codes, scales and zero terms that leave INT8: every value
+    is in [-128, 127], values are non-decreasing in the code for a fixed
+    (s, zs), and the clamp acts on a good share of them."""
+    rng = np.random.default_rng(22)
+    N, K = 32, 2048
+    s = rng.integers(0, 256, size=(N, K // 128)).astype(np.uint8)
+    zs = rng.integers(-128, 128, size=(N, K // 128)).astype(np.int8)
+    q = np.tile(np.arange(16, dtype=np.uint8), (N, K // 16))
+    W = oracle.dequantize_saturating(q, s, zs).astype(np.int64)
+    assert W.min() >= -128 and W.max() <= 127
+    steps = np.diff(W.reshape(N, K // 16, 16), axis=2)
+    assert steps.min() >= 0
+    assert (W == 127).mean() > 0.3
+
+
 # -------------------------------------------------------------- per-channel variant
 
 def test_per_channel_bruteforce_exact():

@@ -1135,6 +1135,9 @@ static qoq_status launch_gemm_t(const GemmArgs &a, cudaStream_t stream, int unit
     p.total_blocks = (uint32_t)blocks;
     // Schedule units (CTAs, or CTA pairs): at most one per SM (pair), all resident.
     p.grid = (int)std::min<long long>(units_max, blocks);
+    // The partial-sum slots are indexed by CTA: the workspace must hold one
+    // per CTA of this grid.
+    if (scratch_bytes_for_grid(TOK, PAIR ? 2 * p.grid : p.grid) > a.ws_capacity) return QOQ_ERR_WORKSPACE;
     // Whole tiles in data-parallel waves while at least one to two waves of
     // tiles remain for the stream-K tail, which evens out the last wave.
     const long long tiles = (long long)p.MT * p.NTw;
@@ -1172,45 +1175,70 @@ static qoq_status launch_gemm_t(const GemmArgs &a, cudaStream_t stream, int unit
                : QOQ_ERR_CUDA;
 }
 
+// Launch plan of a problem: token tile, CTA pairs or not, and the number of
+// schedule units (CTAs, or CTA pairs) the persistent grid may use.
+struct GemmPlan {
+    int tok;
+    bool pair;
+    int units_max;
+};
+
+static bool plan_gemm(int64_t M, int64_t N, int64_t K, int mode, bool saturating, GemmPlan *pl) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return false;
+    const int sms = sm_count_of(dev);
+    if (sms <= 0) return false;
+    pl->tok = token_tile_for(M, N, K);
+    pl->pair = false;
+    pl->units_max = std::min(sms, kMaxGrid);
+    if (pl->tok == 256 && (N / kTileN) % 2 == 0) {
+        // 256-token tiles run on CTA pairs when the n-tiles pair up.
+        int clusters = 0;
+        if (saturating)
+            clusters = pair_clusters_of<256, 0, true>(dev);
+        else
+            clusters = mode == 0 ? pair_clusters_of<256, 0, false>(dev) : pair_clusters_of<256, 1, false>(dev);
+        const int pairs = std::min(clusters, kMaxGrid / 2);
+        if (pairs > 0) {
+            pl->pair = true;
+            pl->units_max = pairs;
+        }
+    }
+    return true;
+}
+
+size_t gemm_scratch_bytes(int64_t M, int64_t N, int64_t K, int group, bool saturating) {
+    GemmPlan pl;
+    if (!plan_gemm(M, N, K, group ? 0 : 1, saturating, &pl)) return 0;
+    const int64_t NTw = pl.pair ? N / kTileN / 2 : N / kTileN;
+    const int64_t blocks = ((M + pl.tok - 1) / pl.tok) * NTw * (K / kTileK);
+    const int64_t units = std::min<int64_t>(pl.units_max, blocks);
+    return scratch_bytes_for_grid(pl.tok, pl.pair ? 2 * units : units);
+}
+
 template <int MODE>
 static qoq_status launch_gemm_mode(const GemmArgs &a, cudaStream_t stream) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return QOQ_ERR_CUDA;
-    const int sms = sm_count_of(dev);
-    if (sms <= 0) return QOQ_ERR_CUDA;
-    const int ctas = std::min(sms, kMaxGrid);
-    switch (token_tile_for(a.M, a.N, a.K)) {
-        case 16: return launch_gemm_t<16, MODE, false>(a, stream, ctas);
-        case 32: return launch_gemm_t<32, MODE, false>(a, stream, ctas);
-        case 64: return launch_gemm_t<64, MODE, false>(a, stream, ctas);
-        case 128: return launch_gemm_t<128, MODE, false>(a, stream, ctas);
-        default: {
-            // 256-token tiles run on CTA pairs when the n-tiles pair up.
-            const int pairs =
-                (a.N / kTileN) % 2 == 0 ? std::min(pair_clusters_of<256, MODE, false>(dev), kMaxGrid / 2) : 0;
-            if (pairs > 0) return launch_gemm_t<256, MODE, true>(a, stream, pairs);
-            return launch_gemm_t<256, MODE, false>(a, stream, ctas);
-        }
+    GemmPlan pl;
+    if (!plan_gemm(a.M, a.N, a.K, MODE, false, &pl)) return QOQ_ERR_CUDA;
+    switch (pl.tok) {
+        case 16: return launch_gemm_t<16, MODE, false>(a, stream, pl.units_max);
+        case 32: return launch_gemm_t<32, MODE, false>(a, stream, pl.units_max);
+        case 64: return launch_gemm_t<64, MODE, false>(a, stream, pl.units_max);
+        case 128: return launch_gemm_t<128, MODE, false>(a, stream, pl.units_max);
+        default:
+            return pl.pair ? launch_gemm_t<256, MODE, true>(a, stream, pl.units_max)
+                           : launch_gemm_t<256, MODE, false>(a, stream, pl.units_max);
     }
 }
 
 // The saturating-decode ablation is built for two token tiles: 16 (decode)
 // and 256 on CTA pairs (prefill).
 static qoq_status launch_gemm_saturating(const GemmArgs &a, cudaStream_t stream) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return QOQ_ERR_CUDA;
-    const int sms = sm_count_of(dev);
-    if (sms <= 0) return QOQ_ERR_CUDA;
-    switch (token_tile_for(a.M, a.N, a.K)) {
-        case 16: return launch_gemm_t<16, 0, false, true>(a, stream, std::min(sms, kMaxGrid));
-        case 256: {
-            const int pairs =
-                (a.N / kTileN) % 2 == 0 ? std::min(pair_clusters_of<256, 0, true>(dev), kMaxGrid / 2) : 0;
-            if (pairs > 0) return launch_gemm_t<256, 0, true, true>(a, stream, pairs);
-            return QOQ_ERR_UNSUPPORTED;
-        }
-        default: return QOQ_ERR_UNSUPPORTED;
-    }
+    GemmPlan pl;
+    if (!plan_gemm(a.M, a.N, a.K, 0, true, &pl)) return QOQ_ERR_CUDA;
+    if (pl.tok == 16) return launch_gemm_t<16, 0, false, true>(a, stream, pl.units_max);
+    if (pl.tok == 256 && pl.pair) return launch_gemm_t<256, 0, true, true>(a, stream, pl.units_max);
+    return QOQ_ERR_UNSUPPORTED;
 }
 
 qoq_status launch_gemm(const GemmArgs &a, cudaStream_t stream) {

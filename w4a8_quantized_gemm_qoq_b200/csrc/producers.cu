@@ -13,7 +13,7 @@
 // then s = FP16(max_k |h| / 127), X8 = clamp(RNE(h / FP32(s)), -127, 127)
 // (0 where s == 0) and rowsum = sum_k X8. Every floating-point step is one
 // correctly rounded binary32 operation (__fdiv_rn, __fsqrt_rn, ...; the
-// quantising division takes the exact reciprocal shortcut of qoq_device.cuh;
+// quantising division takes the exact reciprocal shortcut of quant_math.cuh;
 // no contraction), the sum of squares is exact (128-bit integer accumulation,
 // then one rounding), and e^x is computed here from Cody and Waite's argument
 // reduction and the degree-7 Taylor polynomial, so that the codes these

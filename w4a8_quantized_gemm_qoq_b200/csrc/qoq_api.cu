@@ -57,6 +57,7 @@ qoq_status gemm_common(const int8_t *X8, const void *s_x, const int32_t *rowsum,
     a.fp16_out = fp16_out;
     a.ws = ws;
     a.saturating = saturating;
+    a.ws_capacity = *ws_bytes;
     return launch_gemm(a, static_cast<cudaStream_t>(stream));
 }
 

@@ -77,9 +77,15 @@ inline int token_tile_for(int64_t M, int64_t N, int64_t K) {
 // partial tiles [kMaxGrid][tok][128] (scratch).
 static_assert(256 + 4 * kMaxGrid == QOQ_WORKSPACE_CONTROL_BYTES, "workspace control layout");
 
+// Workspace bytes a launch of `grid_ctas` CTAs with token tile `tok` uses:
+// the control words, then one partial tile per CTA.
+inline size_t scratch_bytes_for_grid(int tok, int64_t grid_ctas) {
+    return 256 + sizeof(int32_t) * kMaxGrid + sizeof(int32_t) * (size_t)grid_ctas * tok * kTileN;
+}
+
+// Workspace size the size query reports: enough for any grid (kMaxGrid CTAs).
 inline size_t workspace_bytes_for(int64_t M, int64_t N, int64_t K) {
-    const int tok = token_tile_for(M, N, K);
-    return 256 + sizeof(int32_t) * kMaxGrid + sizeof(int32_t) * (size_t)kMaxGrid * tok * kTileN;
+    return scratch_bytes_for_grid(token_tile_for(M, N, K), kMaxGrid);
 }
 
 // Kernel launchers (return cudaSuccess or the launch error).
@@ -109,7 +115,15 @@ struct GemmArgs {
     // per-byte saturation to [-128, 127], as a kernel without the protective
     // range would have to.
     bool saturating = false;
+    // Bytes of `ws` the caller provides; a launch whose grid would need more
+    // returns QOQ_ERR_WORKSPACE without launching.
+    size_t ws_capacity = 0;
 };
 qoq_status launch_gemm(const GemmArgs &a, cudaStream_t stream);
+
+// Workspace bytes the launch for this problem on the current device will
+// actually use (its grid, not the kMaxGrid bound): the same grid rule as
+// launch_gemm. Returns 0 if the device cannot be queried.
+size_t gemm_scratch_bytes(int64_t M, int64_t N, int64_t K, int group, bool saturating = false);
 
 }  // namespace qoq

@@ -14,7 +14,8 @@
 
 namespace {
 
-// 8 MiB: enough for token tiles of up to 64 tokens (M <= 64) on a 148-SM GPU.
+// 8 MiB: the control words plus one partial tile per CTA, for token tiles of
+// up to 64 tokens on a GPU of up to 256 SMs (1280 + 256 * 64 * 512 bytes).
 constexpr size_t kStaticScratchBytes = size_t(8) << 20;
 
 static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
@@ -56,17 +57,13 @@ extern "C" qoq_status qoq_gemm_fp16_out_static_ws(const int8_t *X8, const void *
         (reinterpret_cast<uintptr_t>(status) & 3u))
         return QOQ_ERR_ALIGNMENT;
 
-    int dev = 0, sms = 0;
+    int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return QOQ_ERR_CUDA;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
-        return QOQ_ERR_CUDA;
-    // Scratch this call needs: control words plus one partial tile per CTA
-    // of the persistent grid.
-    const int64_t tok = token_tile_for(M, N, K);
-    const int64_t blocks = ((M + tok - 1) / tok) * (N / kTileN) * (K / kTileK);
-    int64_t grid = sms < kMaxGrid ? sms : kMaxGrid;
-    if (blocks < grid) grid = blocks;
-    const size_t need = (size_t)QOQ_WORKSPACE_CONTROL_BYTES + (size_t)grid * tok * kTileN * sizeof(int32_t);
+    // Scratch this call needs: the control words plus one partial tile per
+    // CTA of the grid the launch will use (the launcher's own rule, which
+    // checks the same bound again before it launches).
+    const size_t need = gemm_scratch_bytes(M, N, K, group_size);
+    if (need == 0) return QOQ_ERR_CUDA;
     if (need > kStaticScratchBytes) return QOQ_ERR_WORKSPACE;
 
     void *scratch = nullptr;
@@ -89,6 +86,7 @@ extern "C" qoq_status qoq_gemm_fp16_out_static_ws(const int8_t *X8, const void *
     a.out = Y_fp16;
     a.fp16_out = true;
     a.ws = scratch;
+    a.ws_capacity = kStaticScratchBytes;
     st = launch_gemm(a, s);
     if (st != QOQ_OK) return st;
     if (status != nullptr &&
