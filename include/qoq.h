@@ -163,7 +163,10 @@ qoq_status qoq_quantize_weights(const void *W_fp16, int64_t N, int64_t K, int gr
  * where a bounded wait (1 s) gave up: the wait site (1 producer waiting for a
  * free stage, 2 MMA waiting for a drained accumulator, 3 MMA waiting for a
  * stage's operands, 4 dequantiser waiting for a stage's copies, 5 epilogue
- * waiting for an accumulator, 6 tile owner waiting for a contributor), the
+ * waiting for an accumulator, 6 tile owner waiting for a contributor, 7 last
+ * arriver of a split tile waiting for the owner's partial sums, 8 waiting
+ * for every token row of the fused quantisation, 9 waiting for a free A/X
+ * stage), the
  * CTA index, and the unit, segment or contributor index. After such an error,
  * zero-fill the control bytes again. Size query: workspace == NULL stores the required size for
  * (M, N, K, group_size) in *workspace_bytes and returns QOQ_OK.
@@ -189,6 +192,35 @@ qoq_status qoq_gemm_fp16_out(const int8_t *X8, const void *s_x_fp16, const int32
                              const void *blob, int64_t M, int64_t N, int64_t K, int group_size,
                              void *Y_fp16, void *workspace, size_t *workspace_bytes,
                              void *stream);
+
+/*
+ * The whole linear layer in one call: per-token quantisation of FP16
+ * activations, then the W4A8 GEMM with the fused FP16 epilogue.
+ * (paperlayer.ai summary, section 5 "QServe Serving System", "Runtime and
+ *  precision mapping": activation quantisation is fused into the kernel that
+ *  produces the GEMM's input, so the FP16 activations are read once.)
+ *
+ *   X8, s_x, rowsum = qoq_quantize_act_per_token(X)   (same arithmetic)
+ *   Y = qoq_gemm_fp16_out(X8, s_x, rowsum, blob)       (same arithmetic)
+ *
+ * When the library picks token tiles of at most 64 tokens for (M, N, K)
+ * (decode batches), both steps run in ONE launch: the GEMM's CTAs quantise
+ * the token rows first (rows are claimed from a counter in the workspace, so
+ * no CTA waits for one that has not started) and stream their first weight
+ * tiles meanwhile. For wider token tiles the call launches the quantiser and
+ * then the GEMM. Either way the codes, scales and row sums are written into
+ * the workspace, after the GEMM's scratch.
+ *
+ * X_fp16 [M][K] FP16, read; Y_fp16 [M][N] FP16, written; blob as for
+ * qoq_gemm_fp16_out. The workspace must be 256-byte aligned, zero-filled by
+ * the caller before its first use, and of the size the query
+ * (workspace == NULL) reports for this (M, N, K, group_size); its control
+ * words and status word behave as for qoq_w4a8_gemm (the claim counters
+ * are control words too, left zero by every call that completes).
+ */
+qoq_status qoq_w4a8_linear(const void *X_fp16, const void *blob, int64_t M, int64_t N, int64_t K,
+                           int group_size, void *Y_fp16, void *workspace, size_t *workspace_bytes,
+                           void *stream);
 
 /*
  * Ablation of the protective range: qoq_gemm_fp16_out with a weight decode
@@ -218,15 +250,16 @@ qoq_status qoq_gemm_fp16_out_saturating(const int8_t *X8, const void *s_x_fp16, 
  * workspace of qoq_gemm_fp16_out need not be allocated by the caller.
  *
  * Same computation and arguments as qoq_gemm_fp16_out, except that the
- * stream-K scratch lives in one fixed 8 MiB device array inside the library,
+ * stream-K scratch lives in one fixed 16 MiB device array inside the library,
  * which every GPU that loads the library keeps until the process exits. That
- * bounds the problem: the call needs 1280 + C * T * 512 bytes, where T is the
- * token tile the library picks for (M, N, K) and C the CTAs of the launch
+ * bounds the problem: the call needs 1280 + C * P * T * 512 bytes, where T is
+ * the token tile the library picks for (M, N, K), C the CTAs of the launch
  * (min(SM count, 256, token tiles * N/128 * K/128); twice the CTA pairs for
- * 256-token tiles). On a 148-SM B200 every problem whose token tile is at
- * most 64 fits: all M <= 64, and M up to 256 where few weight tiles make the
- * library keep 64-token tiles (e.g. N = K = 4096). Larger problems return
- * QOQ_ERR_WORKSPACE and launch nothing.
+ * 256-token tiles) and P the partial-sum slots per CTA (2 for token tiles up
+ * to 64, else 1). On a 148-SM B200 every problem whose token tile is at most
+ * 64 fits (9.7 MB at most): all M <= 64, and M up to 256 where few weight
+ * tiles make the library keep 64-token tiles (e.g. N = K = 4096). Larger
+ * problems return QOQ_ERR_WORKSPACE and launch nothing.
  *
  * status: optional device int32; when non-NULL the call copies the device
  * status word of this call (0, QOQ_ERR_BAD_BLOB or QOQ_ERR_TIMEOUT) into it

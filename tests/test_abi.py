@@ -44,6 +44,16 @@ def test_blob_size_query_matches_layout(L):
         assert qoq.blob_bytes(N, K, g) == oracle.blob_layout(N, K, g)["total"]
 
 
+def test_linear_workspace_size_query(L):
+    """qoq_w4a8_linear's workspace holds the GEMM's scratch and, after it, the
+    quantised activations: codes [M][K], FP16 scales and int32 row sums."""
+    for M, N, K in [(1, 4096, 4096), (64, 28672, 4096), (300, 512, 640), (2048, 4096, 14336)]:
+        gemm = qoq.workspace_bytes(M, N, K)
+        lin = qoq.linear_workspace_bytes(M, N, K)
+        assert lin >= gemm + M * K + 2 * M + 4 * M
+        assert lin <= gemm + M * K + 6 * M + 3 * 256
+
+
 def test_workspace_size_query(L):
     small = qoq.workspace_bytes(1, 4096, 4096)
     big = qoq.workspace_bytes(4096, 4096, 4096)
@@ -85,6 +95,17 @@ def test_argument_validation_without_launch(L):
     assert L.qoq_w4a8_gemm(ctypes.c_void_p(16 * 1024 + 8), None, dummy, 4, 128, 128, 128, dummy, dummy, ws,
                            None) == 3
     assert L.qoq_w4a8_gemm(dummy, None, dummy, 0, 128, 128, 128, dummy, dummy, ws, None) == 0   # M = 0
+    # the whole linear layer (act quant + GEMM)
+    assert L.qoq_w4a8_linear(dummy, dummy, 4, 128, 128, 128, dummy, dummy, None, None) == 1     # no size pointer
+    assert L.qoq_w4a8_linear(dummy, dummy, 4, 128, 100, 128, dummy, dummy, ws, None) == 2      # K % 128
+    assert L.qoq_w4a8_linear(dummy, dummy, 4, 128, 128, 64, dummy, dummy, ws, None) == 1       # group size
+    assert L.qoq_w4a8_linear(dummy, dummy, 4, 128, 128, 128, dummy, dummy, _sz(8), None) == 4  # too small
+    assert L.qoq_w4a8_linear(None, dummy, 4, 128, 128, 128, dummy, dummy, ws, None) == 1       # no X
+    assert L.qoq_w4a8_linear(ctypes.c_void_p(16 * 1024 + 8), dummy, 4, 128, 128, 128, dummy, dummy, ws,
+                             None) == 3                                                        # X misaligned
+    assert L.qoq_w4a8_linear(dummy, dummy, 4, 128, 128, 128, dummy, ctypes.c_void_p(16 * 1024 + 16), ws,
+                             None) == 3                                                        # workspace 256-aligned
+    assert L.qoq_w4a8_linear(None, None, 0, 128, 128, 128, None, dummy, ws, None) == 0         # M = 0
     # fused producers
     f = ctypes.c_float
     assert L.qoq_rmsnorm_quant(dummy, dummy, -1, 4096, f(1e-5), dummy, dummy, None, None) == 1

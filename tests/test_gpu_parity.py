@@ -320,3 +320,129 @@ def test_full_matrix_against_library_int8_gemm(M, N, K):
     assert t.equal(acc, ref), "INT32 sums differ from the library INT8 GEMM of the oracle's operands"
     want = oracle.epilogue_fp16(host(ref), s_xo, d["s_w"])
     assert_fp16_close(host(Y), want, "full FP16 output")
+
+
+# ------------------------------------- the whole linear layer in one call
+
+def _oracle_tile_y(X8s, s_xs, rss, W, nt, group):
+    _, d = oracle.quantize_weights(W[nt * 128:(nt + 1) * 128], group)
+    if group:
+        return oracle.epilogue_fp16(oracle.gemm_int(X8s, d["Wint"]), s_xs, d["s_w"])
+    return oracle.epilogue_fp16(oracle.w4a8_gemm_per_channel(X8s, rss, d["q"], d["z"]), s_xs, d["s"])
+
+
+@pytest.mark.parametrize("group", [128, 0])
+@pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (7, 384, 640), (16, 6144, 4096), (33, 28672, 4096),
+                                   (64, 4096, 14336), (64, 6144, 4096), (100, 512, 640), (256, 4096, 4096),
+                                   (300, 512, 640)])
+def test_linear_matches_oracle(M, N, K, group):
+    """qoq_w4a8_linear (per-token quantisation and GEMM in one call; one
+    launch when the token tile is at most 64 tokens): the FP16 output equals
+    the two-call path (act quant, then qoq_gemm_fp16_out) bit for bit, and the
+    oracle within 1 ulp on every row of sampled n-tiles; the workspace's
+    control words (claim counters included) are left zero."""
+    t = torch()
+    X = inputs.make_activations(M, K, seed=900 + M)
+    W = inputs.make_weights(N, K, seed=900 + N)
+    Xd = dev(X)
+    blob = qoq.quantize_weights(dev(W), group)
+    ws = qoq.Workspace.for_linear(M, N, K, group)
+    Y = qoq.linear(Xd, blob, N, K, group, ws=ws)
+    X8, s_x, rs = qoq.quantize_act_per_token(Xd)
+    Y2 = qoq.gemm_fp16_out(X8, s_x, blob, N, K, group, rowsum=rs)
+    t.cuda.synchronize()
+    assert ws.status() == 0, "status %d %s" % (ws.status(), ws.timeout_site())
+    assert ws.control_clear()
+    assert t.equal(Y.view(t.int16), Y2.view(t.int16)), "one-call and two-call paths differ"
+    X8s, s_xs, rss = oracle.quantize_act_per_token(X)
+    Yh = host(Y)
+    for nt in sample_tiles(N // 128, count=3, seed=M):
+        assert_fp16_close(Yh[:, nt * 128:(nt + 1) * 128], _oracle_tile_y(X8s, s_xs, rss, W, nt, group),
+                          "linear tile %d" % nt)
+
+
+def test_linear_graph_replays_are_bit_identical():
+    """One-launch linear calls of the four Llama-3-8B decode shapes captured in
+    a CUDA graph and replayed back to back (each launch's CTAs start while the
+    previous launch runs): every replay reproduces the eager outputs with a
+    clean status and cleared claim counters."""
+    t = torch()
+    probs = []
+    for i, (K, N, _) in enumerate(inputs.LLAMA3_8B):
+        M = (1, 16, 33, 64)[i]
+        X = inputs.make_activations(M, K, seed=950 + i)
+        W = inputs.make_weights(N, K, seed=950 + i)
+        probs.append(dict(M=M, N=N, K=K, X=X, W=W, Xd=dev(X), blob=qoq.quantize_weights(dev(W), 128),
+                          Y=t.empty((M, N), dtype=t.float16, device="cuda"), ws=qoq.Workspace.for_linear(M, N, K)))
+
+    def step():
+        for p in probs:
+            qoq.linear(p["Xd"], p["blob"], p["N"], p["K"], 128, ws=p["ws"], Y=p["Y"])
+
+    stream = t.cuda.Stream()
+    stream.wait_stream(t.cuda.current_stream())
+    with t.cuda.stream(stream):
+        step()
+    stream.synchronize()
+    ref = [p["Y"].clone() for p in probs]
+    g = t.cuda.CUDAGraph()
+    with t.cuda.graph(g, stream=stream):
+        step()
+    for r in range(30):
+        with t.cuda.stream(stream):
+            g.replay()
+        stream.synchronize()
+        for i, p in enumerate(probs):
+            assert p["ws"].status() == 0, "replay %d case %d: %d %s" % (r, i, p["ws"].status(), p["ws"].timeout_site())
+            assert p["ws"].control_clear(), "replay %d case %d: control words left set" % (r, i)
+            assert t.equal(p["Y"], ref[i]), "replay %d case %d differs" % (r, i)
+    del g
+    for i, p in enumerate(probs):
+        X8s, s_xs, rss = oracle.quantize_act_per_token(p["X"])
+        for nt in sample_tiles(p["N"] // 128, count=2, seed=i)[:2]:
+            assert_fp16_close(host(ref[i])[:, nt * 128:(nt + 1) * 128],
+                              _oracle_tile_y(X8s, s_xs, rss, p["W"], nt, 128), "graph linear %d tile %d" % (i, nt))
+
+
+def test_concurrent_gemms_on_two_streams():
+    """Two stream-K GEMMs running at the same time on two streams, each with
+    its own workspace, 20 launches each, interleaved: no CTA of either waits
+    for one that has not started, so every launch completes with status 0 and
+    the outputs of the serial run."""
+    t = torch()
+    cases = [(16, 28672, 4096), (1, 4096, 14336), (64, 4096, 4096)]
+    probs = []
+    for i, (M, N, K) in enumerate(cases):
+        X = inputs.make_activations(M, K, seed=970 + i)
+        W = inputs.make_weights(N, K, seed=970 + i)
+        blob = qoq.quantize_weights(dev(W), 128)
+        X8, s_x, rs = qoq.quantize_act_per_token(dev(X))
+        probs.append(dict(M=M, N=N, K=K, X=X, W=W, X8=X8, s_x=s_x, rs=rs, blob=blob,
+                          ref=qoq.gemm_fp16_out(X8, s_x, blob, N, K, 128, rowsum=rs)))
+    t.cuda.synchronize()
+    streams = [t.cuda.Stream(), t.cuda.Stream()]
+    outs = {}
+    for si, s in enumerate(streams):
+        s.wait_stream(t.cuda.current_stream())
+    for rep in range(20):
+        for i, p in enumerate(probs):
+            s = streams[(i + rep) % 2]
+            key = (i, (i + rep) % 2)
+            if key not in outs:
+                outs[key] = (qoq.Workspace.for_shape(p["M"], p["N"], p["K"]),
+                             t.empty((p["M"], p["N"]), dtype=t.float16, device="cuda"))
+                s.wait_stream(t.cuda.current_stream())
+            ws, Y = outs[key]
+            with t.cuda.stream(s):
+                qoq.gemm_fp16_out(p["X8"], p["s_x"], p["blob"], p["N"], p["K"], 128, rowsum=p["rs"], ws=ws, Y=Y,
+                                  stream=s)
+    t.cuda.synchronize()
+    for (i, si), (ws, Y) in outs.items():
+        assert ws.status() == 0, "case %d stream %d: status %d %s" % (i, si, ws.status(), ws.timeout_site())
+        assert ws.control_clear()
+        assert t.equal(Y, probs[i]["ref"]), "case %d stream %d differs from the serial run" % (i, si)
+    for i, p in enumerate(probs):
+        X8s, s_xs, rss = oracle.quantize_act_per_token(p["X"])
+        nt = sample_tiles(p["N"] // 128, seed=i)[1]
+        assert_fp16_close(host(p["ref"])[:, nt * 128:(nt + 1) * 128],
+                          _oracle_tile_y(X8s, s_xs, rss, p["W"], nt, 128), "concurrent case %d" % i)

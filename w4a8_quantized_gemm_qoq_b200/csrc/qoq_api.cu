@@ -154,6 +154,62 @@ qoq_status qoq_gemm_fp16_out_saturating(const int8_t *X8, const void *s_x_fp16, 
                        stream, true);
 }
 
+qoq_status qoq_w4a8_linear(const void *X_fp16, const void *blob, int64_t M, int64_t N, int64_t K, int group_size,
+                           void *Y_fp16, void *workspace, size_t *workspace_bytes, void *stream) {
+    if (workspace_bytes == nullptr) return QOQ_ERR_INVALID_ARG;
+    if (M < 0 || M > INT32_MAX) return QOQ_ERR_INVALID_ARG;
+    qoq_status st = check_nk(N, K);
+    if (st != QOQ_OK) return st;
+    if ((st = check_group(group_size)) != QOQ_OK) return st;
+    if (M * N > (int64_t)1 << 40 || M * K > (int64_t)1 << 40) return QOQ_ERR_UNSUPPORTED;
+    const size_t need = linear_workspace_bytes(M, N, K);
+    if (workspace == nullptr) {
+        *workspace_bytes = need;
+        return QOQ_OK;
+    }
+    if (*workspace_bytes < need) return QOQ_ERR_WORKSPACE;
+    if (M == 0) return QOQ_OK;
+    if (X_fp16 == nullptr || blob == nullptr || Y_fp16 == nullptr) return QOQ_ERR_INVALID_ARG;
+    if (!aligned(X_fp16, 16) || !aligned(blob, 16) || !aligned(Y_fp16, 16) || !aligned(workspace, 256))
+        return QOQ_ERR_ALIGNMENT;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    const FusedLayout F = fused_layout(M, K, workspace_bytes_for(M, N, K));
+    GemmArgs a;
+    a.blob = blob;
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.group = group_size;
+    a.out = Y_fp16;
+    a.fp16_out = true;
+    a.ws = workspace;
+    a.ws_capacity = *workspace_bytes;
+    const int tok = token_tile_for(M, N, K);
+    if (tok <= kDecodeMaxTok) {
+        // One launch: the decode kernel quantises the rows itself.
+        a.X = X_fp16;
+        a.X8 = nullptr;
+        a.s_x = nullptr;
+        a.rowsum = nullptr;
+        int dev = 0, sms = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+            return QOQ_ERR_CUDA;
+        return launch_decode_gemm(a, s, tok, sms < kMaxGrid ? sms : kMaxGrid);
+    }
+    // Wider token tiles: the per-token quantiser, then the GEMM, both into
+    // and out of the workspace.
+    int8_t *X8 = reinterpret_cast<int8_t *>(ws + F.off_x8);
+    void *s_x = ws + F.off_sx;
+    int32_t *rowsum = reinterpret_cast<int32_t *>(ws + F.off_rowsum);
+    if (launch_act_quant(X_fp16, M, K, X8, s_x, rowsum, s) != cudaSuccess) return QOQ_ERR_CUDA;
+    a.X8 = X8;
+    a.s_x = s_x;
+    a.rowsum = rowsum;
+    return launch_gemm(a, s);
+}
+
 const char *qoq_status_string(qoq_status status) {
     switch (status) {
         case QOQ_OK: return "QOQ_OK";

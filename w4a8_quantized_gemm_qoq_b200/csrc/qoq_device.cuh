@@ -68,6 +68,9 @@ enum WaitSite : int {
     kSiteDequantFull = 4,     // dequant warp waiting for a stage's copies
     kSiteEpilogueAcc = 5,     // epilogue waiting for an accumulator
     kSiteOwnerFlag = 6,       // tile owner waiting for a contributor's partial sums
+    kSiteLastOwner = 7,       // last arriver of a split tile waiting for the owner's partial sums
+    kSiteRowsDone = 8,        // fused activation quantisation: waiting for every token row
+    kSiteXEmpty = 9,          // token-tile producer / dequantiser waiting for a free A/X stage
 };
 
 // Shared abort flag + global status word used by the bounded waits. The CTA
@@ -435,6 +438,50 @@ __device__ __forceinline__ int32_t ld_relaxed_gpu(const int32_t *p) {
 
 __device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 
+// Atomic add at gpu scope with acquire and release semantics; returns the old value.
+__device__ __forceinline__ int32_t atom_add_acq_rel_gpu(int32_t *p, int32_t v) {
+    int32_t old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
+__device__ __forceinline__ void red_add_release_gpu(int32_t *p, int32_t v) {
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void red_or_release_gpu(int32_t *p, int32_t v) {
+    asm volatile("red.release.gpu.global.or.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ int32_t ld_acquire_gpu(const int32_t *p) {
+    int32_t v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Orders this thread's generic-proxy accesses of global memory with its
+// later async-proxy (TMA) accesses, and the other way round.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Spins until (*p & mask) == want (acquire), bounded like the pipeline waits.
+__device__ __forceinline__ bool wait_word_bounded(const int32_t *p, int32_t mask, int32_t want, const Watchdog &wd,
+                                                  int site, int detail, uint64_t limit_ns = kWaitLimitNs) {
+    if ((ld_acquire_gpu(p) & mask) == want) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if ((ld_acquire_gpu(p) & mask) == want) return true;
+        if ((it & 15u) == 0) {
+            if (wd.aborted()) return false;
+            if (globaltimer_ns() - t0 > limit_ns) {
+                wd.fail(QOQ_ERR_TIMEOUT, site, detail);
+                return false;
+            }
+        }
+    }
+}
+
 // Spins until *flag != 0: relaxed loads back to back (a few lanes poll, so no
 // sleep between them), then one acquire fence, which with the relaxed load
 // that saw the releasing store orders every later access after that store.
@@ -458,6 +505,21 @@ __device__ __forceinline__ bool wait_flag_bounded(const int32_t *flag, const Wat
             }
         }
     }
+}
+
+// ------------------------------------------------------ register reallocation
+
+// Per-warpgroup register budgets: every warp of a warpgroup executes the same
+// one. The CTA's pool is what it was launched with (threads x registers per
+// thread at launch); increases wait for decreases, so the budgets must add up
+// to no more than that pool.
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // -------------------------------------------------------------- misc device

@@ -78,14 +78,41 @@ inline int token_tile_for(int64_t M, int64_t N, int64_t K) {
 static_assert(256 + 4 * kMaxGrid == QOQ_WORKSPACE_CONTROL_BYTES, "workspace control layout");
 
 // Workspace bytes a launch of `grid_ctas` CTAs with token tile `tok` uses:
-// the control words, then one partial tile per CTA.
+// the control words, then the partial-sum slots. The general kernel (token
+// tiles of 128 and 256) keeps one partial tile per CTA; the decode kernel
+// (token tiles up to 64) two, one for the tile it contributes to and one for
+// the tile it owns.
+inline size_t general_scratch_bytes(int tok, int64_t grid_ctas) {
+    return QOQ_WORKSPACE_CONTROL_BYTES + sizeof(int32_t) * (size_t)grid_ctas * tok * kTileN;
+}
+inline size_t decode_scratch_bytes(int tok, int64_t grid_ctas) {
+    return QOQ_WORKSPACE_CONTROL_BYTES + sizeof(int32_t) * (size_t)grid_ctas * 2 * tok * kTileN;
+}
+constexpr int kDecodeMaxTok = 64;
 inline size_t scratch_bytes_for_grid(int tok, int64_t grid_ctas) {
-    return 256 + sizeof(int32_t) * kMaxGrid + sizeof(int32_t) * (size_t)grid_ctas * tok * kTileN;
+    return tok <= kDecodeMaxTok ? decode_scratch_bytes(tok, grid_ctas) : general_scratch_bytes(tok, grid_ctas);
 }
 
 // Workspace size the size query reports: enough for any grid (kMaxGrid CTAs).
 inline size_t workspace_bytes_for(int64_t M, int64_t N, int64_t K) {
     return scratch_bytes_for_grid(token_tile_for(M, N, K), kMaxGrid);
+}
+
+// qoq_w4a8_linear keeps the quantised activations in the workspace, after
+// the GEMM's scratch: codes [M][K], FP16 scales [M], row sums [M].
+struct FusedLayout {
+    size_t off_x8, off_sx, off_rowsum, total;
+};
+inline FusedLayout fused_layout(int64_t M, int64_t K, size_t base) {
+    FusedLayout F;
+    F.off_x8 = (size_t)align256((int64_t)base);
+    F.off_sx = (size_t)align256((int64_t)(F.off_x8 + (size_t)M * K));
+    F.off_rowsum = (size_t)align256((int64_t)(F.off_sx + 2 * (size_t)M));
+    F.total = F.off_rowsum + 4 * (size_t)M;
+    return F;
+}
+inline size_t linear_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+    return fused_layout(M, K, workspace_bytes_for(M, N, K)).total;
 }
 
 // Kernel launchers (return cudaSuccess or the launch error).
@@ -102,6 +129,7 @@ cudaError_t launch_silu_mul_quant(const void *GU, int64_t M, int64_t I, int8_t *
 constexpr int kMaxProducerWidth = 32768;
 
 struct GemmArgs {
+    const void *X = nullptr;   // FP16 activations: quantised in the same launch (decode kernel), else null
     const int8_t *X8;
     const void *s_x;
     const int32_t *rowsum;
@@ -125,5 +153,9 @@ qoq_status launch_gemm(const GemmArgs &a, cudaStream_t stream);
 // actually use (its grid, not the kMaxGrid bound): the same grid rule as
 // launch_gemm. Returns 0 if the device cannot be queried.
 size_t gemm_scratch_bytes(int64_t M, int64_t N, int64_t K, int group, bool saturating = false);
+
+// The decode-regime kernel (token tiles 16, 32, 64; gemm_decode.cu). With
+// a.X set it quantises the activations itself (into the workspace).
+qoq_status launch_decode_gemm(const GemmArgs &a, cudaStream_t stream, int tok, int units_max);
 
 }  // namespace qoq

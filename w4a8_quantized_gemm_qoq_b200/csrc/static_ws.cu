@@ -14,9 +14,10 @@
 
 namespace {
 
-// 8 MiB: the control words plus one partial tile per CTA, for token tiles of
-// up to 64 tokens on a GPU of up to 256 SMs (1280 + 256 * 64 * 512 bytes).
-constexpr size_t kStaticScratchBytes = size_t(8) << 20;
+// 16 MiB: the control words plus two partial tiles per CTA (the decode
+// kernel's slots) for token tiles of up to 64 tokens: 1280 + 148 * 2 * 64 *
+// 512 bytes (9.7 MB) on a 148-SM B200.
+constexpr size_t kStaticScratchBytes = size_t(16) << 20;
 
 static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
 

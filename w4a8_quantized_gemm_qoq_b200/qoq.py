@@ -47,6 +47,8 @@ def lib() -> ctypes.CDLL:
         L.qoq_gemm_fp16_out.argtypes = [vp, vp, vp, vp, i64, i64, i64, i32, vp, vp, sz, vp]
         L.qoq_gemm_fp16_out_saturating.argtypes = [vp, vp, vp, i64, i64, i64, i32, vp, vp, sz, vp]
         L.qoq_gemm_fp16_out_saturating.restype = ctypes.c_int
+        L.qoq_w4a8_linear.argtypes = [vp, vp, i64, i64, i64, i32, vp, vp, sz, vp]
+        L.qoq_w4a8_linear.restype = ctypes.c_int
         L.qoq_watchdog_selftest.argtypes = [vp, i64, vp]
         L.qoq_watchdog_selftest.restype = ctypes.c_int
         L.qoq_status_string.argtypes = [ctypes.c_int]
@@ -95,6 +97,13 @@ def workspace_bytes(M: int, N: int, K: int, group_size: int = GROUP) -> int:
     n = ctypes.c_size_t(0)
     _check("qoq_gemm_fp16_out", lib().qoq_gemm_fp16_out(None, None, None, None, M, N, K, group_size, None, None,
                                                         ctypes.byref(n), None))
+    return n.value
+
+
+def linear_workspace_bytes(M: int, N: int, K: int, group_size: int = GROUP) -> int:
+    n = ctypes.c_size_t(0)
+    _check("qoq_w4a8_linear", lib().qoq_w4a8_linear(None, None, M, N, K, group_size, None, None, ctypes.byref(n),
+                                                    None))
     return n.value
 
 
@@ -173,6 +182,11 @@ class Workspace:
     def for_shape(cls, M, N, K, group_size=GROUP, device="cuda"):
         return cls(workspace_bytes(M, N, K, group_size), device)
 
+    @classmethod
+    def for_linear(cls, M, N, K, group_size=GROUP, device="cuda"):
+        """Workspace of qoq_w4a8_linear (GEMM scratch plus the quantised activations)."""
+        return cls(linear_workspace_bytes(M, N, K, group_size), device)
+
     def status(self) -> int:
         return int(self.buf[:4].view(dtype=__import__("torch").int32).item())
 
@@ -241,7 +255,18 @@ def gemm_fp16_out_saturating(X8, s_x, blob, N, K, ws=None, Y=None, stream=None):
     return Y
 
 
-def linear(X, blob, N, K, group_size=GROUP, ws=None, stream=None):
-    """The whole hot path: per-token quantisation of X then the W4A8 GEMM."""
-    X8, s_x, rowsum = quantize_act_per_token(X, stream=stream)
-    return gemm_fp16_out(X8, s_x, blob, N, K, group_size, rowsum=rowsum, ws=ws, stream=stream)
+def linear(X, blob, N, K, group_size=GROUP, ws=None, Y=None, stream=None):
+    """The whole hot path in one call (qoq_w4a8_linear): per-token
+    quantisation of X [M][K] fp16, then the W4A8 GEMM with the FP16 epilogue;
+    one launch when the token tile is at most 64 tokens. Y [M][N] fp16."""
+    import torch
+    X = _cuda_tensor(X, torch.float16, "X")
+    M = X.shape[0]
+    if X.shape[1] != K:
+        raise ValueError("X must have K = %d columns" % K)
+    ws = ws or Workspace.for_linear(M, N, K, group_size, X.device)
+    Y = torch.empty((M, N), dtype=torch.float16, device=X.device) if Y is None else Y
+    n = ctypes.c_size_t(ws.buf.numel())
+    _check("qoq_w4a8_linear", lib().qoq_w4a8_linear(_ptr(X), _ptr(blob), M, N, K, group_size, _ptr(Y), _ptr(ws.buf),
+                                                    ctypes.byref(n), _stream(stream)))
+    return Y
