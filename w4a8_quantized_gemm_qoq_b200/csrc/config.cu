@@ -1,0 +1,43 @@
+// Launch-configuration overrides for benchmark sweeps: the QOQ_FORCE_CONFIG
+// environment variable, read once per process. It changes only how a problem
+// is tiled and launched, never what is computed, and size queries see the
+// same override as launches.
+//
+//   QOQ_FORCE_CONFIG="tok=64,cps=1"
+//     tok=16|32|64|128|256   token tile (MMA N) for every GEMM
+//     cps=1|2                CTAs per SM of the decode kernel (token tiles <= 64)
+// Unknown keys and values are ignored.
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "qoq_internal.h"
+
+namespace qoq {
+
+const ForcedConfig &forced_config() {
+    static ForcedConfig cfg;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        const char *env = std::getenv("QOQ_FORCE_CONFIG");
+        if (env == nullptr) return;
+        const char *p = env;
+        while (*p) {
+            const char *end = std::strchr(p, ',');
+            const size_t len = end ? (size_t)(end - p) : std::strlen(p);
+            int v = 0;
+            if (len > 4 && std::strncmp(p, "tok=", 4) == 0) {
+                v = std::atoi(p + 4);
+                if (v == 16 || v == 32 || v == 64 || v == 128 || v == 256) cfg.tok = v;
+            } else if (len > 4 && std::strncmp(p, "cps=", 4) == 0) {
+                v = std::atoi(p + 4);
+                if (v == 1 || v == 2) cfg.cps = v;
+            }
+            if (!end) break;
+            p = end + 1;
+        }
+    });
+    return cfg;
+}
+
+}  // namespace qoq

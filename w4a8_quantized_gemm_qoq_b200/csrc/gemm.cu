@@ -844,7 +844,7 @@ static qoq_status launch_gemm_t(const GemmArgs &a, cudaStream_t stream, int unit
     p.grid = (int)std::min<long long>(units_max, blocks);
     // The partial-sum slots are indexed by CTA: the workspace must hold one
     // per CTA of this grid.
-    if (general_scratch_bytes(TOK, PAIR ? 2 * p.grid : p.grid) > a.ws_capacity) return QOQ_ERR_WORKSPACE;
+    if (scratch_bytes_for_grid(TOK, PAIR ? 2 * p.grid : p.grid) > a.ws_capacity) return QOQ_ERR_WORKSPACE;
     // Whole tiles in data-parallel waves while at least one to two waves of
     // tiles remain for the stream-K tail, which evens out the last wave.
     const long long tiles = (long long)p.MT * p.NTw;
@@ -920,8 +920,7 @@ size_t gemm_scratch_bytes(int64_t M, int64_t N, int64_t K, int group, bool satur
     const int64_t NTw = pl.pair ? N / kTileN / 2 : N / kTileN;
     const int64_t blocks = ((M + pl.tok - 1) / pl.tok) * NTw * (K / kTileK);
     const int64_t units = std::min<int64_t>(pl.units_max, blocks);
-    if (pl.tok <= kDecodeMaxTok && !saturating) return decode_scratch_bytes(pl.tok, units);
-    return general_scratch_bytes(pl.tok, pl.pair ? 2 * units : units);
+    return scratch_bytes_for_grid(pl.tok, pl.pair ? 2 * units : units);
 }
 
 template <int MODE>

@@ -65,64 +65,62 @@ constexpr int kWarpEpi = 12;      // warps 12..15: epilogue warpgroup
 constexpr int kBarEpi = 1;        // named barrier of the epilogue warpgroup
 constexpr int kSmemPerSm = 233472;          // 228 KB of shared memory per SM
 constexpr int kSmemReservedPerCta = 1024;   // the system's share of every CTA
-constexpr int kWantCtasPerSm = 2;
-// Registers: 64 per thread at launch (two 512-thread CTAs fill the SM's
-// 65536); the control warpgroup (producers, issuers) gives 24 of its own to
-// each of the three compute warpgroups' 8 more: 128 x 40 + 384 x 72 = 512 x 64.
-constexpr int kRegsLaunch = 64;
+// Two CTAs per SM: 64 registers per thread at launch (two 512-thread CTAs fill
+// the SM's 65536); the control warpgroup (producers, issuers) gives 24 of its
+// own so that the three compute warpgroups get 8 more each:
+// 128 x 40 + 384 x 72 = 512 x 64.
 constexpr int kRegsCtl = 40;
 constexpr int kRegsWork = 72;
-static_assert(128 * kRegsCtl + 384 * kRegsWork <= kThreads * kRegsLaunch, "register split exceeds the launch pool");
+static_assert(128 * kRegsCtl + 384 * kRegsWork <= kThreads * 64, "register split exceeds the launch pool");
 }  // namespace dec
 
-template <int TOK, int MODE>
+constexpr int kSmemPerSmAvail = dec::kSmemPerSm;
+
+// CPS: CTAs per SM the configuration is built for. Two: half an SM each,
+// so the next launch's CTAs sit beside this one's and prefetch and
+// dequantise while it runs. One: the whole SM, for the deepest weight ring
+// (the main loop's HBM rate is the bytes in flight per SM over the loaded
+// memory latency).
+template <int TOK, int MODE, int CPS>
 struct DecCfg {
     static_assert(TOK == 16 || TOK == 32 || TOK == 64, "decode token tiles");
+    static_assert(CPS == 1 || CPS == 2, "one or two CTAs per SM");
     static constexpr int kKB = 2;                              // k-tiles per pipeline unit
     static constexpr int kWTile = MODE == 0 ? 8448 : 8192;     // codes (+ s, z*s) per k-tile
     static constexpr int kWStage = kKB * kWTile;
     static constexpr int kXTile = TOK * 128;                   // token tile of one k-tile
     static constexpr int kXStage = kKB * kXTile;
-    static constexpr int kSW = TOK == 64 ? 3 : 4;              // weight stages
-    static constexpr int kSA = 3;                              // A/X stages
     // Up to 32 tokens the two issuers take alternate units, each into its own
     // accumulator; at 64 they split the token columns of every unit.
     static constexpr bool kAlt = TOK <= 32;
     static constexpr int kAccCols = kAlt ? 2 * TOK : TOK;
-    static constexpr int kAccBufs = TOK == 16 ? 2 : 1;
+    static constexpr int kAccBufs = 2;
     static constexpr int kACol0 = kAccBufs * kAccCols;
-    static constexpr int kTmemCols = 256;
+    static constexpr int kTmemCols = CPS == 1 ? 512 : 256;
+    // A/X stages: as many two-k-tile TMEM A buffers as fit, an even number.
+    // The two dequant warpgroups take alternate units (warpgroup g the units
+    // of parity g), and so do the issuers when they alternate; with an even
+    // stage count unit parity fixes stage parity, so each of them waits on
+    // every phase of its own stages and on no others (a parity wait cannot
+    // tell a phase from the one two later).
+    static constexpr int kSA = ((kTmemCols - kACol0) / (kKB * 32)) & ~1;
+    static_assert(kSA >= 2, "A/X ring too shallow");
     static_assert(kACol0 + kSA * kKB * 32 <= kTmemCols, "TMEM over-subscribed");
-    // "Stage complete" barriers. An issuer that takes every other unit would
-    // skip phases of a per-stage barrier (kSA is odd), and the token tile's
-    // copy completes on it, so phases need not complete in unit order; each
-    // issuer therefore has its own set: unit u completes a_full[(u & 1) *
-    // kSA + u % kSA], phase u / (2 kSA), and every issuer waits on every phase
-    // of its own barriers. Issuers that split the token columns share one set.
-    static constexpr int kAFull = kAlt ? 2 * kSA : kSA;
-    static_assert(kSA % 2 == 1, "the a_full phase formula assumes an odd stage count");
     static constexpr int kXBytes = kSA * kXStage;              // first: 1024-aligned swizzle atoms
-    static constexpr int kWBytes = kSW * kWStage;
-    static constexpr int kCtlBytes = 1024;
+    static constexpr int kCtlBytes = 2048;
     static constexpr int kEpiBytes = 4 * 2 * 1024;             // per epilogue warp two 16 x 32 FP16 blocks
+    static constexpr int kSmemBudget = kSmemPerSmAvail / CPS - dec::kSmemReservedPerCta;
+    // Weight stages: what is left, at most 16, an even number (as above).
+    static constexpr int kSWfit = (kSmemBudget - 1024 - kXBytes - kCtlBytes - kEpiBytes) / kWStage;
+    static constexpr int kSW = (kSWfit > 16 ? 16 : kSWfit) & ~1;
+    static_assert(kSW >= 2, "weight ring too shallow");
+    static constexpr int kWBytes = kSW * kWStage;
     static constexpr int kSmemBytes = 1024 + kXBytes + kWBytes + kCtlBytes + kEpiBytes;
     static_assert(kXStage % 1024 == 0 && kXTile % 1024 == 0, "token tiles must keep the swizzle atom aligned");
     static_assert(kWStage % 16 == 0, "bulk copies move multiples of 16 bytes");
-    static_assert(dec::kWantCtasPerSm * (kSmemBytes + dec::kSmemReservedPerCta) <= dec::kSmemPerSm,
-                  "two CTAs per SM must fit");
+    static_assert(kSmemBytes <= 232448, "227 KB per CTA");
+    static_assert(CPS * (kSmemBytes + dec::kSmemReservedPerCta) <= dec::kSmemPerSm, "CPS CTAs per SM must fit");
 };
-
-// The "stage complete" barrier of unit u and the parity of its phase.
-template <int TOK, int MODE>
-__device__ __forceinline__ uint64_t *a_full_of(uint64_t *a_full, int u, uint32_t &parity) {
-    using C = DecCfg<TOK, MODE>;
-    if (C::kAlt) {
-        parity = (uint32_t)(u / (2 * C::kSA)) & 1u;
-        return a_full + (u & 1) * C::kSA + u % C::kSA;
-    }
-    parity = (uint32_t)(u / C::kSA) & 1u;
-    return a_full + u % C::kSA;
-}
 
 struct DecParams {
     const uint8_t *blob;
@@ -132,7 +130,7 @@ struct DecParams {
     int32_t *status;        // workspace word 0
     int32_t *qctl;          // fused quantisation: [0] next row to claim, [1] rows done, [2] CTAs finished
     int32_t *counters;      // [kMaxGrid]: arrival counter of the split tile owned by CTA c
-    int32_t *partials;      // [grid][2][TOK][128]: slot 0 as contributor, slot 1 as owner
+    int32_t *partials;      // [grid][TOK][128]: INT32 sums of the split tile owned by CTA c (zero between launches)
     const __half *X;        // fused: FP16 activations [M][K]
     int8_t *X8q;            // fused: INT8 codes [M][K] (workspace)
     __half *s_xq;           // fused: FP16 scales [M] (workspace)
@@ -145,8 +143,8 @@ struct DecParams {
 };
 
 struct DecCtl {
-    uint64_t w_full[4], w_empty[4];
-    uint64_t a_full[6], ax_empty[3];
+    uint64_t w_full[16], w_empty[16];
+    uint64_t a_full[8], ax_empty[8];
     uint64_t acc_full[2], acc_empty[2];
     uint64_t final_bar[2];
     uint32_t tmem_base;
@@ -158,7 +156,7 @@ struct DecCtl {
     alignas(16) float tok_scale[64];
     int32_t tok_rowsum[64];
 };
-static_assert(sizeof(DecCtl) <= 1024, "control block outgrows its reserve");
+static_assert(sizeof(DecCtl) <= 2048, "control block outgrows its reserve");
 
 // Quantise one 16-byte chunk (eight FP16 values) of a token row: eight codes
 // packed little-endian into two words; returns their sum. The arithmetic of
@@ -247,11 +245,11 @@ __device__ __forceinline__ bool fused_act_quant(const DecParams &p, DecCtl *ctl,
     return !named_bar_any(dec::kBarEpi, 128, !ok);
 }
 
-template <int TOK, int MODE, bool FUSED>
-__global__ void __launch_bounds__(dec::kThreads, 2)
+template <int TOK, int MODE, bool FUSED, int CPS>
+__global__ void __launch_bounds__(dec::kThreads, CPS)
     qoq_decode_kernel(const __grid_constant__ DecParams p, const __grid_constant__ CUtensorMap tmap_x,
                       const __grid_constant__ CUtensorMap tmap_y) {
-    using C = DecCfg<TOK, MODE>;
+    using C = DecCfg<TOK, MODE, CPS>;
     constexpr int SW = C::kSW, SA = C::kSA, KB = C::kKB;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -268,10 +266,12 @@ __global__ void __launch_bounds__(dec::kThreads, 2)
         ctl->abort_flag = 0;
         for (int s = 0; s < SW; ++s) {
             mbar_init(&ctl->w_full[s], 1);
-            mbar_init(&ctl->w_empty[s], 8);              // the eight dequant warps
+            mbar_init(&ctl->w_empty[s], 4);              // the four warps of the unit's dequant warpgroup
         }
-        for (int s = 0; s < C::kAFull; ++s) mbar_init(&ctl->a_full[s], 9);   // 8 dequant warps + token producer
-        for (int s = 0; s < SA; ++s) mbar_init(&ctl->ax_empty[s], C::kAlt ? 1 : 2);
+        for (int s = 0; s < SA; ++s) {
+            mbar_init(&ctl->a_full[s], 5);               // the dequant warpgroup's 4 warps + the token producer
+            mbar_init(&ctl->ax_empty[s], C::kAlt ? 1 : 2);
+        }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&ctl->acc_full[b], 2);             // both issuers commit every segment
             mbar_init(&ctl->acc_empty[b], 4);            // the four epilogue warps
@@ -318,7 +318,7 @@ __global__ void __launch_bounds__(dec::kThreads, 2)
         // Each warpgroup sets its register budget at the top of its own
         // branch, so the compiler allocates each role's code with that budget.
         if (warp < 4) {
-        regs_dec<dec::kRegsCtl>();
+        if (CPS == 2) regs_dec<dec::kRegsCtl>();
         if (warp == dec::kWarpProdW) {
             // -------------------------------------------- weight producer
             // Runs ahead of everything else, including the previous kernel:
@@ -360,20 +360,15 @@ __global__ void __launch_bounds__(dec::kThreads, 2)
                     const int s = u % SA;
                     if (u >= SA && !wait_bounded(&ctl->ax_empty[s], (uint32_t)((u / SA) - 1) & 1u, wd, kSiteXEmpty, u))
                         break;
-                    uint32_t aph;
-                    uint64_t *af = a_full_of<TOK, MODE>(ctl->a_full, u, aph);
-                    mbar_arrive_expect_tx(af, (uint32_t)(cur.nk * C::kXTile));
+                    mbar_arrive_expect_tx(&ctl->a_full[s], (uint32_t)(cur.nk * C::kXTile));
                     for (int j = 0; j < cur.nk; ++j)
-                        tma_load_2d(xst + s * C::kXStage + j * C::kXTile, &tmap_x, af, (cur.kt + j) * kTileK,
-                                    cur.mt * TOK, pol_x);
+                        tma_load_2d(xst + s * C::kXStage + j * C::kXTile, &tmap_x, &ctl->a_full[s],
+                                    (cur.kt + j) * kTileK, cur.mt * TOK, pol_x);
                 }
                 // The token tiles issued last land before the CTA can exit:
                 // a unit's a_full phase completes only with them.
-                for (int i = u > SA ? u - SA : 0; i < u; ++i) {
-                    uint32_t aph;
-                    uint64_t *af = a_full_of<TOK, MODE>(ctl->a_full, i, aph);
-                    wait_drain(af, aph, kDrainNs);
-                }
+                for (int i = u > SA ? u - SA : 0; i < u; ++i)
+                    wait_drain(&ctl->a_full[i % SA], (uint32_t)(i / SA) & 1u, kDrainNs);
             }
             __syncwarp();
         } else if (warp == dec::kWarpIss || warp == dec::kWarpIss + 1) {
@@ -403,9 +398,7 @@ __global__ void __launch_bounds__(dec::kThreads, 2)
                             const int s = u % SA;
                             // The dequantisers' arrivals and the token tile's
                             // bytes both complete a_full[s].
-                            uint32_t aph;
-                            uint64_t *af = a_full_of<TOK, MODE>(ctl->a_full, u, aph);
-                            ok = wait_bounded(af, aph, wd, kSiteMmaOperands, u);
+                            ok = wait_bounded(&ctl->a_full[s], (uint32_t)(u / SA) & 1u, wd, kSiteMmaOperands, u);
                             if (!ok) break;
                             tc_fence_after();
                             const uint32_t a_tmem = tmem_base + (uint32_t)(C::kACol0 + s * KB * 32);
@@ -431,33 +424,63 @@ __global__ void __launch_bounds__(dec::kThreads, 2)
             __syncwarp();
         }
         } else if (warp >= dec::kWarpDq && warp < dec::kWarpEpi) {
-            regs_inc<dec::kRegsWork>();
+            if (CPS == 2) regs_inc<dec::kRegsWork>();
             // ------------------------------------------------ dequant
-            // Warpgroup g decodes k-tile g of every unit; thread (quarter,
-            // lane) owns weight row r, i.e. one whole quantisation group, so
-            // (s, z*s) is a scalar. Per 32-bit word of eight codes: and,
-            // shift+and, two multiply-adds (q*s <= 240 and q*s + 128 - z*s in
-            // [7, 249] never carry between bytes) and two xors (excess-128 to
-            // int8). Nothing here depends on the previous kernel.
+            // Warpgroup g decodes the units of parity g, both k-tiles of each;
+            // thread (quarter, lane) owns weight row r, i.e. one whole
+            // quantisation group per k-tile, so (s, z*s) is a scalar. Per
+            // 32-bit word of eight codes: and, shift+and, two multiply-adds
+            // (q*s <= 240 and q*s + 128 - z*s in [7, 249] never carry between
+            // bytes) and two xors (excess-128 to int8). A TMEM store and its
+            // completion wait cost hundreds of cycles, so with registers to
+            // spare (one CTA per SM) the first k-tile's store is left in
+            // flight while the second is decoded. Nothing here depends on the
+            // previous kernel.
             const int g = (warp - dec::kWarpDq) >> 2;
             const int quarter = warp & 3;
             const int r = quarter * 32 + lane;
             const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+            auto decode = [&](const uint4 (&v)[4], uint32_t sz, uint32_t (&o)[32]) {
+                const uint32_t sc = sz & 0xFFu;
+                const uint32_t c4 = (uint32_t)(128 - (int)(int8_t)(sz >> 8)) * 0x01010101u;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const uint32_t wd4[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint32_t lo = wd4[q] & 0x0F0F0F0Fu;
+                        const uint32_t hi = (wd4[q] >> 4) & 0x0F0F0F0Fu;
+                        if (MODE == 0) {
+                            o[8 * c + 2 * q] = (lo * sc + c4) ^ 0x80808080u;
+                            o[8 * c + 2 * q + 1] = (hi * sc + c4) ^ 0x80808080u;
+                        } else {
+                            o[8 * c + 2 * q] = lo;
+                            o[8 * c + 2 * q + 1] = hi;
+                        }
+                    }
+                }
+            };
             UnitCursor<KB> cur;
             cur.init(me, G, waves, b0, b1, KT, p.NT, p.MT, p.GM);
             for (int u = 0; !cur.done(); ++u, cur.advance()) {
+                if ((u & 1) != g) continue;
                 const int sw = u % SW, sa = u % SA;
                 bool ok = __all_sync(0xffffffffu,
                                      wait_bounded(&ctl->w_full[sw], (uint32_t)(u / SW) & 1u, wd, kSiteDequantFull, u));
                 if (!ok) break;
-                const bool mine = g < cur.nk;
-                uint4 v[4];
-                uint32_t sz = 0u;
-                if (mine) {
-                    const uint32_t wbase = smem_u32(wst + sw * C::kWStage + g * C::kWTile);
-                    if (MODE == 0) sz = lds16(wbase + 8192 + 2 * r);
+                const int nk = cur.nk;
+                uint4 v0[4], v1[4];
+                uint32_t sz0 = 0u, sz1 = 0u;
+                {
+                    const uint32_t wbase = smem_u32(wst + sw * C::kWStage);
+                    if (MODE == 0) sz0 = lds16(wbase + 8192 + 2 * r);
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) v[c] = lds128(wbase + c * 2048 + r * 16);
+                    for (int c = 0; c < 4; ++c) v0[c] = lds128(wbase + c * 2048 + r * 16);
+                    if (nk == 2) {
+                        if (MODE == 0) sz1 = lds16(wbase + C::kWTile + 8192 + 2 * r);
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) v1[c] = lds128(wbase + C::kWTile + c * 2048 + r * 16);
+                    }
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&ctl->w_empty[sw]);   // the packed weights are in registers
@@ -468,43 +491,38 @@ __global__ void __launch_bounds__(dec::kThreads, 2)
                     if (!ok) break;
                 }
                 tc_fence_after();
-                if (mine) {
-                    const uint32_t sc = sz & 0xFFu;
-                    const uint32_t c4 = (uint32_t)(128 - (int)(int8_t)(sz >> 8)) * 0x01010101u;
-                    uint32_t o[32];
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const uint32_t wd4[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const uint32_t lo = wd4[q] & 0x0F0F0F0Fu;
-                            const uint32_t hi = (wd4[q] >> 4) & 0x0F0F0F0Fu;
-                            if (MODE == 0) {
-                                o[8 * c + 2 * q] = (lo * sc + c4) ^ 0x80808080u;
-                                o[8 * c + 2 * q + 1] = (hi * sc + c4) ^ 0x80808080u;
-                            } else {
-                                o[8 * c + 2 * q] = lo;
-                                o[8 * c + 2 * q + 1] = hi;
-                            }
-                        }
+                const uint32_t a_col = tmem_base + lane_addr + (uint32_t)(C::kACol0 + sa * KB * 32);
+                if (CPS == 1) {
+                    uint32_t o0[32], o1[32];
+                    decode(v0, sz0, o0);
+                    tmem_st32(a_col, o0);
+                    if (nk == 2) {
+                        decode(v1, sz1, o1);
+                        tmem_st32(a_col + 32u, o1);
                     }
-                    tmem_st32_wait(tmem_base + lane_addr + (uint32_t)(C::kACol0 + sa * KB * 32 + g * 32), o);
+                    tmem_st_wait();
+                } else {
+                    uint32_t o[32];
+                    decode(v0, sz0, o);
+                    tmem_st32_wait(a_col, o);
+                    if (nk == 2) {
+                        decode(v1, sz1, o);
+                        tmem_st32_wait(a_col + 32u, o);
+                    }
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) {
-                    uint32_t aph;
-                    mbar_arrive(a_full_of<TOK, MODE>(ctl->a_full, u, aph));
-                }
+                if (lane == 0) mbar_arrive(&ctl->a_full[sa]);
                 __syncwarp();
             }
         } else {
             // ------------------------------------------------ epilogue
-            regs_inc<dec::kRegsWork>();
+            if (CPS == 2) regs_inc<dec::kRegsWork>();
             const int quarter = warp & 3;
             const int r = quarter * 32 + lane;
             const int te = threadIdx.x - dec::kWarpEpi * 32;
             const bool leader = te == 0;
+            const bool announcer = te == 96;   // warp 15, lane 0: the owner's early arrival
             const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
             griddep_wait();   // X, scales, row sums, outputs and workspace belong to the previous kernel until now
             bool ok = true;
@@ -514,6 +532,53 @@ __global__ void __launch_bounds__(dec::kThreads, 2)
             int seg = 0, ubase = 0, obuf = 0;
             __half *stage_base = out_stage + (warp - dec::kWarpEpi) * 2 * (16 * 32);
             constexpr int CO = 16;   // token columns per step
+            // Per-tile epilogue inputs: the weight row's scale (and zero
+            // point) in registers, the tile's token scales (and row sums)
+            // staged in shared memory.
+            float col_scale = 0.0f;
+            int col_zero = 0;
+            auto stage_tile = [&](int mt, int nt) {
+                const int n = nt * kTileN + r;
+                col_scale = p.fp16_out ? __half2float(reinterpret_cast<const __half *>(p.blob + p.off_scale)[n]) : 0.0f;
+                col_zero = MODE == 1 ? __half2int_rn(reinterpret_cast<const __half *>(p.blob + p.off_zero)[n]) : 0;
+                const int64_t m0 = (int64_t)mt * TOK;
+                for (int j = te; j < TOK; j += 128) {
+                    const int64_t m = m0 + j < p.M ? m0 + j : p.M - 1;
+                    // At L2: with the fused quantisation other CTAs wrote them in this launch.
+                    ctl->tok_scale[j] = p.fp16_out ? __half2float(__ldcg(p.s_x + m)) : 0.0f;
+                    if (MODE == 1) ctl->tok_rowsum[j] = __ldcg(p.rowsum + m);
+                }
+            };
+            auto emit = [&](const uint32_t (&v)[CO], int mt, int nt, int c0) {
+                const int64_t m0 = (int64_t)mt * TOK;
+                const int n = nt * kTileN + r;
+                if (p.fp16_out) {
+                    store_outputs_fp16<CO, MODE>(&tmap_y, v, m0 + c0, n - lane, lane, col_scale, col_zero,
+                                                 ctl->tok_scale + c0, ctl->tok_rowsum + c0, stage_base + obuf * 512);
+                    obuf ^= 1;
+                } else {
+                    store_outputs_i32<CO, MODE>(static_cast<int32_t *>(p.out), p.M, p.N, v, m0 + c0, n, col_zero,
+                                                ctl->tok_rowsum + c0);
+                }
+            };
+            // The finisher's read of a split tile's sum buffer (zero at launch
+            // start; every other participant added its partial sums into it
+            // before arriving): live columns only, all loads in flight at
+            // once; the buffer is cleared behind it for the next launch.
+            auto take_sum = [&](uint32_t (&v)[CO], int32_t *tsum, int c0, int m_live) {
+                int32_t t[CO];
+#pragma unroll
+                for (int j = 0; j < CO; ++j) t[j] = (c0 + j < m_live) ? ld_cg_s32(tsum + (c0 + j) * kTileN) : 0;
+#pragma unroll
+                for (int j = 0; j < CO; ++j) {
+                    v[j] += (uint32_t)t[j];   // modulo 2^32: exact where the sum fits
+                    if (c0 + j < m_live) tsum[(c0 + j) * kTileN] = 0;
+                }
+            };
+            // A contributor's arrival, checked at the end: this CTA contributes
+            // to at most one split tile (its first segment).
+            bool pend = false;
+            int pend_old = 0, pend_first = 0, pend_nparts = 0, pend_mt = 0, pend_nt = 0;
             while (ok && !cur.done()) {
                 const uint32_t seg_b = cur.b, seg_e = cur.seg_end;
                 const int kt_lo = cur.kt, kt_hi = cur.kt + (int)(seg_e - seg_b);
@@ -526,7 +591,6 @@ __global__ void __launch_bounds__(dec::kThreads, 2)
                 ubase += nunits;
                 const int buf = seg % C::kAccBufs;
                 const uint32_t aph = (uint32_t)(seg / C::kAccBufs) & 1u;
-                const int n = nt * kTileN + r;
                 const int64_t m0 = (int64_t)mt * TOK;
                 const int m_live = (int)(p.M - m0 < TOK ? p.M - m0 : TOK);
                 const int live_end = (m_live + CO - 1) / CO * CO;
@@ -542,19 +606,11 @@ __global__ void __launch_bounds__(dec::kThreads, 2)
                     cnt = p.counters + first;
                 }
                 const int nparts = (int)(last - first + 1);
-                // The owner announces itself as soon as it starts the tile:
-                // if every contributor is already in, it will finish the tile.
-                if (owner && leader) ctl->fix_old = atom_add_acq_rel_gpu(cnt, 1);
-                const float col_scale =
-                    p.fp16_out ? __half2float(reinterpret_cast<const __half *>(p.blob + p.off_scale)[n]) : 0.0f;
-                const int col_zero =
-                    MODE == 1 ? __half2int_rn(reinterpret_cast<const __half *>(p.blob + p.off_zero)[n]) : 0;
-                for (int j = te; j < TOK; j += 128) {
-                    const int64_t m = m0 + j < p.M ? m0 + j : p.M - 1;
-                    // At L2: with the fused quantisation other CTAs wrote them in this launch.
-                    ctl->tok_scale[j] = p.fp16_out ? __half2float(__ldcg(p.s_x + m)) : 0.0f;
-                    if (MODE == 1) ctl->tok_rowsum[j] = __ldcg(p.rowsum + m);
-                }
+                int32_t *tsum = p.partials + (long long)first * TOK * kTileN + r;
+                stage_tile(mt, nt);
+                // The owner announces itself as soon as it starts the tile: if
+                // every contributor is already in, it finishes the tile.
+                if (owner && announcer) ctl->fix_old = atom_add_acq_rel_gpu(cnt, 1);
                 named_bar_sync(dec::kBarEpi, 128);
                 const bool finisher_owner = owner && (ctl->fix_old & 0xFFFF) == nparts - 1;
                 ok = __all_sync(0xffffffffu, wait_bounded(&ctl->acc_full[buf], aph, wd, kSiteEpilogueAcc, seg));
@@ -565,18 +621,6 @@ __global__ void __launch_bounds__(dec::kThreads, 2)
                 tc_fence_after();
                 const uint32_t acc_addr = tmem_base + lane_addr + (uint32_t)(buf * C::kAccCols + prim * TOK);
                 const uint32_t acc2_addr = tmem_base + lane_addr + (uint32_t)(buf * C::kAccCols + (prim ^ 1) * TOK);
-                // This CTA's partial-sum slot for the tile: 0 as contributor, 1 as owner.
-                int32_t *myslot = p.partials + ((long long)me * 2 + (owner ? 1 : 0)) * TOK * kTileN;
-                auto emit = [&](const uint32_t (&v)[CO], int c0) {
-                    if (p.fp16_out) {
-                        store_outputs_fp16<CO, MODE>(&tmap_y, v, m0 + c0, n - lane, lane, col_scale, col_zero,
-                                                     ctl->tok_scale + c0, ctl->tok_rowsum + c0, stage_base + obuf * 512);
-                        obuf ^= 1;
-                    } else {
-                        store_outputs_i32<CO, MODE>(static_cast<int32_t *>(p.out), p.M, p.N, v, m0 + c0, n, col_zero,
-                                                    ctl->tok_rowsum + c0);
-                    }
-                };
 #pragma unroll 1
                 for (int c0 = 0; c0 < live_end; c0 += CO) {
                     uint32_t v[CO];
@@ -588,69 +632,68 @@ __global__ void __launch_bounds__(dec::kThreads, 2)
                         if (lane == 0) mbar_arrive(&ctl->acc_empty[buf]);
                     }
                     if (sole) {
-                        emit(v, c0);
+                        emit(v, mt, nt, c0);
                     } else if (finisher_owner) {
-                        // Every contributor stored its partial sums before it
-                        // arrived; the owner's acquire saw all arrivals.
-#pragma unroll 1
-                        for (uint32_t c = first + 1; c <= last; ++c) {
-                            const int32_t *part = p.partials + ((long long)c * 2) * TOK * kTileN + c0 * kTileN + r;
-                            int32_t t[CO];
-#pragma unroll
-                            for (int j = 0; j < CO; ++j) t[j] = ld_cg_s32(part + j * kTileN);
-#pragma unroll
-                            for (int j = 0; j < CO; ++j) v[j] += (uint32_t)t[j];   // modulo 2^32: exact where the sum fits
-                        }
-                        emit(v, c0);
+                        take_sum(v, tsum, c0, m_live);
+                        emit(v, mt, nt, c0);
                     } else {
 #pragma unroll
                         for (int j = 0; j < CO; ++j)
-                            if (c0 + j < m_live) myslot[(c0 + j) * kTileN + r] = (int32_t)v[j];
+                            if (c0 + j < m_live) red_add_s32(tsum + (c0 + j) * kTileN, (int32_t)v[j]);
                     }
                 }
                 if (!sole) {
                     if (finisher_owner) {
                         if (leader) *cnt = 0;   // nobody touches the counter again in this launch
-                    } else if (owner) {
-                        // Not last: a contributor is still running and will
-                        // finish the tile; it may need these partial sums.
-                        named_bar_sync(dec::kBarEpi, 128);
-                        if (leader) red_or_release_gpu(cnt, 0x10000);
                     } else {
-                        named_bar_sync(dec::kBarEpi, 128);   // every partial-sum store precedes the arrival
-                        if (leader) ctl->fix_old = atom_add_acq_rel_gpu(cnt, 1);
+                        // Every add of this CTA precedes its arrival. The owner
+                        // is not last: a contributor is still running and will
+                        // finish the tile once these sums are in.
                         named_bar_sync(dec::kBarEpi, 128);
-                        if ((ctl->fix_old & 0xFFFF) == nparts - 1) {
-                            // Last arriver: the owner is in (it arrived), but
-                            // may not have stored its partial sums yet.
-                            bool got = true;
-                            if (leader)
-                                got = wait_word_bounded(cnt, 0x10000, 0x10000, wd, kSiteLastOwner, (int)first);
-                            if (named_bar_any(dec::kBarEpi, 128, !got)) {
-                                ok = false;
-                                break;
-                            }
-#pragma unroll 1
-                            for (int c0 = 0; c0 < live_end; c0 += CO) {
-                                uint32_t v[CO];
-#pragma unroll
-                                for (int j = 0; j < CO; ++j) v[j] = 0u;
-#pragma unroll 1
-                                for (uint32_t c = first; c <= last; ++c) {
-                                    const int32_t *part = p.partials + ((long long)c * 2 + (c == first ? 1 : 0)) *
-                                                                           TOK * kTileN + c0 * kTileN + r;
-#pragma unroll
-                                    for (int j = 0; j < CO; ++j) v[j] += (uint32_t)ld_cg_s32(part + j * kTileN);
-                                }
-                                emit(v, c0);
-                            }
-                            if (leader) *cnt = 0;
+                        if (owner) {
+                            if (leader) red_or_release_gpu(cnt, 0x10000);
+                        } else {
+                            // A contributor: arrive now, read the result later.
+                            if (leader) pend_old = atom_add_acq_rel_gpu(cnt, 1);
+                            pend = true;
+                            pend_first = (int)first;
+                            pend_nparts = nparts;
+                            pend_mt = mt;
+                            pend_nt = nt;
                         }
                     }
                 }
                 // Closing barrier: the staged scales of this tile are no longer read.
                 if (named_bar_any(dec::kBarEpi, 128, false)) break;
                 ++seg;
+            }
+            if (ok && pend) {
+                // Did this CTA arrive last at the tile it contributed to?
+                if (leader) ctl->fix_old = pend_old;
+                named_bar_sync(dec::kBarEpi, 128);
+                if ((ctl->fix_old & 0xFFFF) == pend_nparts - 1) {
+                    // The owner is in (it arrived), but may not have added its
+                    // sums yet.
+                    int32_t *cnt = p.counters + pend_first;
+                    bool got = true;
+                    if (leader) got = wait_word_bounded(cnt, 0x10000, 0x10000, wd, kSiteLastOwner, pend_first);
+                    stage_tile(pend_mt, pend_nt);
+                    if (!named_bar_any(dec::kBarEpi, 128, !got)) {
+                        const int64_t m0 = (int64_t)pend_mt * TOK;
+                        const int m_live = (int)(p.M - m0 < TOK ? p.M - m0 : TOK);
+                        const int live_end = (m_live + CO - 1) / CO * CO;
+                        int32_t *tsum = p.partials + (long long)pend_first * TOK * kTileN + r;
+#pragma unroll 1
+                        for (int c0 = 0; c0 < live_end; c0 += CO) {
+                            uint32_t v[CO];
+#pragma unroll
+                            for (int j = 0; j < CO; ++j) v[j] = 0u;
+                            take_sum(v, tsum, c0, m_live);
+                            emit(v, pend_mt, pend_nt, c0);
+                        }
+                        if (leader) *cnt = 0;
+                    }
+                }
             }
             // The output copies must have finished reading shared memory
             // before the CTA ends (their global writes complete with the grid).
@@ -679,18 +722,18 @@ __global__ void __launch_bounds__(dec::kThreads, 2)
 
 // ---------------------------------------------------------------- host side
 
-template <int TOK, int MODE, bool FUSED>
+template <int TOK, int MODE, bool FUSED, int CPS>
 static qoq_status launch_decode_t(const GemmArgs &a, cudaStream_t stream, int units_max) {
-    using C = DecCfg<TOK, MODE>;
+    using C = DecCfg<TOK, MODE, CPS>;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return QOQ_ERR_CUDA;
     static std::once_flag attr_once[64];
     static cudaError_t attr_err[64];
     std::call_once(attr_once[dev], [&] {
-        attr_err[dev] = cudaFuncSetAttribute(qoq_decode_kernel<TOK, MODE, FUSED>,
+        attr_err[dev] = cudaFuncSetAttribute(qoq_decode_kernel<TOK, MODE, FUSED, CPS>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
         if (attr_err[dev] == cudaSuccess)
-            attr_err[dev] = cudaFuncSetAttribute(qoq_decode_kernel<TOK, MODE, FUSED>,
+            attr_err[dev] = cudaFuncSetAttribute(qoq_decode_kernel<TOK, MODE, FUSED, CPS>,
                                                  cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     });
     if (attr_err[dev] != cudaSuccess) return QOQ_ERR_CUDA;
@@ -717,8 +760,9 @@ static qoq_status launch_decode_t(const GemmArgs &a, cudaStream_t stream, int un
     if (blocks >= (1ll << 31)) return QOQ_ERR_UNSUPPORTED;
     p.total_blocks = (uint32_t)blocks;
     p.grid = (int)std::min<long long>(units_max, blocks);
-    const size_t partial_bytes = decode_scratch_bytes(TOK, p.grid);
-    if (partial_bytes > a.ws_capacity) return QOQ_ERR_WORKSPACE;
+    // The split tiles' sum buffers, one per CTA (the owner's index), must be
+    // zero when the launch starts; every launch that completes leaves them so.
+    if (scratch_bytes_for_grid(TOK, p.grid) > a.ws_capacity) return QOQ_ERR_WORKSPACE;
     const long long tiles = (long long)p.MT * p.NT;
     const long long dp_tiles = tiles >= 2ll * p.grid ? (tiles / p.grid - 1) * p.grid : 0;
     p.dp_tiles = (uint32_t)dp_tiles;
@@ -731,7 +775,7 @@ static qoq_status launch_decode_t(const GemmArgs &a, cudaStream_t stream, int un
     if (FUSED) {
         // Codes, scales and row sums of the fused quantisation live in the
         // workspace after the partial sums.
-        const FusedLayout F = fused_layout(a.M, a.K, decode_scratch_bytes(TOK, kMaxGrid));
+        const FusedLayout F = fused_layout(a.M, a.K, scratch_bytes_for_grid(TOK, kMaxGrid));
         if (F.total > a.ws_capacity) return QOQ_ERR_WORKSPACE;
         p.X = static_cast<const __half *>(a.X);
         p.X8q = reinterpret_cast<int8_t *>(ws + F.off_x8);
@@ -767,32 +811,47 @@ static qoq_status launch_decode_t(const GemmArgs &a, cudaStream_t stream, int un
     }
     cfg.attrs = attr;
     cfg.numAttrs = na;
-    return cudaLaunchKernelEx(&cfg, qoq_decode_kernel<TOK, MODE, FUSED>, p, tmap, tmap_y) == cudaSuccess
+    return cudaLaunchKernelEx(&cfg, qoq_decode_kernel<TOK, MODE, FUSED, CPS>, p, tmap, tmap_y) == cudaSuccess
                ? QOQ_OK
                : QOQ_ERR_CUDA;
 }
 
-template <bool FUSED>
+int decode_ctas_per_sm(int64_t M, int64_t N, int64_t K) {
+    if (forced_config().cps) return forced_config().cps;
+    // Measured on B200 (Llama-3-8B shapes, M = 1..256): one CTA per SM is as
+    // fast or faster everywhere; the deeper weight ring outweighs the overlap
+    // two CTAs per SM give between consecutive launches.
+    (void)M;
+    (void)N;
+    (void)K;
+    return 1;
+}
+
+template <bool FUSED, int CPS>
 static qoq_status launch_decode_tok(const GemmArgs &a, cudaStream_t stream, int tok, int units_max) {
     if (a.group) {
         switch (tok) {
-            case 16: return launch_decode_t<16, 0, FUSED>(a, stream, units_max);
-            case 32: return launch_decode_t<32, 0, FUSED>(a, stream, units_max);
-            case 64: return launch_decode_t<64, 0, FUSED>(a, stream, units_max);
+            case 16: return launch_decode_t<16, 0, FUSED, CPS>(a, stream, units_max);
+            case 32: return launch_decode_t<32, 0, FUSED, CPS>(a, stream, units_max);
+            case 64: return launch_decode_t<64, 0, FUSED, CPS>(a, stream, units_max);
         }
     } else {
         switch (tok) {
-            case 16: return launch_decode_t<16, 1, FUSED>(a, stream, units_max);
-            case 32: return launch_decode_t<32, 1, FUSED>(a, stream, units_max);
-            case 64: return launch_decode_t<64, 1, FUSED>(a, stream, units_max);
+            case 16: return launch_decode_t<16, 1, FUSED, CPS>(a, stream, units_max);
+            case 32: return launch_decode_t<32, 1, FUSED, CPS>(a, stream, units_max);
+            case 64: return launch_decode_t<64, 1, FUSED, CPS>(a, stream, units_max);
         }
     }
     return QOQ_ERR_UNSUPPORTED;
 }
 
 qoq_status launch_decode_gemm(const GemmArgs &a, cudaStream_t stream, int tok, int units_max) {
-    return a.X != nullptr ? launch_decode_tok<true>(a, stream, tok, units_max)
-                          : launch_decode_tok<false>(a, stream, tok, units_max);
+    const int cps = decode_ctas_per_sm(a.M, a.N, a.K);
+    if (a.X != nullptr)
+        return cps == 1 ? launch_decode_tok<true, 1>(a, stream, tok, units_max)
+                        : launch_decode_tok<true, 2>(a, stream, tok, units_max);
+    return cps == 1 ? launch_decode_tok<false, 1>(a, stream, tok, units_max)
+                    : launch_decode_tok<false, 2>(a, stream, tok, units_max);
 }
 
 }  // namespace qoq

@@ -54,6 +54,14 @@ inline BlobLayout blob_layout(int64_t N, int64_t K, int group) {
     return L;
 }
 
+// Overrides of the launch heuristics from the QOQ_FORCE_CONFIG environment
+// variable (config.cu); 0 = not forced.
+struct ForcedConfig {
+    int tok = 0;   // token tile
+    int cps = 0;   // CTAs per SM of the decode kernel
+};
+const ForcedConfig &forced_config();
+
 // Token-tile width (MMA N) for an M x N x K problem. Small M uses the
 // smallest tile that holds all tokens. Beyond that the choice trades weight
 // re-reads and dequantisation (once per token tile) against enough work units
@@ -63,6 +71,7 @@ inline BlobLayout blob_layout(int64_t N, int64_t K, int group) {
 inline int token_tile_for(int64_t M, int64_t N, int64_t K) {
     const int64_t NT = N / kTileN, KT = K / kTileK;
     auto blocks = [&](int64_t tok) { return ((M + tok - 1) / tok) * NT * KT; };
+    if (forced_config().tok) return forced_config().tok;
     if (M <= 16) return 16;
     if (M <= 32) return 32;
     if (M <= 64) return blocks(64) >= 2500 ? 64 : 32;
@@ -78,20 +87,18 @@ inline int token_tile_for(int64_t M, int64_t N, int64_t K) {
 static_assert(256 + 4 * kMaxGrid == QOQ_WORKSPACE_CONTROL_BYTES, "workspace control layout");
 
 // Workspace bytes a launch of `grid_ctas` CTAs with token tile `tok` uses:
-// the control words, then the partial-sum slots. The general kernel (token
-// tiles of 128 and 256) keeps one partial tile per CTA; the decode kernel
-// (token tiles up to 64) two, one for the tile it contributes to and one for
-// the tile it owns.
-inline size_t general_scratch_bytes(int tok, int64_t grid_ctas) {
-    return QOQ_WORKSPACE_CONTROL_BYTES + sizeof(int32_t) * (size_t)grid_ctas * tok * kTileN;
-}
-inline size_t decode_scratch_bytes(int tok, int64_t grid_ctas) {
-    return QOQ_WORKSPACE_CONTROL_BYTES + sizeof(int32_t) * (size_t)grid_ctas * 2 * tok * kTileN;
-}
+// the control words, then one INT32 partial tile per CTA. The general kernel
+// (token tiles of 128 and 256) uses them as scratch; the decode kernel (token
+// tiles up to 64) as the sum buffers of its split tiles, which must be zero
+// when a launch starts and which every launch that completes leaves zero.
 constexpr int kDecodeMaxTok = 64;
 inline size_t scratch_bytes_for_grid(int tok, int64_t grid_ctas) {
-    return tok <= kDecodeMaxTok ? decode_scratch_bytes(tok, grid_ctas) : general_scratch_bytes(tok, grid_ctas);
+    return QOQ_WORKSPACE_CONTROL_BYTES + sizeof(int32_t) * (size_t)grid_ctas * tok * kTileN;
 }
+
+// CTAs per SM of the decode kernel for a problem: one (the whole SM, deepest
+// weight ring) or two (half an SM, so that consecutive launches overlap).
+int decode_ctas_per_sm(int64_t M, int64_t N, int64_t K);
 
 // Workspace size the size query reports: enough for any grid (kMaxGrid CTAs).
 inline size_t workspace_bytes_for(int64_t M, int64_t N, int64_t K) {

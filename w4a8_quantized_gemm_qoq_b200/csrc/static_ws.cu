@@ -14,10 +14,10 @@
 
 namespace {
 
-// 16 MiB: the control words plus two partial tiles per CTA (the decode
-// kernel's slots) for token tiles of up to 64 tokens: 1280 + 148 * 2 * 64 *
-// 512 bytes (9.7 MB) on a 148-SM B200.
-constexpr size_t kStaticScratchBytes = size_t(16) << 20;
+// 8 MiB: the control words plus one INT32 partial tile per CTA for token
+// tiles of up to 64 tokens: 1280 + 148 * 64 * 512 bytes (4.85 MB) on a 148-SM
+// B200.
+constexpr size_t kStaticScratchBytes = size_t(8) << 20;
 
 static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
 
@@ -71,9 +71,10 @@ extern "C" qoq_status qoq_gemm_fp16_out_static_ws(const int8_t *X8, const void *
     qoq_status st = static_scratch_address(dev, &scratch);
     if (st != QOQ_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // The array keeps whatever the previous call left; the control words must
-    // start at zero for every call.
-    if (cudaMemsetAsync(scratch, 0, QOQ_WORKSPACE_CONTROL_BYTES, s) != cudaSuccess) return QOQ_ERR_CUDA;
+    // The array keeps whatever the previous call left (after an error, not
+    // necessarily zeros); the control words and the partial-sum buffers this
+    // call uses must start at zero.
+    if (cudaMemsetAsync(scratch, 0, need, s) != cudaSuccess) return QOQ_ERR_CUDA;
 
     GemmArgs a;
     a.X8 = X8;
