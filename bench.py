@@ -1,18 +1,23 @@
-"""Benchmark of the QoQ W4A8 hot path on B200: per-token activation
-quantisation + W4A8 GEMM with the fused FP16 epilogue.
+"""Benchmark of the QoQ W4A8 hot path on B200: the linear layer (per-token
+activation quantisation + W4A8 GEMM with the fused FP16 epilogue) through the
+library's one-call entry point, qoq_w4a8_linear (one launch for decode
+batches, where the GEMM quantises its own activations; the quantiser and the
+GEMM for prefill batches).
 
-One step = every GEMM of the workload once, each preceded by the per-token
-quantisation of its activations:
-  decode  (default): Llama-3-8B linear shapes (K->N) 4096->6144 (qkv),
+One step = every GEMM of the workload once:
+  llama3_8b (default): Llama-3-8B linear shapes (K->N) 4096->6144 (qkv),
                      4096->4096 (o), 4096->28672 (gate+up), 14336->4096 (down)
-                     x M in {1, 4, 16, 64, 256}: 20 GEMMs, HBM-bound regime
-  prefill:           the same shapes x M in {2048, 8192, 16384}, per-token
-                     scales spanning 1e-3..1e1: INT8-tensor-bound regime
+                     x M in {1, 4, 16, 64, 256} (decode: HBM-bound) and
+                     M in {2048, 8192, 16384} (prefill, per-token scales
+                     spanning 1e-3..1e1: INT8-tensor-bound): 32 GEMMs
+  decode, prefill:   the two halves of it
+  qwen, perchannel:  Qwen1.5-72B shapes; the per-channel variant on
+                     Llama-2-7B shapes
 Weights are packed once (offline step, not timed); every GEMM of a step reads
-its own copy of the packed weights, so the weights a step streams (about
-550 MB for decode) exceed the 126 MB L2 and every launch reads from HBM.
+its own copy of the packed weights, so the weights a step streams exceed the
+126 MB L2 and every launch reads from HBM.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode|prefill]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
     python bench.py --impl reference ...   (the CPU oracle, timed on host cores)
 
 Prints one JSON line. Multi-GPU (torchrun): every rank runs the same step on
@@ -41,22 +46,33 @@ GROUP = 128
 SHAPES = [(K, N) for (K, N, _) in inputs.LLAMA3_8B]
 NAMES = [name for (_, _, name) in inputs.LLAMA3_8B]
 WORKLOADS = {
-    "decode": dict(M=inputs.DECODE_M, span=None, shapes=inputs.LLAMA3_8B, group=GROUP, std=0.02, bound="hbm",
+    "llama3_8b": dict(M=inputs.DECODE_M + inputs.PREFILL_M, span_from=2048, shapes=inputs.LLAMA3_8B, group=GROUP,
+                      std=0.02,
+                      desc="Llama-3-8B linear layers (qkv 4096->6144, o 4096->4096, gate_up 4096->28672, "
+                           "down 14336->4096) x M in {1,4,16,64,256} (decode) and {2048,8192,16384} (prefill, "
+                           "per-token scales 1e-3..1e1), g128, act-quant + W4A8 GEMM + FP16 epilogue"),
+    "decode": dict(M=inputs.DECODE_M, span_from=None, shapes=inputs.LLAMA3_8B, group=GROUP, std=0.02,
                    desc="Llama-3-8B decode GEMMs (qkv 4096->6144, o 4096->4096, gate_up 4096->28672, "
                         "down 14336->4096) x M in {1,4,16,64,256}, g128, act-quant + GEMM"),
-    "prefill": dict(M=inputs.PREFILL_M, span=(-3, 1), shapes=inputs.LLAMA3_8B, group=GROUP, std=0.02,
-                    bound="tensor",
+    "prefill": dict(M=inputs.PREFILL_M, span_from=0, shapes=inputs.LLAMA3_8B, group=GROUP, std=0.02,
                     desc="Llama-3-8B prefill GEMMs (same four shapes) x M in {2048,8192,16384}, g128, "
                          "per-token scales 1e-3..1e1, act-quant + GEMM"),
-    "qwen": dict(M=inputs.QWEN_M, span=None, shapes=inputs.QWEN15_72B, group=GROUP, std=0.01, bound="mixed",
+    "qwen": dict(M=inputs.QWEN_M, span_from=None, shapes=inputs.QWEN15_72B, group=GROUP, std=0.01,
                  desc="Qwen1.5-72B GEMMs (qkv 8192->24576, o 8192->8192, gate_up 8192->49152, "
                       "down 24576->8192) x M in {1,16,128,512,4096}, g128, act-quant + GEMM"),
-    "perchannel": dict(M=inputs.PER_CHANNEL_M, span=None, shapes=inputs.LLAMA2_7B, group=0, std=0.02,
-                       bound="mixed",
+    "perchannel": dict(M=inputs.PER_CHANNEL_M, span_from=None, shapes=inputs.LLAMA2_7B, group=0, std=0.02,
                        desc="per-channel variant (no group level) on Llama-2-7B GEMMs (qkv 4096->12288, "
                             "o 4096->4096, gate_up 4096->22016, down 11008->4096) x M in 1..1024 (powers of 2), "
                             "act-quant + GEMM"),
 }
+# Regimes the roofline is graded in: HBM-bound decode batches, INT8-tensor-bound prefill batches.
+DECODE_HBM_MAX_M = 64
+PREFILL_TENSOR_MIN_M = 2048
+
+
+def token_span(wl, M):
+    """Per-token scale span of the workload's M (prefill batches: 1e-3..1e1)."""
+    return (-3, 1) if wl["span_from"] is not None and M >= wl["span_from"] else None
 
 
 def gemm_bytes(M, N, K, group=GROUP):
@@ -87,12 +103,12 @@ def load_peaks():
         return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
 
 
-def measured_traffic(workload):
-    """DRAM bytes per GEMM launch (dram__bytes_read.sum + dram__bytes_write.sum)
-    from the committed ncu summary of this workload, or None when there is
-    none or the GEMM sources have changed since it was taken."""
+def measured_traffic(name, sources):
+    """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum)
+    from the committed ncu summary profiles/<name>.md, or None when there is
+    none or the kernel's sources have changed since it was taken."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", "qoq_gemm_%s_llama3_8b_dram.md" % workload)
+    path = os.path.join(ROOT, "profiles", name + ".md")
     if not os.path.exists(path):
         return None
     vals = {}
@@ -102,8 +118,8 @@ def measured_traffic(workload):
                 k, v = line.split(":", 1)
                 vals[k] = v.strip()
     h = hashlib.sha256()
-    for name in ("gemm.cu", "qoq_device.cuh"):
-        with open(os.path.join(ROOT, "w4a8_quantized_gemm_qoq_b200", "csrc", name), "rb") as f:
+    for src in sources:
+        with open(os.path.join(ROOT, "w4a8_quantized_gemm_qoq_b200", "csrc", src), "rb") as f:
             h.update(f.read())
     if vals.get("kernel_sources_sha256") != h.hexdigest() or "traffic_per_launch_bytes" not in vals:
         return None
@@ -201,33 +217,38 @@ def sum_over_ranks(x: float, device=None) -> float:
 # ------------------------------------------------------------- GPU arm
 
 class Problem:
-    def __init__(self, K, N, M, blob, X, span, device, group=GROUP, name=""):
+    """One linear layer of the step: FP16 X [M][K], its own packed-weight copy,
+    FP16 Y [M][N] and the workspace of the one-call path; plus the buffers of
+    the two-call path (X8, s_x, row sums, GEMM workspace) for the GEMM-only
+    roofline timing."""
+
+    def __init__(self, K, N, M, blob, X, device, group=GROUP, name=""):
         import torch
         from w4a8_quantized_gemm_qoq_b200 import qoq
         self.K, self.N, self.M = K, N, M
         self.group, self.name = group, name
         self.blob = blob
         self.X = X
+        self.tok, self.launches = qoq.plan(M, N, K)
+        self.Y = torch.empty((M, N), dtype=torch.float16, device=device)
+        self.ws_lin = qoq.Workspace.for_linear(M, N, K, group, device)
         self.X8 = torch.empty((M, K), dtype=torch.int8, device=device)
         self.s_x = torch.empty((M,), dtype=torch.float16, device=device)
         self.rowsum = torch.empty((M,), dtype=torch.int32, device=device)
-        self.Y = torch.empty((M, N), dtype=torch.float16, device=device)
         self.ws = qoq.Workspace.for_shape(M, N, K, group, device)
 
-    def run(self, qoq, ev=None):
-        if ev is not None:
-            ev[0].record()
-        qoq.quantize_act_per_token(self.X, self.X8, self.s_x, self.rowsum)
-        if ev is not None:
-            ev[1].record()
-        qoq.gemm_fp16_out(self.X8, self.s_x, self.blob, self.N, self.K, self.group, rowsum=self.rowsum,
-                          ws=self.ws, Y=self.Y)
-        if ev is not None:
-            ev[2].record()
+    def run(self, qoq, stream=None):
+        qoq.linear(self.X, self.blob, self.N, self.K, self.group, ws=self.ws_lin, Y=self.Y, stream=stream)
 
-    def run_gemm(self, qoq):
+    def quantize(self, qoq, stream=None):
+        qoq.quantize_act_per_token(self.X, self.X8, self.s_x, self.rowsum, stream=stream)
+
+    def run_gemm(self, qoq, stream=None):
         qoq.gemm_fp16_out(self.X8, self.s_x, self.blob, self.N, self.K, self.group, rowsum=self.rowsum,
-                          ws=self.ws, Y=self.Y)
+                          ws=self.ws, Y=self.Y, stream=stream)
+
+    def status(self):
+        return self.ws_lin.status() or self.ws.status()
 
 
 def build_problems(workload, device, seed):
@@ -242,10 +263,32 @@ def build_problems(workload, device, seed):
         for mi, M in enumerate(wl["M"]):
             blob = blob0 if mi == 0 else blob0.clone()        # one copy per GEMM: no L2 reuse in a step
             X = torch.from_numpy(inputs.make_activations(M, K, seed=seed + 100 * si + mi,
-                                                         token_scale_span=wl["span"])).to(device)
-            probs.append(Problem(K, N, M, blob, X, wl["span"], device, wl["group"], name))
+                                                         token_scale_span=token_span(wl, M))).to(device)
+            probs.append(Problem(K, N, M, blob, X, device, wl["group"], name))
     torch.cuda.synchronize()
     return probs
+
+
+def graph_time_us(fn, stream, reps):
+    """Capture fn() in a CUDA graph, replay it 3 times untimed, then `reps`
+    times between CUDA events on `stream`; returns microseconds per replay."""
+    import torch
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g.replay()
+    stream.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+    stream.synchronize()
+    del g
+    return 1000.0 * e0.elapsed_time(e1) / reps
 
 
 def run_gpu(args, rank, world, local_rank):
@@ -258,41 +301,30 @@ def run_gpu(args, rank, world, local_rank):
     wl = WORKLOADS[args.workload]
     probs = build_problems(args.workload, device, seed=rank * 1000)
     stream = torch.cuda.Stream(device)
+    stream.wait_stream(torch.cuda.current_stream())   # inputs and zeroed workspaces were made on the default stream
     nP = len(probs)
 
-    # One CUDA graph per step shape: a plain one, and EV_GRAPHS copies that
-    # also record per-launch events (external event nodes) for the last steps
-    # of the timed region.
-    EV_GRAPHS = 4
+    def check(where):
+        bad = [(p.K, p.N, p.M, p.status(), p.ws_lin.timeout_site()) for p in probs if p.status() != 0]
+        assert not bad, "device status %s (K, N, M, code, (site, block, detail)): %s" % (where, bad)
+
     with torch.cuda.stream(stream):
-        for p in probs:                      # eager warm-up: library load, attributes, first launch
+        for p in probs:                      # eager pass: library load, attributes, first launch
             p.run(qoq)
     stream.synchronize()
-    bad = [(p.K, p.N, p.M, p.ws.status(), p.ws.timeout_site()) for p in probs if p.ws.status() != 0]
-    assert not bad, "device status after the eager pass (K, N, M, code, (site, block, detail)): %s" % bad
-    ev = [[[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for _ in range(nP)]
-          for _ in range(EV_GRAPHS)]
-    plain = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(plain, stream=stream):
+    check("after the eager pass")
+    step = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(step, stream=stream):
         for p in probs:
             p.run(qoq)
-    ev_graphs = []
-    for g in range(EV_GRAPHS):
-        cg = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(cg, stream=stream):
-            for p, e in zip(probs, ev[g]):
-                p.run(qoq, e)
-        ev_graphs.append(cg)
-
     with torch.cuda.stream(stream):
         for _ in range(max(3, args.warmup)):
-            plain.replay()
+            step.replay()
     stream.synchronize()
-    bad = [(p.K, p.N, p.M, p.ws.status(), p.ws.timeout_site()) for p in probs if p.ws.status() != 0]
-    assert not bad, "device status (K, N, M, code, (site, block, detail)): %s" % bad
+    check("after warm-up")
 
+    # ---- the timed region: K replays of the step, nothing else.
     K = args.steps
-    n_ev = min(EV_GRAPHS, K)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
@@ -306,122 +338,150 @@ def run_gpu(args, rank, world, local_rank):
     with ClockSampler(uuid) as clk:
         with torch.cuda.stream(stream):
             t0.record()
-            for k in range(K):
-                j = k - (K - n_ev)
-                (ev_graphs[j] if j >= 0 else plain).replay()
+            for _ in range(K):
+                step.replay()
             t1.record()
         stream.synchronize()
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     step_ms = max_over_ranks(t0.elapsed_time(t1) / K, device) if world > 1 else t0.elapsed_time(t1) / K
-    gemm_ms = [sum(ev[g][i][1].elapsed_time(ev[g][i][2]) for g in range(n_ev)) / n_ev for i in range(nP)]
-    act_ms = [sum(ev[g][i][0].elapsed_time(ev[g][i][1]) for g in range(n_ev)) / n_ev for i in range(nP)]
-    bad = [(p.K, p.N, p.M, p.ws.status(), p.ws.timeout_site()) for p in probs if p.ws.status() != 0]
-    assert not bad, "device status (K, N, M, code, (site, block, detail)): %s" % bad
+    check("after the timed steps")
+    del step
 
-    # The dominant kernel alone: the step's GEMMs (inputs already quantised by
-    # the step) replayed back to back in one graph, CUDA events around the
-    # replays only; every GEMM still reads its own weight copy, so the graph
-    # streams more than L2 holds. Its per-launch average is the roofline's
-    # launch duration (per-launch events inside the step break the overlap of
-    # consecutive kernels and overstate each launch).
-    gg = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(gg, stream=stream):
-        for p in probs:
-            p.run_gemm(qoq)
-    with torch.cuda.stream(stream):
-        for _ in range(3):
-            gg.replay()
-    stream.synchronize()
-    KG = max(K, 10)
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    g0 = torch.cuda.Event(enable_timing=True)
-    g1 = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        g0.record()
-        for _ in range(KG):
-            gg.replay()
-        g1.record()
-    stream.synchronize()
-    gemm_only_ms = g0.elapsed_time(g1) / KG
-    if world > 1:
-        gemm_only_ms = max_over_ranks(gemm_only_ms, device)
-    bad = [(p.K, p.N, p.M, p.ws.status(), p.ws.timeout_site()) for p in probs if p.ws.status() != 0]
-    assert not bad, "device status (K, N, M, code, (site, block, detail)): %s" % bad
-    gemm_only_us = 1000.0 * gemm_only_ms
-
+    analysis = analyse(args, probs, qoq, stream, peaks, wl, world, device)
     ops_step = sum(gemm_ops(p.M, p.N, p.K) for p in probs)
-    per = []
-    tot_bytes = tot_gemm_us = 0.0
-    for i, p in enumerate(probs):
-        us = 1000.0 * gemm_ms[i]
-        b = gemm_bytes(p.M, p.N, p.K, p.group)
-        r_us, bound = roof_us(p.M, p.N, p.K, peaks, p.group)
-        aq_us = 1000.0 * act_ms[i]
-        per.append({"shape": p.name, "K": p.K, "N": p.N, "M": p.M,
-                    "gemm_us_in_step": round(us, 3), "act_quant_us_in_step": round(aq_us, 3),
-                    "act_quant_GBps_in_step": round((3.0 * p.M * p.K + 6 * p.M) / aq_us / 1e3, 1),
-                    "TOPS": round(gemm_ops(p.M, p.N, p.K) / us / 1e6, 2), "GBps": round(b / us / 1e3, 1),
-                    "roof_us": round(r_us, 3), "bound": bound, "frac_of_roofline": round(r_us / us, 3)})
-        tot_bytes += b
-        tot_gemm_us += us
-    timing = {"launch_us": round(gemm_only_us / nP, 3), "launches": nP, "replays": KG,
-              "how": "graph of the step's %d GEMM launches replayed back to back; CUDA events around the "
-                     "replays on the launching stream" % nP}
-    if wl["bound"] == "hbm":
-        achieved = tot_bytes / gemm_only_us / 1e3
-        roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm"], "unit": "GB/s",
-                    "frac": round(achieved / peaks["hbm"], 4), "traffic": measured_traffic("decode"),
-                    "algorithmic_bytes_per_launch": round(tot_bytes / nP),
-                    "peak_source": peaks["src"], "kernel": "qoq_gemm_kernel",
-                    "frac_of_time_roofline": round(sum(x["roof_us"] for x in per) / gemm_only_us, 4),
-                    "timing": timing}
-    elif wl["bound"] == "tensor":
-        achieved = ops_step / gemm_only_us / 1e6
-        pk = 2.0 * peaks["bf16"]
-        roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": pk, "unit": "TOPS",
-                    "frac": round(achieved / pk, 4), "traffic": None, "peak_source": peaks["src"] +
-                    " (INT8 = 2 x measured bf16 burst, nominal ratio)", "kernel": "qoq_gemm_kernel",
-                    "frac_of_time_roofline": round(sum(x["roof_us"] for x in per) / gemm_only_us, 4),
-                    "timing": timing}
-    else:
-        # Shapes on both sides of the crossover: the fraction is roofline time
-        # (each GEMM's slower bound) over measured time, summed over the step.
-        roof = sum(x["roof_us"] for x in per)
-        roofline = {"bound": "mixed", "achieved": round(roof / gemm_only_us, 4), "peak": 1.0,
-                    "unit": "fraction of each GEMM's roofline time", "frac": round(roof / gemm_only_us, 4),
-                    "traffic": None, "peak_source": peaks["src"], "kernel": "qoq_gemm_kernel",
-                    "frac_of_time_roofline": round(roof / gemm_only_us, 4), "timing": timing}
-
-    e2e = run_e2e(args, probs, qoq, stream) if rank == 0 else None
-    w8a8 = run_w8a8(probs, stream, gemm_only_us, max(K, 10)) if rank == 0 else None
-    producers = run_producers(stream, peaks) if rank == 0 and not args.no_context else None
-    saturation = run_saturation(stream) if rank == 0 and args.saturation else None
     res = {
         "metric": METRIC, "value": round(world * ops_step / (step_ms * 1e-3) / 1e12, 3), "unit": "TOPS",
         "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup),
         "ms_per_step": round(step_ms, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "int8", "data": "synthetic",
-        "config": {"workload": wl["desc"], "M": wl["M"], "shapes_K_N": [(K, N) for (K, N, _) in wl["shapes"]],
-                   "group_size": wl["group"],
-                   "l2": "inputs larger than L2: each GEMM of a step reads its own packed-weight copy "
-                         "(%.0f MB per step)" % (sum(0.5 * p.N * p.K + (p.N * p.K / 64 if p.group else 4 * p.N)
-                                                     for p in probs) / 1e6),
-                   "launch": "CUDA graph replay of the step; per-launch events from the last %d steps" % n_ev,
-                   "parallelism": "replicas (one independent step per GPU)" if world > 1 else "single GPU"},
-        "roofline": roofline,
-        "gpu_launches": 2 * nP * args.steps,
+        "gpu_launches": sum(p.launches for p in probs) * args.steps,
         "clocks": clk.summary(),
-        "e2e": e2e,
-        "per_gemm": per,
-        "w8a8_context": w8a8,
-        "producers_context": producers,
-        "saturation_context": saturation,
     }
+    res["config"] = {
+        "workload": wl["desc"], "M": wl["M"], "shapes_K_N": [(K_, N_) for (K_, N_, _) in wl["shapes"]],
+        "group_size": wl["group"],
+        "l2": "inputs larger than L2: each GEMM of a step reads its own packed-weight copy (%.0f MB per step)"
+              % (sum(0.5 * p.N * p.K + (p.N * p.K / 64 if p.group else 4 * p.N) for p in probs) / 1e6),
+        "launch": "CUDA graph replay of the step (qoq_w4a8_linear per GEMM: %d launches per step)"
+                  % sum(p.launches for p in probs),
+        "parallelism": "replicas (one independent step per GPU)" if world > 1 else "single GPU"}
+    res.update(analysis)
+    res["e2e"] = run_e2e(args, probs, qoq, stream) if rank == 0 else None
+    res["w8a8_context"] = run_w8a8(probs, stream, res["gemm_us_per_step"], max(K, 10)) if rank == 0 else None
+    res["producers_context"] = run_producers(stream, peaks) if rank == 0 and not args.no_context else None
+    res["saturation_context"] = run_saturation(stream) if rank == 0 and args.saturation else None
     return res
+
+
+def linear_bytes(p):
+    """Algorithmic HBM bytes of one qoq_w4a8_linear call: the GEMM's (packed
+    weights, scales, X8, s_x, Y) with the FP16 activations read in place of
+    X8 (2 M K instead of M K)."""
+    return gemm_bytes(p.M, p.N, p.K, p.group) + p.M * p.K
+
+
+def analyse(args, probs, qoq, stream, peaks, wl, world, device):
+    """Everything measured after the timed steps: per-launch durations inside
+    the step (external event nodes between the calls: they break the overlap
+    of consecutive launches, so they overstate each one), and the roofline of
+    each regime from graphs of that regime's launches alone, back to back,
+    with CUDA events around the replays only."""
+    import torch
+    reps = max(args.steps, 10)
+    nP = len(probs)
+    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)] for _ in probs]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for p, e in zip(probs, ev):
+            e[0].record()
+            p.run(qoq)
+            e[1].record()
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g.replay()
+    stream.synchronize()
+    in_step = [1000.0 * e[0].elapsed_time(e[1]) for e in ev]
+    del g
+
+    out = {}
+    regimes = {}
+    # Decode batches (HBM-bound): the one-call launches (GEMM quantising its
+    # own activations) back to back.
+    dec = [p for p in probs if p.M <= DECODE_HBM_MAX_M]
+    if dec:
+        us = graph_time_us(lambda: [p.run(qoq) for p in dec], stream, reps)
+        b = sum(linear_bytes(p) for p in dec)
+        ach = b / us / 1e3
+        regimes["decode"] = {
+            "bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm"], "unit": "GB/s",
+            "frac": round(ach / peaks["hbm"], 4),
+            "traffic": measured_traffic("qoq_decode_linear_llama3_8b_dram", ("gemm_decode.cu", "gemm_common.cuh",
+                                                                            "qoq_device.cuh", "quant_math.cuh")),
+            "algorithmic_bytes_per_launch": round(b / len(dec)), "peak_source": peaks["src"] + " (HBM copy)",
+            "kernel": "qoq_decode_kernel (one launch per linear call: per-token quantisation + GEMM)",
+            "frac_of_time_roofline": round(sum(roof_us(p.M, p.N, p.K, peaks, p.group)[0] for p in dec) / us, 4),
+            "timing": {"launch_us": round(us / len(dec), 3), "launches": len(dec), "replays": reps,
+                       "M": sorted({p.M for p in dec}),
+                       "how": "graph of the step's M <= %d linear calls replayed back to back; CUDA events around "
+                              "the replays on the launching stream" % DECODE_HBM_MAX_M}}
+    # Every GEMM alone on pre-quantised activations (the two-call path).
+    with torch.cuda.stream(stream):
+        for p in probs:
+            p.quantize(qoq)
+    stream.synchronize()
+    out["gemm_us_per_step"] = round(graph_time_us(lambda: [p.run_gemm(qoq) for p in probs], stream, reps), 2)
+    pre = [p for p in probs if p.M >= PREFILL_TENSOR_MIN_M]
+    if pre:
+        us = graph_time_us(lambda: [p.run_gemm(qoq) for p in pre], stream, reps)
+        ops = sum(gemm_ops(p.M, p.N, p.K) for p in pre)
+        ach = ops / us / 1e6
+        pk = 2.0 * peaks["bf16"]
+        regimes["prefill"] = {
+            "bound": "tensor", "achieved": round(ach, 1), "peak": pk, "unit": "TOPS", "frac": round(ach / pk, 4),
+            "traffic": measured_traffic("qoq_gemm_prefill_llama3_8b_dram", ("gemm.cu", "gemm_common.cuh",
+                                                                           "qoq_device.cuh")),
+            "algorithmic_ops_per_launch": round(ops / len(pre)),
+            "peak_source": peaks["src"] + " (INT8 = 2 x measured bf16 burst, the nominal 4.5/2.25 ratio)",
+            "kernel": "qoq_gemm_kernel (256-token tiles on CTA pairs)",
+            "frac_of_time_roofline": round(sum(roof_us(p.M, p.N, p.K, peaks, p.group)[0] for p in pre) / us, 4),
+            "timing": {"launch_us": round(us / len(pre), 3), "launches": len(pre), "replays": reps,
+                       "M": sorted({p.M for p in pre}),
+                       "how": "graph of the step's M >= %d GEMM launches (activations quantised beforehand) "
+                              "replayed back to back; CUDA events around the replays" % PREFILL_TENSOR_MIN_M}}
+    # The dominant kernel: the regime with the larger share of the step.
+    share = {k: sum(t for p, t in zip(probs, in_step) if (p.M <= DECODE_HBM_MAX_M if k == "decode"
+                                                             else p.M >= PREFILL_TENSOR_MIN_M))
+             for k in regimes}
+    if regimes:
+        dom = max(share, key=share.get)
+        out["roofline"] = dict(regimes[dom], regime=dom)
+        for k, v in regimes.items():
+            if k != dom:
+                out["roofline_" + k] = dict(v, regime=k)
+    else:
+        roof = sum(roof_us(p.M, p.N, p.K, peaks, p.group)[0] for p in probs)
+        us = graph_time_us(lambda: [p.run(qoq) for p in probs], stream, reps)
+        out["roofline"] = {"bound": "mixed", "achieved": round(roof / us, 4), "peak": 1.0,
+                           "unit": "fraction of each GEMM's roofline time", "frac": round(roof / us, 4),
+                           "traffic": None, "peak_source": peaks["src"], "kernel": "qoq_w4a8_linear"}
+    per, by_m = [], {}
+    for p, us in zip(probs, in_step):
+        r_us, bound = roof_us(p.M, p.N, p.K, peaks, p.group)
+        per.append({"shape": p.name, "K": p.K, "N": p.N, "M": p.M, "token_tile": p.tok, "launches": p.launches,
+                    "us_in_step": round(us, 3), "TOPS": round(gemm_ops(p.M, p.N, p.K) / us / 1e6, 2),
+                    "GBps": round(linear_bytes(p) / us / 1e3, 1), "roof_us": round(r_us, 3), "bound": bound,
+                    "frac_of_roofline": round(r_us / us, 3)})
+        d = by_m.setdefault(p.M, {"M": p.M, "us_in_step": 0.0, "roof_us": 0.0, "ops": 0.0})
+        d["us_in_step"] += us
+        d["roof_us"] += r_us
+        d["ops"] += gemm_ops(p.M, p.N, p.K)
+    out["per_gemm"] = per
+    out["by_M"] = [{"M": d["M"], "us_in_step": round(d["us_in_step"], 2), "TOPS": round(d["ops"] / d["us_in_step"]
+                                                                                       / 1e6, 2),
+                    "frac_of_roofline": round(d["roof_us"] / d["us_in_step"], 3)} for d in by_m.values()]
+    return out
 
 
 def run_shape(args):
@@ -641,20 +701,19 @@ def run_w8a8(probs, stream, w4a8_us, reps):
 
 def run_e2e(args, probs, qoq, stream):
     """Same metric through the public API with host buffers: every step copies
-    each problem's FP16 activations host->device (pinned), runs the two calls,
-    and reads the FP16 output back device->host."""
+    each problem's FP16 activations host->device (pinned), makes the one
+    linear call (qoq_w4a8_linear), and reads the FP16 output back
+    device->host, all eager on one stream."""
     import torch
     hx = [p.X.cpu().pin_memory() for p in probs]
     hy = [torch.empty(p.Y.shape, dtype=torch.float16).pin_memory() for p in probs]
-    dx = [torch.empty_like(p.X) for p in probs]
     h2d = sum(x.numel() * 2 for x in hx)
     d2h = sum(y.numel() * 2 for y in hy)
 
     def once():
-        for p, a, b, c in zip(probs, hx, dx, hy):
-            b.copy_(a, non_blocking=True)
-            X8, s_x, rs = qoq.quantize_act_per_token(b, p.X8, p.s_x, p.rowsum)
-            qoq.gemm_fp16_out(X8, s_x, p.blob, p.N, p.K, p.group, rowsum=rs, ws=p.ws, Y=p.Y)
+        for p, a, c in zip(probs, hx, hy):
+            p.X.copy_(a, non_blocking=True)
+            p.run(qoq)
             c.copy_(p.Y, non_blocking=True)
 
     steps = max(1, args.steps)
@@ -680,36 +739,40 @@ def run_e2e(args, probs, qoq, stream):
 # ------------------------------------------------------------- CPU oracle
 
 def oracle_sample(workload, seed=0):
-    """A bounded sample of the workload for the CPU oracle: the o-projection
-    GEMM (K=N=4096) at M=16 (decode-sized workloads) or M=64 (prefill), weights
-    quantised beforehand (offline), act-quant + int64 GEMM + FP16 epilogue
-    timed; the per-channel workload uses the per-channel scheme."""
+    """A bounded sample of the workload for the CPU oracle: every shape of the
+    workload, its first 1024 weight rows (8 of the n-tiles) and all of K, at
+    the workload's M values up to 256 (larger M: a 64-row slab, whose rate
+    stands for the rest); weights quantised beforehand (the offline step),
+    then per GEMM the oracle's act quant + int64 GEMM (OpenMP over the output
+    elements) + FP16 epilogue, timed. Returns (run, ops per run, description)."""
     import oracle
-    K, N = 4096, 4096
-    M = 64 if workload == "prefill" else 16
     wl = WORKLOADS[workload]
-    W = inputs.make_weights(N, K, seed=seed, std=wl["std"])
-    X = inputs.make_activations(M, K, seed=seed, token_scale_span=wl["span"])
-    if wl["group"]:
-        d = oracle.quantize_weights_group(W)
+    rows = 1024
+    jobs = []
+    for si, (K, N, name) in enumerate(wl["shapes"]):
+        W = inputs.make_weights(rows, K, seed=seed + si, std=wl["std"])
+        d = oracle.quantize_weights_group(W) if wl["group"] else oracle.quantize_weights_per_channel(W)
+        for M in sorted({min(M, 256) if M <= 256 else 64 for M in wl["M"]}):
+            X = inputs.make_activations(M, K, seed=seed + si, token_scale_span=token_span(wl, M))
+            jobs.append((X, d))
 
-        def once():
+    def once():
+        for X, d in jobs:
             X8, s_x, rowsum = oracle.quantize_act_per_token(X)
-            acc = oracle.gemm_int(X8, d["Wint"])
-            oracle.epilogue_fp16(acc, s_x, d["s_w"])
-    else:
-        d = oracle.quantize_weights_per_channel(W)
-
-        def once():
-            X8, s_x, rowsum = oracle.quantize_act_per_token(X)
-            t = oracle.w4a8_gemm_per_channel(X8, rowsum, d["q"], d["z"])
-            oracle.epilogue_fp16(t, s_x, d["s"])
-    desc = "o-proj GEMM K=N=4096, M=%d: act quant + int64 triple-loop GEMM + FP16 epilogue " \
-           "(weights pre-quantised%s)" % (M, "" if wl["group"] else ", per-channel variant")
-    return once, gemm_ops(M, N, K), desc
+            if wl["group"]:
+                oracle.epilogue_fp16(oracle.gemm_int(X8, d["Wint"]), s_x, d["s_w"])
+            else:
+                oracle.epilogue_fp16(oracle.w4a8_gemm_per_channel(X8, rowsum, d["q"], d["z"]), s_x, d["s"])
+    ops = sum(gemm_ops(X.shape[0], rows, X.shape[1]) for X, _ in jobs)
+    Ms = sorted({X.shape[0] for X, _ in jobs})
+    desc = ("every shape of the workload, first %d weight rows, full K, M in %s (M > 256 as a 64-row slab): act "
+            "quant + int64 GEMM (OpenMP, %d threads) + FP16 epilogue; weights pre-quantised"
+            % (rows, Ms, oracle.gemm_threads()))
+    return once, ops, desc
 
 
 def time_oracle(workload, budget_s=10.0, min_runs=1):
+    import oracle
     once, ops, desc = oracle_sample(workload)
     once()   # compile/load the C part outside the timing
     n, t0 = 0, time.perf_counter()
@@ -719,22 +782,20 @@ def time_oracle(workload, budget_s=10.0, min_runs=1):
         el = time.perf_counter() - t0
         if n >= min_runs and el >= budget_s:
             break
-    return {"value": round(ops * n / el / 1e12, 6), "unit": "TOPS", "cores": 1, "kind": "oracle",
-            "sample": "%s; %d runs in %.1f s" % (desc, n, el)}
+    return {"value": round(ops * n / el / 1e12, 6), "unit": "TOPS", "cores": oracle.gemm_threads(),
+            "kind": "oracle", "sample": "%s; %d runs in %.1f s" % (desc, n, el)}
 
 
 def run_reference(args):
     """--impl reference: the CPU oracle, as it stands, on the host cores."""
-    cb_steps = []
+    import oracle
     once, ops, desc = oracle_sample(args.workload)
     once()
     for _ in range(max(0, args.warmup)):
         once()
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        s = time.perf_counter()
         once()
-        cb_steps.append(time.perf_counter() - s)
     el = time.perf_counter() - t0
     val = ops * args.steps / el / 1e12
     return {"impl": "reference", "metric": METRIC, "value": round(val, 6), "unit": "TOPS", "n_gpus": 1,
@@ -742,18 +803,18 @@ def run_reference(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64",
             "data": "synthetic",
             "config": {"workload": WORKLOADS[args.workload]["desc"], "sample": desc},
-            "cpu_baseline": {"value": round(val, 6), "unit": "TOPS", "cores": 1, "kind": "oracle",
-                             "sample": "%s; one sample GEMM per step" % desc},
+            "cpu_baseline": {"value": round(val, 6), "unit": "TOPS", "cores": oracle.gemm_threads(),
+                             "kind": "oracle", "sample": "%s; one sample per step" % desc},
             "e2e": {"value": round(val, 6), "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="llama3_8b")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--saturation", action="store_true",

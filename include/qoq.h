@@ -296,6 +296,16 @@ qoq_status qoq_gemm_fp16_out_static_ws(const int8_t *X8, const void *s_x_fp16, c
  */
 qoq_status qoq_watchdog_selftest(int32_t *status, int64_t limit_ns, void *stream);
 
+/*
+ * Launch plan of a problem (no device work; the library has no counterpart
+ * in the QServe pages): the token tile (MMA N: 16, 32, 64, 128 or 256) the
+ * GEMM calls use for (M, N, K), and how many kernels qoq_w4a8_linear
+ * launches for it (1 when the token tile is at most 64, else 2). Either
+ * output pointer may be NULL. Returns QOQ_ERR_INVALID_ARG / _UNSUPPORTED for
+ * shapes the GEMM calls reject.
+ */
+qoq_status qoq_plan(int64_t M, int64_t N, int64_t K, int32_t *token_tile, int32_t *linear_launches);
+
 /* Name of a status code (static string, never NULL). */
 const char *qoq_status_string(qoq_status status);
 

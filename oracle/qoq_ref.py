@@ -334,12 +334,13 @@ _lock = threading.Lock()
 
 
 def build_c_oracle(force: bool = False) -> str:
-    """Compile qoq_gemm.c with gcc (plain -O2, no fast-math) into oracle/_build/."""
+    """Compile qoq_gemm.c with gcc (plain -O2, no fast-math, OpenMP over output
+    elements) into oracle/_build/."""
     src = os.path.join(_HERE, "qoq_gemm.c")
     if force or not os.path.exists(_SO) or os.path.getmtime(_SO) < os.path.getmtime(src):
         os.makedirs(os.path.dirname(_SO), exist_ok=True)
         tmp = _SO + ".%d.tmp" % os.getpid()
-        subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-ffp-contract=off",
+        subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-ffp-contract=off", "-fopenmp",
                                "-o", tmp, src])
         os.replace(tmp, _SO)
     return _SO
@@ -352,8 +353,14 @@ def _c():
             lib = ctypes.CDLL(build_c_oracle())
             lib.oracle_gemm_s8s8_i64.restype = ctypes.c_int64
             lib.oracle_gemm_s8s8_i64.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int64] * 3
+            lib.oracle_threads.restype = ctypes.c_int
             _lib = lib
     return _lib
+
+
+def gemm_threads() -> int:
+    """Host threads the integer GEMM runs on."""
+    return int(_c().oracle_threads())
 
 
 def gemm_int(X8: np.ndarray, Wint: np.ndarray) -> np.ndarray:

@@ -54,6 +54,17 @@ def test_linear_workspace_size_query(L):
         assert lin <= gemm + M * K + 6 * M + 3 * 256
 
 
+def test_plan_query(L):
+    """Token tiles and launch counts of the one-call linear path: two launches
+    (quantiser, then GEMM) unless the token tile is at most 64 and the fused
+    launch is selected, and always two for prefill batches."""
+    tok, nl = qoq.plan(1, 4096, 4096)
+    assert tok == 16 and nl in (1, 2)
+    assert qoq.plan(64, 28672, 4096)[0] == 64
+    assert qoq.plan(2048, 28672, 4096) == (256, 2)
+    assert L.qoq_plan(4, 100, 128, None, None) == 2
+
+
 def test_workspace_size_query(L):
     small = qoq.workspace_bytes(1, 4096, 4096)
     big = qoq.workspace_bytes(4096, 4096, 4096)

@@ -446,3 +446,20 @@ def test_concurrent_gemms_on_two_streams():
         nt = sample_tiles(p["N"] // 128, seed=i)[1]
         assert_fp16_close(host(p["ref"])[:, nt * 128:(nt + 1) * 128],
                           _oracle_tile_y(X8s, s_xs, rss, p["W"], nt, 128), "concurrent case %d" % i)
+
+
+@pytest.mark.parametrize("fuse", [0, 1])
+def test_linear_both_launch_configurations(fuse):
+    """The one-call linear path with the activation quantisation in its own
+    launch (fuse=0) and inside the decode GEMM's launch (fuse=1), each in a
+    fresh process (the configuration is read once per process): bit for bit
+    the two-call path, within 1 ulp of the oracle, and stable over graph
+    replays."""
+    import os
+    import subprocess
+    import sys
+    here = os.path.dirname(os.path.abspath(__file__))
+    env = dict(os.environ, QOQ_FORCE_CONFIG="fuse=%d" % fuse)
+    r = subprocess.run([sys.executable, os.path.join(here, "linear_check.py"), str(2 - fuse)], env=env,
+                       capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0 and "linear_check ok" in r.stdout, r.stdout[-2000:] + r.stderr[-4000:]

@@ -6,6 +6,9 @@
 //   QOQ_FORCE_CONFIG="tok=64,cps=1"
 //     tok=16|32|64|128|256   token tile (MMA N) for every GEMM
 //     cps=1|2                CTAs per SM of the decode kernel (token tiles <= 64)
+//     fuse=0|1               qoq_w4a8_linear: quantise the activations inside
+//                            the decode GEMM's launch (1) or with the separate
+//                            quantiser first (0)
 // Unknown keys and values are ignored.
 #include <cstdlib>
 #include <cstring>
@@ -32,6 +35,9 @@ const ForcedConfig &forced_config() {
             } else if (len > 4 && std::strncmp(p, "cps=", 4) == 0) {
                 v = std::atoi(p + 4);
                 if (v == 1 || v == 2) cfg.cps = v;
+            } else if (len > 5 && std::strncmp(p, "fuse=", 5) == 0) {
+                v = std::atoi(p + 5);
+                if (v == 0 || v == 1) cfg.fuse = v + 1;
             }
             if (!end) break;
             p = end + 1;

@@ -17,11 +17,7 @@
 // token tile (MMA N = 16..64) staged by TMA in shared memory; exact INT32
 // sums; the same FP32 epilogue. What differs is the shape of the launch,
 // built for decode, where each launch streams 8-60 MB of weights in a few
-// microseconds and per-launch fixed costs decide the throughput:
-//   * half an SM per CTA (256 TMEM columns, <= 110 KB shared memory, 64
-//     registers x 512 threads), so that with programmatic dependent launch the
-//     next GEMM's CTAs sit next to this one's and issue their weight copies
-//     and dequantise their first stages while this launch is still running;
+// microseconds and per-launch fixed costs weigh as much as the stream:
 //   * two rings: packed weights (filled by one producer warp, released by the
 //     dequantisers as soon as they have read them) and A/X stages (a TMEM A
 //     buffer plus the token tile, released by the MMA). Weights never depend
@@ -30,23 +26,32 @@
 //     wait for the previous kernel. The token tile's TMA completes on the
 //     same barrier the dequantisers arrive on, so the MMA issuer waits once
 //     per unit;
-//   * both dequant warpgroups work on every unit (warpgroup g decodes k-tile
-//     g of the two-k-tile unit), so each waits on every phase of every stage
-//     barrier and odd stage counts are safe;
+//   * the two dequant warpgroups take alternate two-k-tile units (warpgroup g
+//     the units of parity g, as do the two MMA issuers when they alternate);
+//     ring sizes are even, so each waits on every phase of its own stages
+//     only. A TMEM store and its completion wait cost hundreds of cycles, so
+//     the first k-tile's store stays in flight while the second is decoded;
+//   * one CTA per SM by default (deepest rings); a two-CTA-per-SM
+//     configuration (half the shared memory, 256 TMEM columns, per-warpgroup
+//     register budgets) lets consecutive launches overlap and is selectable
+//     for sweeps (QOQ_FORCE_CONFIG=cps=2);
 //   * stream-K fix-up by the last arriver: the CTAs sharing a tile count
-//     their arrivals on a per-tile counter; contributors store their INT32
-//     partial sums before arriving, the owner (the CTA with the tile's first
-//     k-tile, which reaches it last) arrives as soon as it starts the tile's
-//     epilogue; whoever arrives last adds the others' partial sums and writes
-//     the output. No CTA waits for one that may not have started, so the
-//     launch needs no co-residency (a last contributor that finds the owner
-//     already arrived waits only for that running owner's partial sums);
-//   * fused activation quantisation (the qoq_w4a8_linear call): the
-//     epilogue warps, idle until the first accumulator is ready, claim token
-//     rows one at a time from a grid-wide counter and quantise them (the same
-//     arithmetic as qoq_quantize_act_per_token) into the workspace; the token
-//     tiles are loaded once every row is done. Rows are claimed, not
-//     assigned, so the first CTAs to start do all of them.
+//     their arrivals on a per-tile counter and add their INT32 partial sums
+//     into the tile's sum buffer (red.add) before arriving; the owner (the CTA
+//     with the tile's first k-tile, which reaches it last) arrives when it
+//     starts the tile's epilogue, and whoever arrives last reads the buffer
+//     once, writes the output and leaves buffer and counter zero for the next
+//     launch. No CTA waits for one that may not have started, so the launch
+//     needs no co-residency (a last contributor that finds the owner already
+//     arrived waits only for that running owner's sums). A contributor reads
+//     its arrival's result only at the end of its schedule;
+//   * optional fused activation quantisation (qoq_w4a8_linear with
+//     QOQ_FORCE_CONFIG=fuse=1): the epilogue warps, idle until the first
+//     accumulator is ready, claim token rows one at a time from a grid-wide
+//     counter and quantise them (the arithmetic of
+//     qoq_quantize_act_per_token) into the workspace; the token tiles are
+//     loaded once every row is done. Rows are claimed, not assigned, so the
+//     first CTAs to start do all of them.
 #include <algorithm>
 #include <cstring>
 
@@ -825,6 +830,19 @@ int decode_ctas_per_sm(int64_t M, int64_t N, int64_t K) {
     (void)N;
     (void)K;
     return 1;
+}
+
+bool linear_fused(int64_t M, int64_t N, int64_t K) {
+    if (forced_config().fuse) return forced_config().fuse == 2;
+    // Measured on B200 (Llama-3-8B decode step, M <= 256): the fused launch's
+    // grid-wide claim -> quantise -> publish -> poll chain adds about four L2
+    // round trips after griddepcontrol.wait, more than the separate
+    // quantiser's launch costs (0.555 vs 0.468 ms per step), so the linear
+    // call uses two launches unless QOQ_FORCE_CONFIG asks for fuse=1.
+    (void)M;
+    (void)N;
+    (void)K;
+    return false;
 }
 
 template <bool FUSED, int CPS>

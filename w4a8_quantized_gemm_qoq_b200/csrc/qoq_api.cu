@@ -186,7 +186,7 @@ qoq_status qoq_w4a8_linear(const void *X_fp16, const void *blob, int64_t M, int6
     a.ws = workspace;
     a.ws_capacity = *workspace_bytes;
     const int tok = token_tile_for(M, N, K);
-    if (tok <= kDecodeMaxTok) {
+    if (tok <= kDecodeMaxTok && linear_fused(M, N, K)) {
         // One launch: the decode kernel quantises the rows itself.
         a.X = X_fp16;
         a.X8 = nullptr;
@@ -198,8 +198,8 @@ qoq_status qoq_w4a8_linear(const void *X_fp16, const void *blob, int64_t M, int6
             return QOQ_ERR_CUDA;
         return launch_decode_gemm(a, s, tok, sms < kMaxGrid ? sms : kMaxGrid);
     }
-    // Wider token tiles: the per-token quantiser, then the GEMM, both into
-    // and out of the workspace.
+    // Otherwise the per-token quantiser, then the GEMM, both into and out of
+    // the workspace.
     int8_t *X8 = reinterpret_cast<int8_t *>(ws + F.off_x8);
     void *s_x = ws + F.off_sx;
     int32_t *rowsum = reinterpret_cast<int32_t *>(ws + F.off_rowsum);
@@ -208,6 +208,16 @@ qoq_status qoq_w4a8_linear(const void *X_fp16, const void *blob, int64_t M, int6
     a.s_x = s_x;
     a.rowsum = rowsum;
     return launch_gemm(a, s);
+}
+
+qoq_status qoq_plan(int64_t M, int64_t N, int64_t K, int32_t *token_tile, int32_t *linear_launches) {
+    if (M < 0 || M > INT32_MAX) return QOQ_ERR_INVALID_ARG;
+    qoq_status st = check_nk(N, K);
+    if (st != QOQ_OK) return st;
+    const int tok = token_tile_for(M, N, K);
+    if (token_tile) *token_tile = tok;
+    if (linear_launches) *linear_launches = (tok <= kDecodeMaxTok && linear_fused(M, N, K)) ? 1 : 2;
+    return QOQ_OK;
 }
 
 const char *qoq_status_string(qoq_status status) {

@@ -59,7 +59,12 @@ inline BlobLayout blob_layout(int64_t N, int64_t K, int group) {
 struct ForcedConfig {
     int tok = 0;   // token tile
     int cps = 0;   // CTAs per SM of the decode kernel
+    int fuse = 0;  // qoq_w4a8_linear at token tiles <= 64: 1 = separate quantiser, 2 = fused launch
 };
+
+// Whether qoq_w4a8_linear quantises the activations inside the decode GEMM's
+// launch for a problem whose token tile is at most 64.
+bool linear_fused(int64_t M, int64_t N, int64_t K);
 const ForcedConfig &forced_config();
 
 // Token-tile width (MMA N) for an M x N x K problem. Small M uses the

@@ -49,6 +49,8 @@ def lib() -> ctypes.CDLL:
         L.qoq_gemm_fp16_out_saturating.restype = ctypes.c_int
         L.qoq_w4a8_linear.argtypes = [vp, vp, i64, i64, i64, i32, vp, vp, sz, vp]
         L.qoq_w4a8_linear.restype = ctypes.c_int
+        L.qoq_plan.argtypes = [i64, i64, i64, vp, vp]
+        L.qoq_plan.restype = ctypes.c_int
         L.qoq_watchdog_selftest.argtypes = [vp, i64, vp]
         L.qoq_watchdog_selftest.restype = ctypes.c_int
         L.qoq_status_string.argtypes = [ctypes.c_int]
@@ -105,6 +107,13 @@ def linear_workspace_bytes(M: int, N: int, K: int, group_size: int = GROUP) -> i
     _check("qoq_w4a8_linear", lib().qoq_w4a8_linear(None, None, M, N, K, group_size, None, None, ctypes.byref(n),
                                                     None))
     return n.value
+
+
+def plan(M: int, N: int, K: int):
+    """(token tile, kernels qoq_w4a8_linear launches) for an M x N x K problem."""
+    tok, nl = ctypes.c_int32(0), ctypes.c_int32(0)
+    _check("qoq_plan", lib().qoq_plan(M, N, K, ctypes.byref(tok), ctypes.byref(nl)))
+    return tok.value, nl.value
 
 
 # ------------------------------------------------------------------ calls
