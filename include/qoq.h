@@ -297,6 +297,70 @@ qoq_status qoq_gemm_fp16_out_static_ws(const int8_t *X8, const void *s_x_fp16, c
 qoq_status qoq_watchdog_selftest(int32_t *status, int64_t limit_ns, void *stream);
 
 /*
+ * KV4 cache: per-head, dynamic, asymmetric 4-bit keys and values.
+ * (paperlayer.ai summary, section 5 "QServe Serving System", "KV4 attention":
+ *  per-head dynamic KV4 scales and zero points, attention arithmetic on CUDA
+ *  cores; section 6 "Evaluation", "Experimental setup": per-head asymmetric
+ *  INT4 KV caches.)
+ *
+ * Every vector of D values (one sequence, one KV head, one token) gets its own
+ * FP16 scale s and zero z, computed when the token is written (nothing is
+ * calibrated), with the per-channel weight quantiser's arithmetic:
+ *   lo = min(0, min x), hi = max(0, max x), s = FP16((hi - lo) / 15),
+ *   z = RNE(-lo / s) (an integer 0..15, stored exactly in FP16),
+ *   q = clamp(RNE(x / s) + z, 0, 15); s == 0 gives q = z = 0.
+ * Each FP32 step is one correctly rounded operation.
+ *
+ * Cache layout (caller-owned device memory, max_tokens slots per sequence):
+ *   codes  uint8 [B][Hkv][max_tokens][D/2], byte j = q[2j] | q[2j+1] << 4
+ *   scales FP16  [B][Hkv][max_tokens]
+ *   zeros  FP16  [B][Hkv][max_tokens]
+ *
+ * qoq_kv4_cache_write quantises src FP16 [B][Hkv][n_tokens][D] (row-major,
+ * 16-byte aligned) into slots t0 .. t0 + n_tokens - 1 of every (sequence, KV
+ * head): the whole cache at once (t0 = 0) or the decode step's new token
+ * (n_tokens = 1). D must be 64 or 128, t0 + n_tokens <= max_tokens, codes
+ * 16-byte aligned, scales and zeros 2-byte aligned (else QOQ_ERR_UNSUPPORTED /
+ * QOQ_ERR_INVALID_ARG / QOQ_ERR_ALIGNMENT before any launch). n_tokens == 0
+ * or B == 0 is a no-op.
+ */
+qoq_status qoq_kv4_cache_write(const void *src_fp16, int64_t B, int64_t Hkv, int64_t max_tokens, int64_t t0,
+                               int64_t n_tokens, int64_t D, uint8_t *codes, void *scales_fp16,
+                               void *zeros_fp16, void *stream);
+
+/*
+ * KV4 decode attention: one query token per sequence against its KV4 cache,
+ * grouped-query (query head hq reads KV head hq / (Hq / Hkv)).
+ * (paperlayer.ai summary, section 5, "KV4 attention"; section 6, "Ablation
+ *  and breakdown": the attention kernel at batch 64 x 1024 tokens.)
+ *
+ *   k_t, v_t = (q_t - z_t) * s_t            (dequantised key / value, t < T_b)
+ *   score_t = (q . k_t) / sqrt(D);  p = softmax_t(score);  out = sum_t p_t v_t
+ *
+ * computed in FP32 on CUDA cores and rounded once to FP16; the order of the
+ * sums is the kernel's (tokens in chunks of 256, chunks combined with the
+ * usual running-maximum rescaling), so results are compared with the exact
+ * mathematics under a tolerance, not bit for bit.
+ *
+ * q_fp16 [B][Hq][D] FP16; the K and V caches as written by
+ * qoq_kv4_cache_write (same B, Hkv, max_tokens, D); seq_lens int32 [B] with
+ * 1 <= T_b <= max_tokens, or NULL for T_b = max_tokens; out_fp16 [B][Hq][D]
+ * FP16, written. Hq must be a multiple of Hkv with Hq / Hkv <= 8, D 64 or 128.
+ *
+ * Workspace: device memory of *workspace_bytes bytes (size query with
+ * workspace == NULL), zero-filled by the caller before its first use; its
+ * leading 4 * B * Hkv bytes are per-(sequence, head) counters that every
+ * call which completes leaves zero, the rest is scratch for the chunks'
+ * partial results. Calls that may overlap on the device need separate
+ * workspaces. A seq_lens entry outside [1, max_tokens] is clamped into it.
+ */
+qoq_status qoq_kv4_decode_attention(const void *q_fp16, const uint8_t *k_codes, const void *k_scales,
+                                    const void *k_zeros, const uint8_t *v_codes, const void *v_scales,
+                                    const void *v_zeros, const int32_t *seq_lens, int64_t B, int64_t Hq,
+                                    int64_t Hkv, int64_t max_tokens, int64_t D, void *out_fp16, void *workspace,
+                                    size_t *workspace_bytes, void *stream);
+
+/*
  * Launch plan of a problem (no device work; the library has no counterpart
  * in the QServe pages): the token tile (MMA N: 16, 32, 64, 128 or 256) the
  * GEMM calls use for (M, N, K), and how many kernels qoq_w4a8_linear

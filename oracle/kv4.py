@@ -1,7 +1,8 @@
 """Plain CPU reference of KV4 decode attention -- TEST INFRASTRUCTURE.
 
-Only tests may use this module (no kernel implements it yet). Like the rest
-of ``oracle/``, it shares no code with the CUDA library.
+Only tests, the smoke check and the benchmark's CPU-baseline arm may use this
+module. Like the rest of ``oracle/``, it shares no code with the CUDA library
+(whose kernels implement the same definitions in kv4_attention.cu).
 
 Sources (web summaries of QServe: W4A8KV4 Quantization and System Co-design
 for Efficient LLM Serving, arXiv 2405.04532):
@@ -49,6 +50,14 @@ def quantize_kv4(X: np.ndarray):
     lead, D = X.shape[:-1], X.shape[-1]
     d = quantize_weights_per_channel(X.reshape(-1, D))
     return dict(q=d["q"].reshape(*lead, D), s=d["s"].reshape(lead), z=d["z"].reshape(lead))
+
+
+def pack_kv4(q: np.ndarray) -> np.ndarray:
+    """Codes [..., D] (0..15) -> the cache's bytes [..., D/2]: byte j holds
+    q[2j] in its low nibble and q[2j+1] in its high nibble (this repository's
+    layout; the pages fix only the 4-bit width)."""
+    q = np.asarray(q, dtype=np.uint8)
+    return (q[..., 0::2] | (q[..., 1::2] << 4)).astype(np.uint8)
 
 
 def dequantize_kv4(q: np.ndarray, s: np.ndarray, z: np.ndarray) -> np.ndarray:

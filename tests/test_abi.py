@@ -65,6 +65,25 @@ def test_plan_query(L):
     assert L.qoq_plan(4, 100, 128, None, None) == 2
 
 
+def test_kv4_argument_validation_without_launch(L):
+    dummy = ctypes.c_void_p(16 * 1024)   # never dereferenced: every call below fails validation first
+    w = L.qoq_kv4_cache_write
+    assert w(dummy, 2, 8, 64, 0, 64, 96, dummy, dummy, dummy, None) == 2      # D not 64 or 128
+    assert w(dummy, 2, 8, 64, 10, 60, 128, dummy, dummy, dummy, None) == 1    # past max_tokens
+    assert w(None, 2, 8, 64, 0, 4, 128, dummy, dummy, dummy, None) == 1       # no source
+    assert w(ctypes.c_void_p(16 * 1024 + 8), 2, 8, 64, 0, 4, 128, dummy, dummy, dummy, None) == 3
+    assert w(None, 0, 8, 64, 0, 4, 128, None, None, None, None) == 0          # B = 0: no-op
+    a = L.qoq_kv4_decode_attention
+    n = ctypes.c_size_t(0)
+    assert a(*([None] * 8), 64, 32, 8, 1024, 128, None, None, ctypes.byref(n), None) == 0
+    assert n.value == qoq.kv4_workspace_bytes(64, 32, 8, 1024, 128) > 4 * 64 * 8
+    assert a(*([dummy] * 8), 2, 30, 8, 64, 128, dummy, dummy, _sz(1 << 30), None) == 2   # Hq % Hkv
+    assert a(*([dummy] * 8), 2, 72, 8, 64, 128, dummy, dummy, _sz(1 << 30), None) == 2   # group of 9
+    assert a(*([dummy] * 8), 2, 32, 8, 64, 128, dummy, dummy, _sz(8), None) == 4         # workspace too small
+    assert a(*([dummy] * 8), 2, 32, 8, 64, 128, dummy, ctypes.c_void_p(16 * 1024 + 16), _sz(1 << 30),
+             None) == 3                                                                    # workspace alignment
+
+
 def test_workspace_size_query(L):
     small = qoq.workspace_bytes(1, 4096, 4096)
     big = qoq.workspace_bytes(4096, 4096, 4096)

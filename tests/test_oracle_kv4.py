@@ -147,3 +147,10 @@ def test_llama3_8b_heads_shape(D):
                                            seed=9)
     o = kv4.decode_attention(q, *_cache(K, V))
     assert o.shape == (2, 32, D) and np.all(np.isfinite(o))
+
+
+def test_pack_kv4_hand_worked():
+    """Codes 1, 2, 3, ..., 8 pack to bytes 0x21, 0x43, 0x65, 0x87 (low nibble
+    the even dimension); 15, 0 -> 0x0F; 0, 15 -> 0xF0."""
+    q = np.array([[1, 2, 3, 4, 5, 6, 7, 8], [15, 0, 0, 15, 9, 9, 0, 0]], dtype=np.uint8)
+    assert kv4.pack_kv4(q).tolist() == [[0x21, 0x43, 0x65, 0x87], [0x0F, 0xF0, 0x99, 0x00]]

@@ -210,6 +210,53 @@ qoq_status qoq_w4a8_linear(const void *X_fp16, const void *blob, int64_t M, int6
     return launch_gemm(a, s);
 }
 
+qoq_status qoq_kv4_cache_write(const void *src_fp16, int64_t B, int64_t Hkv, int64_t max_tokens, int64_t t0,
+                               int64_t n_tokens, int64_t D, uint8_t *codes, void *scales_fp16, void *zeros_fp16,
+                               void *stream) {
+    if (B < 0 || Hkv <= 0 || max_tokens <= 0 || t0 < 0 || n_tokens < 0) return QOQ_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return QOQ_ERR_UNSUPPORTED;
+    if (t0 + n_tokens > max_tokens || max_tokens > INT32_MAX) return QOQ_ERR_INVALID_ARG;
+    if (B * Hkv * max_tokens > ((int64_t)1 << 40)) return QOQ_ERR_UNSUPPORTED;
+    if (B == 0 || n_tokens == 0) return QOQ_OK;
+    if (src_fp16 == nullptr || codes == nullptr || scales_fp16 == nullptr || zeros_fp16 == nullptr)
+        return QOQ_ERR_INVALID_ARG;
+    if (!aligned(src_fp16, 16) || !aligned(codes, 16) || !aligned(scales_fp16, 2) || !aligned(zeros_fp16, 2))
+        return QOQ_ERR_ALIGNMENT;
+    return launch_kv4_cache_write(src_fp16, B, Hkv, max_tokens, t0, n_tokens, D, codes, scales_fp16, zeros_fp16,
+                                  static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? QOQ_OK
+               : QOQ_ERR_CUDA;
+}
+
+qoq_status qoq_kv4_decode_attention(const void *q_fp16, const uint8_t *k_codes, const void *k_scales,
+                                    const void *k_zeros, const uint8_t *v_codes, const void *v_scales,
+                                    const void *v_zeros, const int32_t *seq_lens, int64_t B, int64_t Hq, int64_t Hkv,
+                                    int64_t max_tokens, int64_t D, void *out_fp16, void *workspace,
+                                    size_t *workspace_bytes, void *stream) {
+    if (workspace_bytes == nullptr) return QOQ_ERR_INVALID_ARG;
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || max_tokens <= 0) return QOQ_ERR_INVALID_ARG;
+    if (Hq % Hkv != 0 || Hq / Hkv > 8 || (D != 64 && D != 128)) return QOQ_ERR_UNSUPPORTED;
+    if (B > 65535 || Hkv > 65535 || max_tokens > INT32_MAX / 2) return QOQ_ERR_UNSUPPORTED;
+    const size_t need = kv4_workspace_bytes(B, Hkv, max_tokens, D);
+    if (workspace == nullptr) {
+        *workspace_bytes = need;
+        return QOQ_OK;
+    }
+    if (*workspace_bytes < need) return QOQ_ERR_WORKSPACE;
+    if (B == 0) return QOQ_OK;
+    if (q_fp16 == nullptr || k_codes == nullptr || k_scales == nullptr || k_zeros == nullptr || v_codes == nullptr ||
+        v_scales == nullptr || v_zeros == nullptr || out_fp16 == nullptr)
+        return QOQ_ERR_INVALID_ARG;
+    if (!aligned(q_fp16, 16) || !aligned(k_codes, 16) || !aligned(v_codes, 16) || !aligned(out_fp16, 16) ||
+        !aligned(workspace, 256) || !aligned(k_scales, 2) || !aligned(k_zeros, 2) || !aligned(v_scales, 2) ||
+        !aligned(v_zeros, 2) || (seq_lens && !aligned(seq_lens, 4)))
+        return QOQ_ERR_ALIGNMENT;
+    return launch_kv4_attention(q_fp16, k_codes, k_scales, k_zeros, v_codes, v_scales, v_zeros, seq_lens, B, Hq, Hkv,
+                                max_tokens, D, out_fp16, workspace, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? QOQ_OK
+               : QOQ_ERR_CUDA;
+}
+
 qoq_status qoq_plan(int64_t M, int64_t N, int64_t K, int32_t *token_tile, int32_t *linear_launches) {
     if (M < 0 || M > INT32_MAX) return QOQ_ERR_INVALID_ARG;
     qoq_status st = check_nk(N, K);

@@ -137,6 +137,14 @@ cudaError_t launch_rmsnorm_quant(const void *X, const void *gamma, int64_t M, in
 cudaError_t launch_silu_mul_quant(const void *GU, int64_t M, int64_t I, int8_t *X8, void *s_x, int32_t *rowsum,
                                   cudaStream_t stream);
 
+// KV4 cache and decode attention (kv4_attention.cu).
+cudaError_t launch_kv4_cache_write(const void *src, int64_t B, int64_t Hkv, int64_t Tmax, int64_t t0, int64_t nt,
+                                   int64_t D, uint8_t *codes, void *scales, void *zeros, cudaStream_t stream);
+size_t kv4_workspace_bytes(int64_t B, int64_t Hkv, int64_t Tmax, int64_t D);
+cudaError_t launch_kv4_attention(const void *q, const uint8_t *kc, const void *ks, const void *kz, const uint8_t *vc,
+                                 const void *vs, const void *vz, const int32_t *seq_lens, int64_t B, int64_t Hq,
+                                 int64_t Hkv, int64_t Tmax, int64_t D, void *out, void *ws, cudaStream_t stream);
+
 // Row width limit of the fused producers (the FP32 row lives in shared memory).
 constexpr int kMaxProducerWidth = 32768;
 

@@ -49,6 +49,10 @@ def lib() -> ctypes.CDLL:
         L.qoq_gemm_fp16_out_saturating.restype = ctypes.c_int
         L.qoq_w4a8_linear.argtypes = [vp, vp, i64, i64, i64, i32, vp, vp, sz, vp]
         L.qoq_w4a8_linear.restype = ctypes.c_int
+        L.qoq_kv4_cache_write.argtypes = [vp, i64, i64, i64, i64, i64, i64, vp, vp, vp, vp]
+        L.qoq_kv4_cache_write.restype = ctypes.c_int
+        L.qoq_kv4_decode_attention.argtypes = [vp] * 8 + [i64] * 5 + [vp, vp, sz, vp]
+        L.qoq_kv4_decode_attention.restype = ctypes.c_int
         L.qoq_plan.argtypes = [i64, i64, i64, vp, vp]
         L.qoq_plan.restype = ctypes.c_int
         L.qoq_watchdog_selftest.argtypes = [vp, i64, vp]
@@ -279,3 +283,54 @@ def linear(X, blob, N, K, group_size=GROUP, ws=None, Y=None, stream=None):
     _check("qoq_w4a8_linear", lib().qoq_w4a8_linear(_ptr(X), _ptr(blob), M, N, K, group_size, _ptr(Y), _ptr(ws.buf),
                                                     ctypes.byref(n), _stream(stream)))
     return Y
+
+
+# ------------------------------------------------------------------ KV4
+
+class KV4Cache:
+    """A per-head, dynamic, asymmetric 4-bit cache of one tensor (K or V):
+    codes uint8 [B][Hkv][max_tokens][D/2], scales and zeros FP16
+    [B][Hkv][max_tokens] (include/qoq.h, qoq_kv4_cache_write)."""
+
+    def __init__(self, B, Hkv, max_tokens, D, device="cuda"):
+        import torch
+        self.B, self.Hkv, self.T, self.D = B, Hkv, max_tokens, D
+        self.codes = torch.zeros((B, Hkv, max_tokens, D // 2), dtype=torch.uint8, device=device)
+        self.scales = torch.zeros((B, Hkv, max_tokens), dtype=torch.float16, device=device)
+        self.zeros = torch.zeros((B, Hkv, max_tokens), dtype=torch.float16, device=device)
+
+    def write(self, src, t0=0, stream=None):
+        """Quantise src [B][Hkv][n][D] FP16 into slots t0 .. t0 + n - 1."""
+        import torch
+        src = _cuda_tensor(src, torch.float16, "src")
+        B, H, n, D = src.shape
+        if (B, H, D) != (self.B, self.Hkv, self.D):
+            raise ValueError("src shape %s does not match the cache" % (tuple(src.shape),))
+        _check("qoq_kv4_cache_write", lib().qoq_kv4_cache_write(_ptr(src), B, H, self.T, t0, n, D, _ptr(self.codes),
+                                                                _ptr(self.scales), _ptr(self.zeros),
+                                                                _stream(stream)))
+        return self
+
+
+def kv4_workspace_bytes(B, Hq, Hkv, max_tokens, D) -> int:
+    n = ctypes.c_size_t(0)
+    _check("qoq_kv4_decode_attention", lib().qoq_kv4_decode_attention(*([None] * 8), B, Hq, Hkv, max_tokens, D, None,
+                                                                      None, ctypes.byref(n), None))
+    return n.value
+
+
+def kv4_decode_attention(q, kcache, vcache, seq_lens=None, ws=None, out=None, stream=None):
+    """q [B][Hq][D] FP16 against the KV4 caches -> out [B][Hq][D] FP16."""
+    import torch
+    q = _cuda_tensor(q, torch.float16, "q")
+    B, Hq, D = q.shape
+    if seq_lens is not None:
+        seq_lens = _cuda_tensor(seq_lens, torch.int32, "seq_lens")
+    ws = ws or Workspace(kv4_workspace_bytes(B, Hq, kcache.Hkv, kcache.T, D), q.device)
+    out = torch.empty((B, Hq, D), dtype=torch.float16, device=q.device) if out is None else out
+    n = ctypes.c_size_t(ws.buf.numel())
+    _check("qoq_kv4_decode_attention", lib().qoq_kv4_decode_attention(
+        _ptr(q), _ptr(kcache.codes), _ptr(kcache.scales), _ptr(kcache.zeros), _ptr(vcache.codes),
+        _ptr(vcache.scales), _ptr(vcache.zeros), _ptr(seq_lens), B, Hq, kcache.Hkv, kcache.T, D, _ptr(out),
+        _ptr(ws.buf), ctypes.byref(n), _stream(stream)))
+    return out
