@@ -371,6 +371,7 @@ def run_gpu(args, rank, world, local_rank):
     res["e2e"] = run_e2e(args, probs, qoq, stream) if rank == 0 else None
     res["w8a8_context"] = run_w8a8(probs, stream, res["gemm_us_per_step"], max(K, 10)) if rank == 0 else None
     res["producers_context"] = run_producers(stream, peaks) if rank == 0 and not args.no_context else None
+    res["kv4_attention_context"] = run_kv4(stream, peaks) if rank == 0 and not args.no_context else None
     res["saturation_context"] = run_saturation(stream) if rank == 0 and args.saturation else None
     return res
 
@@ -650,6 +651,55 @@ def run_producers(stream, peaks, reps=20):
             del xs, fp16_in, x
     torch.cuda.empty_cache()
     return out
+
+
+def run_kv4(stream, peaks, reps=20):
+    """KV4 decode attention (context, not in the timed step): batch 64 x 1024
+    cached tokens, Llama-3-8B heads (32 query heads over 8 KV heads, D = 128),
+    the pages' attention measurement shape. One graph of `reps` launches,
+    alternating between two copies of the 4-bit cache (142 MB together, more
+    than L2), events around the replays. Algorithmic bytes per launch: K and V
+    codes (D/2 bytes per token and head) with their FP16 scale and zero, the
+    FP16 queries and outputs. Beside it, the same attention over FP16 K/V
+    through PyTorch's scaled_dot_product_attention (the library's kernel,
+    context for the pages' KV4-over-FP16 argument)."""
+    import torch
+    from w4a8_quantized_gemm_qoq_b200 import qoq
+    dev = torch.device("cuda", torch.cuda.current_device())
+    a = inputs.LLAMA3_8B_ATTN
+    B, T, Hq, Hkv, D = 64, 1024, a["Hq"], a["Hkv"], a["D"]
+    q, K, V = inputs.make_decode_attention(B, T, Hq, Hkv, D, seed=21)
+    qd = torch.from_numpy(q).to(dev)
+    Kd, Vd = torch.from_numpy(K).to(dev), torch.from_numpy(V).to(dev)
+    caches = []
+    for _ in range(2):
+        caches.append((qoq.KV4Cache(B, Hkv, T, D).write(Kd), qoq.KV4Cache(B, Hkv, T, D).write(Vd)))
+    ws = qoq.Workspace(qoq.kv4_workspace_bytes(B, Hq, Hkv, T, D))
+    out = torch.empty((B, Hq, D), dtype=torch.float16, device=dev)
+    torch.cuda.synchronize()
+    stream.wait_stream(torch.cuda.current_stream())
+    us = graph_time_us(lambda: [qoq.kv4_decode_attention(qd, *caches[i % 2], ws=ws, out=out) for i in range(reps)],
+                       stream, 2) / reps
+    nbytes = 2 * B * Hkv * T * (D // 2 + 4) + 2 * B * Hq * D * 2
+    res = {"B": B, "T": T, "Hq": Hq, "Hkv": Hkv, "D": D, "us": round(us, 3), "GBps": round(nbytes / us / 1e3, 1),
+           "frac_of_hbm": round(nbytes / us / 1e3 / peaks["hbm"], 3), "bytes_per_launch": nbytes,
+           "kernel": "kv4_attn_kernel (one launch)"}
+    try:
+        import torch.nn.functional as F
+        q4 = qd.view(B, Hq, 1, D)
+        kv16 = [(Kd, Vd), (Kd.clone(), Vd.clone())]
+        with torch.cuda.stream(stream):   # eager first call: kernel selection and workspace outside capture
+            F.scaled_dot_product_attention(q4, Kd, Vd, enable_gqa=True)
+        stream.synchronize()
+        us16 = graph_time_us(lambda: [F.scaled_dot_product_attention(q4, *kv16[i % 2], enable_gqa=True)
+                                      for i in range(reps)], stream, 2) / reps
+        res["fp16_kv_sdpa_us"] = round(us16, 3)
+        res["kv4_speedup_over_fp16_kv"] = round(us16 / us, 3)
+    except Exception as exc:   # context only
+        res["fp16_kv_sdpa"] = "unavailable: %s" % str(exc)[:120]
+    del caches, Kd, Vd
+    torch.cuda.empty_cache()
+    return res
 
 
 def run_w8a8(probs, stream, w4a8_us, reps):

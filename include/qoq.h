@@ -337,10 +337,15 @@ qoq_status qoq_kv4_cache_write(const void *src_fp16, int64_t B, int64_t Hkv, int
  *   k_t, v_t = (q_t - z_t) * s_t            (dequantised key / value, t < T_b)
  *   score_t = (q . k_t) / sqrt(D);  p = softmax_t(score);  out = sum_t p_t v_t
  *
- * computed in FP32 on CUDA cores and rounded once to FP16; the order of the
- * sums is the kernel's (tokens in chunks of 256, chunks combined with the
- * usual running-maximum rescaling), so results are compared with the exact
- * mathematics under a tolerance, not bit for bit.
+ * The products run on tensor cores with FP16 inputs and FP32 accumulation:
+ * the 4-bit codes enter them exactly (as FP16 values c * 2^-24 and c * 2^-20),
+ * the zero points are subtracted in FP32 (z * sum(q) from each score,
+ * z * (P s) from each output), the softmax weights times the value scale are
+ * rounded to FP16 for the second product, and the output is rounded once to
+ * FP16. The order of the sums is the kernel's (64-token tiles per warp,
+ * spans of 256 * t tokens per CTA, combined with the usual running-maximum
+ * rescaling), so results are compared with the exact mathematics under a
+ * tolerance (|o - o*| <= 2^-10 max|v| + 2^-24 per head), not bit for bit.
  *
  * q_fp16 [B][Hq][D] FP16; the K and V caches as written by
  * qoq_kv4_cache_write (same B, Hkv, max_tokens, D); seq_lens int32 [B] with
@@ -348,11 +353,15 @@ qoq_status qoq_kv4_cache_write(const void *src_fp16, int64_t B, int64_t Hkv, int
  * FP16, written. Hq must be a multiple of Hkv with Hq / Hkv <= 8, D 64 or 128.
  *
  * Workspace: device memory of *workspace_bytes bytes (size query with
- * workspace == NULL), zero-filled by the caller before its first use; its
- * leading 4 * B * Hkv bytes are per-(sequence, head) counters that every
- * call which completes leaves zero, the rest is scratch for the chunks'
- * partial results. Calls that may overlap on the device need separate
- * workspaces. A seq_lens entry outside [1, max_tokens] is clamped into it.
+ * workspace == NULL; 256-byte aligned), zero-filled by the caller before its
+ * first use. Bytes [0, 256) are the status words: int32 [0] stays 0, or
+ * becomes QOQ_ERR_TIMEOUT with [1] = 10 (a warp's wait for its K/V code copy
+ * ran out after 1 s), [2] = the CTA's x index, [3] = 2 * tile + (0 for K,
+ * 1 for V); the caller clears it. Then 4 * B * Hkv bytes of per-(sequence,
+ * head) counters that every call which completes leaves zero; the rest is
+ * scratch for the CTAs' partial results. Calls that may overlap on the
+ * device need separate workspaces. A seq_lens entry outside [1, max_tokens]
+ * is clamped into it.
  */
 qoq_status qoq_kv4_decode_attention(const void *q_fp16, const uint8_t *k_codes, const void *k_scales,
                                     const void *k_zeros, const uint8_t *v_codes, const void *v_scales,

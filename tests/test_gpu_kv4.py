@@ -2,17 +2,9 @@
 (oracle/kv4.py), through the C ABI.
 
 Bar: the cache write (codes, FP16 scales, FP16 zeros) bit-exact; the
-attention output within
-
-    |o - o*| <= 2^-10 * max_t |v_hat_t| + 2^-24
-
-of the exact mathematics o* (binary64), per (sequence, query head), where
-max_t |v_hat_t| is the largest dequantised value of that sequence's V. The
-bound: the kernel rounds the softmax weights times the value scale to FP16
-for the tensor-core product (relative error <= 2^-11 per weight, so at most
-2^-11 max|v_hat| on the weighted mean), rounds the output once to FP16 (at
-most 2^-11 |o*| <= 2^-11 max|v_hat|), and sums in FP32 (errors near 2^-20
-relative, inside the slack of the first two terms' worst cases).
+attention output within the tolerance stated in tests/kv4_check.py, which
+holds the shared attention checks and is also run in processes of its own
+with longer warp walks forced.
 """
 import numpy as np
 import pytest
@@ -20,6 +12,7 @@ import pytest
 from oracle import kv4
 from w4a8_quantized_gemm_qoq_b200 import inputs, qoq
 from gpu_helpers import dev, host, torch
+from kv4_check import check_attention, run_attention
 
 pytestmark = [pytest.mark.gpu, pytest.mark.filterwarnings("ignore::RuntimeWarning")]
 
@@ -75,38 +68,8 @@ def test_cache_append_one_token():
     _check_cache(c, K)
 
 
-def _attention(q, K, V, Tmax=None, seq_lens=None):
-    B, Hkv, T, D = K.shape
-    Hq = q.shape[1]
-    Tmax = Tmax or T
-    kc = qoq.KV4Cache(B, Hkv, Tmax, D).write(dev(K))
-    vc = qoq.KV4Cache(B, Hkv, Tmax, D).write(dev(V))
-    ws = qoq.Workspace(qoq.kv4_workspace_bytes(B, Hq, Hkv, Tmax, D))
-    sl = dev(np.asarray(seq_lens, dtype=np.int32)) if seq_lens is not None else None
-    out = qoq.kv4_decode_attention(dev(q), kc, vc, seq_lens=sl, ws=ws)
-    torch().cuda.synchronize()
-    assert not bool(ws.buf[:4 * B * Hkv].any().item()), "arrival counters not left zero"
-    return host(out), (kc, vc, ws, sl)
-
-
-def _check_attention(out, q, K, V, seq_lens=None):
-    B, Hkv, T, D = K.shape
-    Hq = q.shape[1]
-    G = Hq // Hkv
-    worst = 0.0
-    for b in range(B):
-        Tb = T if seq_lens is None else int(seq_lens[b])
-        Kb = kv4.quantize_kv4(K[b:b + 1, :, :Tb])
-        Vb = kv4.quantize_kv4(V[b:b + 1, :, :Tb])
-        want = kv4.decode_attention(q[b:b + 1], Kb, Vb)[0]
-        vh = np.abs(kv4.dequantize_kv4(Vb["q"], Vb["s"], Vb["z"]).astype(np.float64))[0]
-        for hq in range(Hq):
-            vmax = vh[hq // G].max()
-            err = np.abs(out[b, hq].astype(np.float64) - want[hq]).max()
-            tol = 2.0 ** -10 * vmax + 2.0 ** -24
-            assert err <= tol, "b=%d hq=%d: error %.3g above %.3g" % (b, hq, err, tol)
-            worst = max(worst, err / (2.0 ** -10 * vmax + 2.0 ** -24))
-    return worst
+_attention = run_attention
+_check_attention = check_attention
 
 
 @pytest.mark.parametrize("B,T,Hq,Hkv,D", [(2, 1, 8, 8, 128), (3, 7, 8, 2, 64), (2, 128, 32, 8, 128),
@@ -161,4 +124,20 @@ def test_decode_attention_graph_replays():
             g.replay()
         stream.synchronize()
         assert np.array_equal(host(out).view(np.uint16), out0.view(np.uint16))
-        assert not bool(ws.buf[:4 * 8 * 8].any().item())
+        assert not bool(ws.buf[:256 + 4 * 8 * 8].any().item())
+
+
+@pytest.mark.parametrize("kvt", [2, 3, 8])
+def test_decode_attention_longer_warp_walks(kvt):
+    """Every warp walks up to kvt 64-token tiles (QOQ_FORCE_CONFIG=kvt=N, in a
+    process of its own), refilling its K and V buffers while it computes:
+    ragged last tiles, warps with fewer tiles than others, spans longer than
+    the sequence."""
+    import os
+    import subprocess
+    import sys
+    here = os.path.dirname(os.path.abspath(__file__))
+    env = dict(os.environ, QOQ_FORCE_CONFIG="kvt=%d" % kvt)
+    r = subprocess.run([sys.executable, os.path.join(here, "kv4_check.py")], env=env, capture_output=True,
+                       text=True, timeout=900)
+    assert r.returncode == 0 and "kv4_check ok" in r.stdout, r.stdout[-2000:] + r.stderr[-4000:]

@@ -9,6 +9,8 @@
 //     fuse=0|1               qoq_w4a8_linear: quantise the activations inside
 //                            the decode GEMM's launch (1) or with the separate
 //                            quantiser first (0)
+//     kvt=1..8               KV4 attention: 64-token tiles per warp (sets the
+//                            tokens per CTA to 256 * kvt)
 // Unknown keys and values are ignored.
 #include <cstdlib>
 #include <cstring>
@@ -35,6 +37,9 @@ const ForcedConfig &forced_config() {
             } else if (len > 4 && std::strncmp(p, "cps=", 4) == 0) {
                 v = std::atoi(p + 4);
                 if (v == 1 || v == 2) cfg.cps = v;
+            } else if (len > 4 && std::strncmp(p, "kvt=", 4) == 0) {
+                v = std::atoi(p + 4);
+                if (v >= 1 && v <= 8) cfg.kvt = v;
             } else if (len > 5 && std::strncmp(p, "fuse=", 5) == 0) {
                 v = std::atoi(p + 5);
                 if (v == 0 || v == 1) cfg.fuse = v + 1;

@@ -71,6 +71,7 @@ enum WaitSite : int {
     kSiteLastOwner = 7,       // last arriver of a split tile waiting for the owner's partial sums
     kSiteRowsDone = 8,        // fused activation quantisation: waiting for every token row
     kSiteXEmpty = 9,          // token-tile producer / dequantiser waiting for a free A/X stage
+    kSiteKvTile = 10,         // KV4 attention warp waiting for its K/V code tile
 };
 
 // Shared abort flag + global status word used by the bounded waits. The CTA

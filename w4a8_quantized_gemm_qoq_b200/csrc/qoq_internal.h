@@ -60,6 +60,7 @@ struct ForcedConfig {
     int tok = 0;   // token tile
     int cps = 0;   // CTAs per SM of the decode kernel
     int fuse = 0;  // qoq_w4a8_linear at token tiles <= 64: 1 = separate quantiser, 2 = fused launch
+    int kvt = 0;   // KV4 attention: 64-token tiles per warp
 };
 
 // Whether qoq_w4a8_linear quantises the activations inside the decode GEMM's
