@@ -203,13 +203,17 @@ qoq_status qoq_gemm_fp16_out(const int8_t *X8, const void *s_x_fp16, const int32
  *   X8, s_x, rowsum = qoq_quantize_act_per_token(X)   (same arithmetic)
  *   Y = qoq_gemm_fp16_out(X8, s_x, rowsum, blob)       (same arithmetic)
  *
- * When the library picks token tiles of at most 64 tokens for (M, N, K)
- * (decode batches), both steps run in ONE launch: the GEMM's CTAs quantise
- * the token rows first (rows are claimed from a counter in the workspace, so
- * no CTA waits for one that has not started) and stream their first weight
- * tiles meanwhile. For wider token tiles the call launches the quantiser and
- * then the GEMM. Either way the codes, scales and row sums are written into
- * the workspace, after the GEMM's scratch.
+ * By default the call launches the quantiser and then the GEMM (two
+ * launches; the GEMM's weight copies start while the quantiser runs). For
+ * token tiles of at most 64 tokens (decode batches) a one-launch form is
+ * built as well: the GEMM's CTAs quantise the token rows first (rows are
+ * claimed from a counter in the workspace, so no CTA waits for one that has
+ * not started) and stream their first weight tiles meanwhile. It measured
+ * slower on B200 (its claim/publish/poll chain costs more than the second
+ * launch), so it runs only when the environment variable QOQ_FORCE_CONFIG
+ * holds fuse=1; qoq_plan reports which form a problem gets. Either way the
+ * codes, scales and row sums are written into the workspace, after the
+ * GEMM's scratch.
  *
  * X_fp16 [M][K] FP16, read; Y_fp16 [M][N] FP16, written; blob as for
  * qoq_gemm_fp16_out. The workspace must be 256-byte aligned, zero-filled by
@@ -250,16 +254,16 @@ qoq_status qoq_gemm_fp16_out_saturating(const int8_t *X8, const void *s_x_fp16, 
  * workspace of qoq_gemm_fp16_out need not be allocated by the caller.
  *
  * Same computation and arguments as qoq_gemm_fp16_out, except that the
- * stream-K scratch lives in one fixed 16 MiB device array inside the library,
+ * stream-K scratch lives in one fixed 8 MiB device array inside the library,
  * which every GPU that loads the library keeps until the process exits. That
- * bounds the problem: the call needs 1280 + C * P * T * 512 bytes, where T is
- * the token tile the library picks for (M, N, K), C the CTAs of the launch
- * (min(SM count, 256, token tiles * N/128 * K/128); twice the CTA pairs for
- * 256-token tiles) and P the partial-sum slots per CTA (2 for token tiles up
- * to 64, else 1). On a 148-SM B200 every problem whose token tile is at most
- * 64 fits (9.7 MB at most): all M <= 64, and M up to 256 where few weight
- * tiles make the library keep 64-token tiles (e.g. N = K = 4096). Larger
- * problems return QOQ_ERR_WORKSPACE and launch nothing.
+ * bounds the problem: the call needs 1280 + C * T * 512 bytes (one INT32
+ * partial-sum tile of T x 128 per CTA), where T is the token tile the library
+ * picks for (M, N, K) and C the CTAs of the launch (min(SM count, token
+ * tiles * N/128 * K/128); twice the CTA pairs for 256-token tiles). On a
+ * 148-SM B200 every problem whose token tile is at most 64 fits (4.9 MB at
+ * most): all M <= 64, and M up to 256 where few weight tiles make the library
+ * keep 64-token tiles (e.g. N = K = 4096). Larger problems return
+ * QOQ_ERR_WORKSPACE and launch nothing.
  *
  * status: optional device int32; when non-NULL the call copies the device
  * status word of this call (0, QOQ_ERR_BAD_BLOB or QOQ_ERR_TIMEOUT) into it
@@ -373,7 +377,8 @@ qoq_status qoq_kv4_decode_attention(const void *q_fp16, const uint8_t *k_codes, 
  * Launch plan of a problem (no device work; the library has no counterpart
  * in the QServe pages): the token tile (MMA N: 16, 32, 64, 128 or 256) the
  * GEMM calls use for (M, N, K), and how many kernels qoq_w4a8_linear
- * launches for it (1 when the token tile is at most 64, else 2). Either
+ * launches for it (2, or 1 when the one-launch form is selected by
+ * QOQ_FORCE_CONFIG=fuse=1 and the token tile is at most 64). Either
  * output pointer may be NULL. Returns QOQ_ERR_INVALID_ARG / _UNSUPPORTED for
  * shapes the GEMM calls reject.
  */
