@@ -56,6 +56,12 @@ constexpr int kWarpProducer = 0;
 constexpr int kWarpMma = 1;             // warps 1, 2: the two MMA issuers
 constexpr int kIssuers = 2;
 constexpr int kWarpDequant0 = 4;         // warps 4..: the dequant warpgroups, then the epilogue warpgroups
+// Register budgets of the 256-token configuration (512 threads launched with
+// 128 registers each): control warpgroup 56, dequant 128, epilogue 2 x 160.
+constexpr int kRegsCtlHalves = 56;
+constexpr int kRegsEpiHalves = 160;
+static_assert(128 * kRegsCtlHalves + 128 * 128 + 256 * kRegsEpiHalves <= kThreads * 128,
+              "register split exceeds the launch pool");
 
 template <int TOK, int MODE, bool PAIR = false>
 struct GemmCfg {
@@ -256,6 +262,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto stage_w = [&](int s) { return smem + s * C::kStageBytes + C::kXBytes; };
 
     if (!bad_blob) {
+        // 256-token tiles: the epilogue warpgroups hold half a tile of packed
+        // FP16 results in registers (to hand the accumulator back early), so
+        // the control warpgroup gives them part of its budget; each
+        // warpgroup sets it at the top of its own branch.
+        if (warp < kWarpDequant0) {
+        if constexpr (C::kHalves) regs_dec<kRegsCtlHalves>();
         if (warp == kWarpProducer) {
             // ------------------------------------------------ TMA producer
             const uint64_t pol_w = policy_evict_first();   // weights: streamed once
@@ -408,6 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 wait_drain(&ctl->final_bar[k], 0, kDrainNs);
             }
             __syncwarp();
+        }
         } else if (warp >= kWarpDequant0 && warp < C::kWarpEpi0) {
             // ------------------------------------------------ dequant
             // With two warpgroups, warpgroup g takes the units i with
@@ -493,6 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
             }
         } else if (warp >= C::kWarpEpi0) {
+            if constexpr (C::kHalves) regs_inc<kRegsEpiHalves>();
             // ------------------------------------------------ epilogue
             // kEpiGroups warpgroups. Each reads its share of the accumulator's
             // parts: with two (256-token tiles), warpgroup e takes issuer e's
