@@ -1,8 +1,8 @@
 """Benchmark of the QoQ W4A8 hot path on B200: the linear layer (per-token
 activation quantisation + W4A8 GEMM with the fused FP16 epilogue) through the
-library's one-call entry point, qoq_w4a8_linear (one launch for decode
-batches, where the GEMM quantises its own activations; the quantiser and the
-GEMM for prefill batches).
+library's one-call entry point, qoq_w4a8_linear (the quantiser, then the
+GEMM; decode batches run on the decode-regime GEMM kernel, prefill batches on
+256-token tiles of CTA pairs).
 
 One step = every GEMM of the workload once:
   llama3_8b (default): Llama-3-8B linear shapes (K->N) 4096->6144 (qkv),
@@ -421,7 +421,7 @@ def analyse(args, probs, qoq, stream, peaks, wl, world, device):
             "traffic": measured_traffic("qoq_decode_linear_llama3_8b_dram", ("gemm_decode.cu", "gemm_common.cuh",
                                                                             "qoq_device.cuh", "quant_math.cuh")),
             "algorithmic_bytes_per_launch": round(b / len(dec)), "peak_source": peaks["src"] + " (HBM copy)",
-            "kernel": "qoq_decode_kernel (one launch per linear call: per-token quantisation + GEMM)",
+            "kernel": "act_quant_kernel + qoq_decode_kernel (the linear call's two launches)",
             "frac_of_time_roofline": round(sum(roof_us(p.M, p.N, p.K, peaks, p.group)[0] for p in dec) / us, 4),
             "timing": {"launch_us": round(us / len(dec), 3), "launches": len(dec), "replays": reps,
                        "M": sorted({p.M for p in dec}),

@@ -271,7 +271,8 @@ def gemm_fp16_out_saturating(X8, s_x, blob, N, K, ws=None, Y=None, stream=None):
 def linear(X, blob, N, K, group_size=GROUP, ws=None, Y=None, stream=None):
     """The whole hot path in one call (qoq_w4a8_linear): per-token
     quantisation of X [M][K] fp16, then the W4A8 GEMM with the FP16 epilogue;
-    one launch when the token tile is at most 64 tokens. Y [M][N] fp16."""
+    two launches, or one for token tiles of at most 64 tokens when
+    QOQ_FORCE_CONFIG holds fuse=1 (plan() reports which). Y [M][N] fp16."""
     import torch
     X = _cuda_tensor(X, torch.float16, "X")
     M = X.shape[0]
