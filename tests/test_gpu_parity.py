@@ -102,6 +102,20 @@ def test_prefill_token_scales():
     check_full(X, W, 128, "scaled tokens")
 
 
+@pytest.mark.parametrize("M,K", [(1, 4096), (2000, 4096), (5000, 128), (1000, 14336), (700, 24576), (300, 32768)])
+def test_act_quant_every_row(M, K):
+    """Per-token quantisation, every row bit-exact (codes, FP16 scales, row
+    sums) with the oracle: rows held in registers (16-byte chunks per thread
+    1, 2, 8 and 12), the two-pass path (K > 24576), one row and thousands."""
+    X = inputs.make_activations(M, K, seed=K + M, token_scale_span=(-3, 1))
+    X8, s_x, rs = qoq.quantize_act_per_token(dev(X))
+    torch().cuda.synchronize()
+    X8o, s_xo, rso = oracle.quantize_act_per_token(X)
+    assert np.array_equal(host(X8), X8o)
+    assert np.array_equal(host(s_x).view(np.uint16), s_xo.view(np.uint16))
+    assert np.array_equal(host(rs), rso)
+
+
 def test_degenerate_inputs():
     """Zero rows and columns, constant rows, one-hot tokens."""
     K, N = 256, 256
