@@ -102,11 +102,13 @@ def test_prefill_token_scales():
     check_full(X, W, 128, "scaled tokens")
 
 
-@pytest.mark.parametrize("M,K", [(1, 4096), (2000, 4096), (5000, 128), (1000, 14336), (700, 24576), (300, 32768)])
+@pytest.mark.parametrize("M,K", [(1, 4096), (100, 14336), (64, 32768), (2000, 4096), (5000, 128), (1000, 14336),
+                                 (700, 24576), (300, 32768)])
 def test_act_quant_every_row(M, K):
     """Per-token quantisation, every row bit-exact (codes, FP16 scales, row
-    sums) with the oracle: rows held in registers (16-byte chunks per thread
-    1, 2, 8 and 12), the two-pass path (K > 24576), one row and thousands."""
+    sums) with the oracle, in each form the launch picks by shape: 512 threads
+    with the row in registers (a few rows), 256 threads in registers, the
+    two-pass form with 256 and 128 threads (many rows)."""
     X = inputs.make_activations(M, K, seed=K + M, token_scale_span=(-3, 1))
     X8, s_x, rs = qoq.quantize_act_per_token(dev(X))
     torch().cuda.synchronize()

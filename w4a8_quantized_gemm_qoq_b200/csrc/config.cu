@@ -11,6 +11,9 @@
 //                            quantiser first (0)
 //     kvt=1..8               KV4 attention: 64-token tiles per warp (sets the
 //                            tokens per CTA to 256 * kvt)
+//     aqt=128|256|512        activation quantiser: threads per CTA
+//     aq2=1|2                activation quantiser: the two-pass form (1) or the
+//                            row in registers where it fits (2) at every shape
 // Unknown keys and values are ignored.
 #include <cstdlib>
 #include <cstring>
@@ -37,6 +40,12 @@ const ForcedConfig &forced_config() {
             } else if (len > 4 && std::strncmp(p, "cps=", 4) == 0) {
                 v = std::atoi(p + 4);
                 if (v == 1 || v == 2) cfg.cps = v;
+            } else if (len > 4 && std::strncmp(p, "aq2=", 4) == 0) {
+                v = std::atoi(p + 4);
+                if (v == 1 || v == 2) cfg.aq2 = v;
+            } else if (len > 4 && std::strncmp(p, "aqt=", 4) == 0) {
+                v = std::atoi(p + 4);
+                if (v == 128 || v == 256 || v == 512) cfg.aqt = v;
             } else if (len > 4 && std::strncmp(p, "kvt=", 4) == 0) {
                 v = std::atoi(p + 4);
                 if (v >= 1 && v <= 8) cfg.kvt = v;

@@ -61,6 +61,8 @@ struct ForcedConfig {
     int cps = 0;   // CTAs per SM of the decode kernel
     int fuse = 0;  // qoq_w4a8_linear at token tiles <= 64: 1 = separate quantiser, 2 = fused launch
     int kvt = 0;   // KV4 attention: 64-token tiles per warp
+    int aqt = 0;   // activation quantiser: threads per CTA (one row per CTA)
+    int aq2 = 0;   // activation quantiser: 1 = the two-pass form, 2 = the register form
 };
 
 // Whether qoq_w4a8_linear quantises the activations inside the decode GEMM's

@@ -21,7 +21,6 @@ namespace qoq {
 
 // ------------------------------------------------------------ activations
 
-constexpr int kActThreads = 256;
 
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
@@ -45,13 +44,13 @@ __device__ __forceinline__ int quant_code(float x, float s, int lim) {
 // scale, then round-half-even codes and their row sum. NCH > 0 keeps the row
 // in registers (NCH 16-byte chunks per thread, one pass over HBM); NCH == 0
 // reads the row twice (any K).
-template <int NCH>
-__global__ void __launch_bounds__(kActThreads) act_quant_kernel(const __half *__restrict__ X, int K,
+template <int NCH, int TH>
+__global__ void __launch_bounds__(TH) act_quant_kernel(const __half *__restrict__ X, int K,
                                                                  int8_t *__restrict__ X8,
                                                                  __half *__restrict__ s_x,
                                                                  int32_t *__restrict__ rowsum) {
-    __shared__ float red_f[kActThreads / 32];
-    __shared__ int red_i[kActThreads / 32];
+    __shared__ float red_f[TH / 32];
+    __shared__ int red_i[TH / 32];
     __shared__ float s_shared, inv_shared;
     // X may come from the previous kernel in the stream; release the next one
     // (the GEMM) so its set-up and weight copies overlap this kernel.
@@ -78,7 +77,7 @@ __global__ void __launch_bounds__(kActThreads) act_quant_kernel(const __half *__
     if (NCH > 0) {
 #pragma unroll
         for (int i = 0; i < NR; ++i) {
-            const int k = (i * kActThreads + threadIdx.x) * 8;
+            const int k = (i * TH + threadIdx.x) * 8;
             // The load address is clamped into the row, so no form of the
             // guard can read past the end of X; out-of-row chunks become 0.
             const uint4 u = *reinterpret_cast<const uint4 *>(row + (k < K ? k : K - 8));
@@ -86,14 +85,14 @@ __global__ void __launch_bounds__(kActThreads) act_quant_kernel(const __half *__
             absmax8(v[i]);
         }
     } else {
-        for (int k = threadIdx.x * 8; k < K; k += kActThreads * 8) absmax8(*reinterpret_cast<const uint4 *>(row + k));
+        for (int k = threadIdx.x * 8; k < K; k += TH * 8) absmax8(*reinterpret_cast<const uint4 *>(row + k));
     }
     amax = warp_max(amax);
     if (lane == 0) red_f[warp] = amax;
     __syncthreads();
     if (threadIdx.x == 0) {
         float a = red_f[0];
-        for (int w = 1; w < kActThreads / 32; ++w) a = fmaxf(a, red_f[w]);
+        for (int w = 1; w < TH / 32; ++w) a = fmaxf(a, red_f[w]);
         __half sh = __float2half_rn(__fdiv_rn(a, 127.0f));
         s_x[m] = sh;
         s_shared = __half2float(sh);
@@ -124,11 +123,11 @@ __global__ void __launch_bounds__(kActThreads) act_quant_kernel(const __half *__
     if (NCH > 0) {
 #pragma unroll
         for (int i = 0; i < NR; ++i) {
-            const int k = (i * kActThreads + threadIdx.x) * 8;
+            const int k = (i * TH + threadIdx.x) * 8;
             if (k < K) quant8(v[i], k);
         }
     } else {
-        for (int k = threadIdx.x * 8; k < K; k += kActThreads * 8) quant8(*reinterpret_cast<const uint4 *>(row + k), k);
+        for (int k = threadIdx.x * 8; k < K; k += TH * 8) quant8(*reinterpret_cast<const uint4 *>(row + k), k);
     }
     if (rowsum != nullptr) {
         sum = warp_sum(sum);
@@ -136,38 +135,66 @@ __global__ void __launch_bounds__(kActThreads) act_quant_kernel(const __half *__
         __syncthreads();
         if (threadIdx.x == 0) {
             int t = 0;
-            for (int w = 0; w < kActThreads / 32; ++w) t += red_i[w];
+            for (int w = 0; w < TH / 32; ++w) t += red_i[w];
             rowsum[m] = t;
         }
     }
 }
 
-template <int NCH>
+template <int NCH, int TH>
 static cudaError_t launch_act_quant_t(const void *X, int64_t M, int64_t K, int8_t *X8, void *s_x,
                                       int32_t *rowsum, cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)M);
-    cfg.blockDim = dim3(kActThreads);
+    cfg.blockDim = dim3(TH);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = kProgrammaticLaunch ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, act_quant_kernel<NCH>, static_cast<const __half *>(X), (int)K, X8,
+    return cudaLaunchKernelEx(&cfg, act_quant_kernel<NCH, TH>, static_cast<const __half *>(X), (int)K, X8,
                               static_cast<__half *>(s_x), rowsum);
 }
 
+template <int TH>
+static cudaError_t launch_act_quant_th(const void *X, int64_t M, int64_t K, int8_t *X8, void *s_x, int32_t *rowsum,
+                                       bool two_pass, cudaStream_t stream) {
+    const int64_t per_pass = (int64_t)TH * 8;   // halves one pass of the CTA covers
+    const int64_t nch = (K + per_pass - 1) / per_pass;
+    if (two_pass) return launch_act_quant_t<0, TH>(X, M, K, X8, s_x, rowsum, stream);
+    if (nch <= 1) return launch_act_quant_t<1, TH>(X, M, K, X8, s_x, rowsum, stream);
+    if (nch <= 2) return launch_act_quant_t<2, TH>(X, M, K, X8, s_x, rowsum, stream);
+    if (nch <= 4) return launch_act_quant_t<4, TH>(X, M, K, X8, s_x, rowsum, stream);
+    if (nch <= 8) return launch_act_quant_t<8, TH>(X, M, K, X8, s_x, rowsum, stream);
+    if (nch <= 12) return launch_act_quant_t<12, TH>(X, M, K, X8, s_x, rowsum, stream);
+    return launch_act_quant_t<0, TH>(X, M, K, X8, s_x, rowsum, stream);
+}
+
+// CTA size and form by shape, from B200 measurements on the Llama-3-8B rows
+// (K = 4096 and 14336, M = 16 .. 16384): a few rows want the most threads per
+// row (the row's latency is the launch's); many rows want the most rows in
+// flight per SM, i.e. few registers per thread (the two-pass form reads each
+// row twice, the second time from L1/L2, and keeps nothing in registers).
+// Same arithmetic in every form.
 cudaError_t launch_act_quant(const void *X, int64_t M, int64_t K, int8_t *X8, void *s_x, int32_t *rowsum,
                              cudaStream_t stream) {
-    const int64_t per_pass = (int64_t)kActThreads * 8;   // halves one pass of the CTA covers
-    const int64_t nch = (K + per_pass - 1) / per_pass;
-    if (nch <= 1) return launch_act_quant_t<1>(X, M, K, X8, s_x, rowsum, stream);
-    if (nch <= 2) return launch_act_quant_t<2>(X, M, K, X8, s_x, rowsum, stream);
-    if (nch <= 4) return launch_act_quant_t<4>(X, M, K, X8, s_x, rowsum, stream);
-    if (nch <= 8) return launch_act_quant_t<8>(X, M, K, X8, s_x, rowsum, stream);
-    if (nch <= 12) return launch_act_quant_t<12>(X, M, K, X8, s_x, rowsum, stream);
-    return launch_act_quant_t<0>(X, M, K, X8, s_x, rowsum, stream);
+    int th;
+    bool two_pass;
+    if (M <= 256) {
+        th = 512, two_pass = false;
+    } else if (K > 4096) {
+        th = 256, two_pass = true;
+    } else if (M <= 4096) {
+        th = 256, two_pass = false;
+    } else {
+        th = 128, two_pass = true;
+    }
+    if (forced_config().aqt) th = forced_config().aqt;
+    if (forced_config().aq2) two_pass = forced_config().aq2 == 1;
+    if (th == 128) return launch_act_quant_th<128>(X, M, K, X8, s_x, rowsum, two_pass, stream);
+    if (th == 512) return launch_act_quant_th<512>(X, M, K, X8, s_x, rowsum, two_pass, stream);
+    return launch_act_quant_th<256>(X, M, K, X8, s_x, rowsum, two_pass, stream);
 }
 
 // ---------------------------------------------------------------- weights
