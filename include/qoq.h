@@ -170,6 +170,16 @@ qoq_status qoq_quantize_weights(const void *W_fp16, int64_t N, int64_t K, int gr
  * CTA index, and the unit, segment or contributor index. After such an error,
  * zero-fill the control bytes again. Size query: workspace == NULL stores the required size for
  * (M, N, K, group_size) in *workspace_bytes and returns QOQ_OK.
+ *
+ * Concurrency: problems whose token tile is at most 64 tokens (qoq_plan;
+ * decode batches) never have a CTA wait for one that may not have started,
+ * so such calls may run at the same time on different streams. Wider token
+ * tiles (prefill batches) run a kernel whose tile owners wait for the other
+ * CTAs that share their tile; its grid is sized so that all its CTAs are
+ * resident at once on an otherwise idle GPU. Two such launches overlapping on
+ * the device can take each other's SM slots: the waits then run out (1 s) and
+ * report QOQ_ERR_TIMEOUT (site 6) instead of hanging. Serialise prefill-size
+ * calls on one GPU.
  */
 qoq_status qoq_w4a8_gemm(const int8_t *X8, const int32_t *rowsum, const void *blob,
                          int64_t M, int64_t N, int64_t K, int group_size,
