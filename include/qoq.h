@@ -163,23 +163,18 @@ qoq_status qoq_quantize_weights(const void *W_fp16, int64_t N, int64_t K, int gr
  * where a bounded wait (1 s) gave up: the wait site (1 producer waiting for a
  * free stage, 2 MMA waiting for a drained accumulator, 3 MMA waiting for a
  * stage's operands, 4 dequantiser waiting for a stage's copies, 5 epilogue
- * waiting for an accumulator, 6 tile owner waiting for a contributor, 7 last
- * arriver of a split tile waiting for the owner's partial sums, 8 waiting
+ * waiting for an accumulator, 6 a flag wait (only the watchdog self-test
+ * uses it), 7 last arriver of a split tile waiting for the owner's partial
+ * sums, which the owner stores after it has arrived, 8 waiting
  * for every token row of the fused quantisation, 9 waiting for a free A/X
  * stage), the
  * CTA index, and the unit, segment or contributor index. After such an error,
  * zero-fill the control bytes again. Size query: workspace == NULL stores the required size for
  * (M, N, K, group_size) in *workspace_bytes and returns QOQ_OK.
  *
- * Concurrency: problems whose token tile is at most 64 tokens (qoq_plan;
- * decode batches) never have a CTA wait for one that may not have started,
- * so such calls may run at the same time on different streams. Wider token
- * tiles (prefill batches) run a kernel whose tile owners wait for the other
- * CTAs that share their tile; its grid is sized so that all its CTAs are
- * resident at once on an otherwise idle GPU. Two such launches overlapping on
- * the device can take each other's SM slots: the waits then run out (1 s) and
- * report QOQ_ERR_TIMEOUT (site 6) instead of hanging. Serialise prefill-size
- * calls on one GPU.
+ * Concurrency: a tile split between CTAs is finished by whichever of them
+ * arrives last, and no CTA waits for one that may not have started, so calls
+ * with separate workspaces may run at the same time on different streams.
  */
 qoq_status qoq_w4a8_gemm(const int8_t *X8, const int32_t *rowsum, const void *blob,
                          int64_t M, int64_t N, int64_t K, int group_size,

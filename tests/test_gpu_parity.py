@@ -421,12 +421,15 @@ def test_linear_graph_replays_are_bit_identical():
 
 
 def test_concurrent_gemms_on_two_streams():
-    """Two stream-K GEMMs running at the same time on two streams, each with
-    its own workspace, 20 launches each, interleaved: no CTA of either waits
-    for one that has not started, so every launch completes with status 0 and
-    the outputs of the serial run."""
+    """Stream-K GEMMs running at the same time on two streams, each with its
+    own workspace, 20 launches each, interleaved: decode sizes (decode kernel)
+    and prefill sizes (256-token tiles on CTA pairs, 128-token tiles; every
+    tile split between CTAs at these sizes). No CTA of either waits for one
+    that has not started, so every launch completes with status 0 and the
+    outputs of the serial run."""
     t = torch()
-    cases = [(16, 28672, 4096), (1, 4096, 14336), (64, 4096, 4096)]
+    cases = [(16, 28672, 4096), (1, 4096, 14336), (64, 4096, 4096), (2048, 4096, 4096), (1000, 6144, 4096),
+             (300, 4096, 4096)]
     probs = []
     for i, (M, N, K) in enumerate(cases):
         X = inputs.make_activations(M, K, seed=970 + i)

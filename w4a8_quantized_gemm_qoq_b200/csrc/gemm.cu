@@ -40,10 +40,13 @@
 //   * persistent stream-K at k-tile granularity: the (token tile, n-tile,
 //     k-tile) blocks, tiles in groups of up to 8 token tiles with the token
 //     tile fastest, are split evenly over at most one CTA (pair) per SM (pair). A tile cut
-//     between CTAs is finished by its owner -- the CTA holding the tile's
-//     first k-tile, which it reaches last -- after the other contributors
-//     (which reach their share of the tile first) have stored their INT32
-//     partial sums and raised a flag. The sum is exact in any order.
+//     between CTAs is finished by whichever of them arrives last on the
+//     tile's counter: usually its owner (the CTA holding the tile's first
+//     k-tile, which it reaches last), adding the partial sums the others
+//     stored; if another CTA of the tile started late, the owner stores its
+//     own partial sums instead and that CTA finishes the tile. No CTA waits
+//     for one that may not have started, so no co-residency is assumed. The
+//     sum is exact in any order.
 #include <algorithm>
 #include <cstring>
 
@@ -132,8 +135,8 @@ struct GemmParams {
     const int32_t *rowsum;
     void *out;
     int32_t *status;
-    int32_t *flags;         // [grid]: contributor c has stored its partial tile
-    int32_t *partials;      // [grid][TOK][128]: contributor c's partial sums
+    int32_t *flags;         // [grid]: arrival counter of the split tile owned by schedule unit c (bit 16: owner's sums stored)
+    int32_t *partials;      // [grid][2][TOK][128]: CTA c's partial sums as a contributor (0) and as an owner (1)
     int M, N, K, group;
     int NT, KT, MT;
     int NTw;                // n-tiles of the schedule: NT, or NT / 2 CTA pairs' 256-row tiles
@@ -152,6 +155,7 @@ struct SharedCtl {
     uint64_t final_bar[2];
     uint32_t tmem_base;
     int abort_flag;
+    int fix_old;            // the epilogue leader's arrival-counter value, broadcast
     // The owner's epilogue inputs of the current token tile, staged once per
     // tile: FP32(s_x) and (per-channel variant) the row sums.
     alignas(16) float tok_scale[256];
@@ -521,7 +525,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int te = threadIdx.x - (C::kWarpEpi0 + 4 * e) * 32;   // thread within the warpgroup
             const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
             const bool leader = (threadIdx.x == C::kWarpEpi0 * 32);
-            const bool poller = (warp == C::kWarpEpi0);
             // A part of the accumulator goes back to the issuer's CTA.
             auto acc_release = [&](uint64_t *bar) {
                 if (PAIR)
@@ -556,56 +559,59 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // Token columns of the tile that hold tokens (>= 1): the steps
                 // past them (a ragged last tile) are neither loaded nor stored.
                 const int m_live = (int)(p.M - m0 < TOK ? p.M - m0 : TOK);
-                // Owner (or sole computer) of a tile: the CTA holding its first
-                // k-tile. Contributors c_first .. c_last (none if c_last < c_first).
+                // Roles in a tile: sole computer (all of its k-tiles), owner (its
+                // first k-tile, not all) or contributor. The schedule units
+                // sharing a split tile, t_first (the owner) .. t_last, count their
+                // arrivals on the tile's counter, and whoever arrives last adds
+                // the others' partial sums and writes the tile. The owner arrives
+                // as it starts the tile's epilogue: with every contributor in
+                // (the usual case: contributors reach their share first), it
+                // finishes the tile from its accumulator; otherwise it stores its
+                // partial sums in its owner slot and sets bit 16 of the counter,
+                // and the last contributor, finding the owner arrived, waits only
+                // for that bit. No CTA waits for one that may not have started.
                 const bool owner = kt_lo == 0;
-                const uint32_t c_first = me + 1;
-                const uint32_t c_last =
-                    (!owner || kt_hi == KT) ? me : cta_of(tile_b + (uint32_t)KT - 1 - p.sk_base, BS, G);
+                const bool sole = owner && kt_hi == KT;
+                uint32_t t_first = me, t_last = me;
+                if (!sole) {
+                    t_first = owner ? me : cta_of(tile_b - p.sk_base, BS, G);
+                    t_last = cta_of(tile_b + (uint32_t)KT - 1 - p.sk_base, BS, G);
+                }
+                const int nparts = (int)(t_last - t_first + 1);
+                int32_t *cnt = p.flags + fidx(t_first);
+                // Contributors whose slots the finishing owner adds.
+                const uint32_t c_first = t_first + 1, c_last = t_last;
                 constexpr int CO = 16;   // token columns per step
                 // The parts this warpgroup reads: [h_lo, h_hi) of NP, PART columns each.
                 constexpr int NP = C::kHalves ? 2 : 1;
                 constexpr int PART = TOK / NP;
                 const int h_lo = C::kEpiGroups == 2 ? e : 0, h_hi = C::kEpiGroups == 2 ? e + 1 : NP;
-                const bool polls = c_last >= c_first;
                 float col_scale = 0.0f;
                 int col_zero = 0;
-                if (owner) {
-                    // Inputs that depend neither on the accumulator nor on the
-                    // contributors, fetched first: the weight row's scale (and
-                    // zero point), and the token scales (and row sums) of this
-                    // warpgroup's columns, staged in shared memory once per tile.
-                    // The previous segment's readers have passed its closing
-                    // barrier; the barrier after the accumulator wait orders
-                    // these stores before every read. While contributors are
-                    // polled, the polling warp takes no part in the staging.
+                // The tile's epilogue inputs that depend neither on the
+                // accumulator nor on other CTAs: the weight row's scale (and
+                // zero point), and the token scales (and row sums) of this
+                // warpgroup's columns, staged in shared memory once per tile.
+                // The previous segment's readers have passed its closing
+                // barrier; a barrier before the first read orders these stores.
+                auto stage_tile = [&]() {
                     col_scale = __half2float(reinterpret_cast<const __half *>(p.blob + p.off_scale)[n]);
                     if (MODE == 1)
                         col_zero = __half2int_rn(reinterpret_cast<const __half *>(p.blob + p.off_zero)[n]);
-                    if (!polls || !poller) {
-                        const bool skip = polls && e == 0;   // warp 0 of this warpgroup polls
-                        const int jend = h_hi * PART;
-                        for (int j = h_lo * PART + (skip ? te - 32 : te); j < jend; j += skip ? 96 : 128) {
-                            const int64_t m = m0 + j < p.M ? m0 + j : p.M - 1;
-                            ctl->tok_scale[j] = p.fp16_out ? __half2float(p.s_x[m]) : 0.0f;
-                            if (MODE == 1) ctl->tok_rowsum[j] = p.rowsum[m];
-                        }
+                    for (int j = h_lo * PART + te; j < h_hi * PART; j += 128) {
+                        const int64_t m = m0 + j < p.M ? m0 + j : p.M - 1;
+                        ctl->tok_scale[j] = p.fp16_out ? __half2float(p.s_x[m]) : 0.0f;
+                        if (MODE == 1) ctl->tok_rowsum[j] = p.rowsum[m];
                     }
+                };
+                // The owner's arrival, as it starts the tile's epilogue.
+                bool finish_here = sole;
+                if (owner && !sole) {
+                    if (leader) ctl->fix_old = atom_add_acq_rel_gpu(cnt, 1);
+                    named_bar_sync(kBarAll, NEPI);
+                    finish_here = (ctl->fix_old & 0xFFFF) == nparts - 1;
                 }
-                if (polls) {
-                    // Contributors reach their share of the tile first, so their
-                    // flags are usually up before this CTA's own accumulator is:
-                    // poll them now (lanes of the first epilogue warp in
-                    // parallel). The barrier orders everyone's partial-sum reads
-                    // after the polls.
-                    bool got = true;
-                    if (poller) {
-                        for (uint32_t c = c_first + (uint32_t)lane; c <= c_last && got; c += 32)
-                            got = wait_flag_bounded(p.flags + fidx(c), wd, (int)c);
-                        got = __all_sync(0xffffffffu, got);
-                    }
-                    if (named_bar_any(kBarAll, NEPI, !got)) break;
-                }
+                if (owner) stage_tile();
                 // Each part is handed back to its issuer right after its last
                 // TMEM load. Every lane spins on its own; the votes reconverge
                 // the warps before the named barriers, and all epilogue warps
@@ -613,7 +619,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int live_end = (m_live + CO - 1) / CO * CO;   // token columns read and stored
                 const uint32_t acc_addr = tmem_base + lane_addr + (uint32_t)(buf * C::kAccCols + prim * TOK);
                 const uint32_t acc2_addr = tmem_base + lane_addr + (uint32_t)(buf * C::kAccCols + (prim ^ 1) * TOK);
-                int32_t *slot = p.partials + (long long)blockIdx.x * TOK * kTileN;   // a contributor's partial tile
+                // This CTA's partial-sum slot for the tile: slot 0 as a
+                // contributor, slot 1 as an owner that is not the last to arrive.
+                auto slot_of = [&](uint32_t c, int role) {
+                    return p.partials + ((long long)fidx(c) * 2 + role) * TOK * kTileN;
+                };
+                int32_t *slot = slot_of(me, owner ? 1 : 0);
                 bool fail = false;
                 for (int h = h_lo; h < h_hi && !fail; ++h) {
                     const int bi = C::kHalves ? h : buf;
@@ -633,7 +644,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (lane == 0) acc_release(&ctl->acc_empty[bi]);
                         continue;
                     }
-                    if (C::kHalves && owner && !polls && p.fp16_out) {
+                    if (C::kHalves && sole && p.fp16_out) {
                         // A whole tile of this CTA (no partial sums): convert the
                         // part to FP16 in registers, hand the accumulator back,
                         // then store while the issuer runs the next tile.
@@ -675,9 +686,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                             __syncwarp();
                             if (lane == 0) acc_release(&ctl->acc_empty[bi]);
                         }
-                        if (!owner) {
-                            // Contributor: the live token columns of the partial
-                            // sums go to this CTA's slot.
+                        if (!finish_here) {
+                            // Not the last to arrive: the live token columns of
+                            // the partial sums go to this CTA's slot.
 #pragma unroll
                             for (int j = 0; j < CO; ++j)
                                 if (c0 + j < m_live) slot[(c0 + j) * kTileN + r] = (int32_t)v[j];
@@ -695,8 +706,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 int32_t t[8][4];
 #pragma unroll
                                 for (int cc = 0; cc < 8; ++cc) {
-                                    const int32_t *part =
-                                        p.partials + (long long)fidx(c + cc) * TOK * kTileN + c0 * kTileN + r;
+                                    const int32_t *part = slot_of(c + cc, 0) + c0 * kTileN + r;
 #pragma unroll
                                     for (int j = 0; j < 4; ++j)
                                         t[cc][j] = (c + cc <= c_last) ? ld_cg_s32(part + j * kTileN) : 0;
@@ -712,8 +722,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 int32_t t[4][CO];
 #pragma unroll
                                 for (int cc = 0; cc < 4; ++cc) {
-                                    const int32_t *part =
-                                        p.partials + (long long)fidx(c + cc) * TOK * kTileN + c0 * kTileN + r;
+                                    const int32_t *part = slot_of(c + cc, 0) + c0 * kTileN + r;
 #pragma unroll
                                     for (int j = 0; j < CO; ++j)
                                         t[cc][j] = (c + cc <= c_last) ? ld_cg_s32(part + j * kTileN) : 0;
@@ -736,18 +745,65 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 // Closing barrier of the segment (all epilogue warps): every
-                // read of the staged scales and of the contributors' partial
-                // sums is done, and (contributor) every partial-sum store comes
-                // before the leader's release store of the flag (release is
-                // cumulative, so the owner's acquire sees them all). It also
-                // carries the failure vote, so that all warps leave together.
+                // read of the staged scales and of other CTAs' partial sums is
+                // done, and every partial-sum store of this CTA comes before the
+                // leader's release (release is cumulative, so the finisher's
+                // acquire sees them all). It also carries the failure vote, so
+                // that all warps leave together.
                 if (named_bar_any(kBarAll, NEPI, fail)) break;
-                if (!owner) {
-                    if (leader) st_release_gpu(p.flags + blockIdx.x, 1);
-                    __syncwarp();
-                } else if (polls && poller) {
-                    for (uint32_t c = c_first + (uint32_t)lane; c <= c_last; c += 32) p.flags[fidx(c)] = 0;
-                    __syncwarp();
+                if (!sole) {
+                    if (owner) {
+                        if (finish_here) {
+                            if (leader) *cnt = 0;   // nobody touches the counter again in this launch
+                        } else {
+                            if (leader) red_or_release_gpu(cnt, 0x10000);   // the owner's sums are in
+                        }
+                    } else {
+                        // A contributor arrives; the last one finishes the tile.
+                        if (leader) ctl->fix_old = atom_add_acq_rel_gpu(cnt, 1);
+                        named_bar_sync(kBarAll, NEPI);
+                        if ((ctl->fix_old & 0xFFFF) == nparts - 1) {
+                            // The owner has arrived (it is running) but may not
+                            // have stored its sums yet.
+                            bool got = true;
+                            if (leader) got = wait_word_bounded(cnt, 0x10000, 0x10000, wd, kSiteLastOwner, (int)t_first);
+                            stage_tile();
+                            if (named_bar_any(kBarAll, NEPI, !got)) break;
+                            for (int h = h_lo; h < h_hi; ++h) {
+                                const int c_lo = h * PART;
+                                const int c_hi = live_end < c_lo + PART ? live_end : c_lo + PART;
+#pragma unroll 1
+                                for (int c0 = c_lo; c0 < c_hi; c0 += CO) {
+                                    uint32_t v[CO];
+#pragma unroll
+                                    for (int j = 0; j < CO; ++j) v[j] = 0u;
+                                    // The owner's slot, then every contributor's
+                                    // (this CTA's included); live columns only.
+#pragma unroll 1
+                                    for (uint32_t c = t_first; c <= t_last; ++c) {
+                                        const int32_t *part = slot_of(c, c == t_first ? 1 : 0) + c0 * kTileN + r;
+                                        int32_t t[CO];
+#pragma unroll
+                                        for (int j = 0; j < CO; ++j) t[j] = c0 + j < m_live ? ld_cg_s32(part + j * kTileN) : 0;
+#pragma unroll
+                                        for (int j = 0; j < CO; ++j) v[j] += (uint32_t)t[j];   // modulo 2^32: exact where the sum fits
+                                    }
+                                    if (p.fp16_out) {
+                                        store_outputs_fp16<CO, MODE>(&tmap_y, v, m0 + c0, n - lane, lane, col_scale, col_zero,
+                                                                     ctl->tok_scale + c0, ctl->tok_rowsum + c0,
+                                                                     out_stage + ((warp - C::kWarpEpi0) * 2 + obuf) * (16 * 32));
+                                        obuf ^= 1;
+                                    } else {
+                                        store_outputs_i32<CO, MODE>(static_cast<int32_t *>(p.out), p.M, p.N, v, m0 + c0, n,
+                                                                    col_zero, ctl->tok_rowsum + c0);
+                                    }
+                                }
+                            }
+                            // The staged scales are read; the counter is cleared for the next launch.
+                            if (named_bar_any(kBarAll, NEPI, false)) break;
+                            if (leader) *cnt = 0;
+                        }
+                    }
                 }
                 ++seg;
             }
@@ -779,8 +835,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // Number of two-CTA clusters of the paired kernel that can be resident at
 // once (clusters live inside one GPC, so this can be below SMs / 2); the
-// persistent schedule never launches more, so every cluster is resident and
-// stream-K partners can wait on one another. 0 when pairs cannot launch.
+// persistent schedule launches no more than one such wave. 0 when pairs cannot
+// launch.
 template <int TOK, int MODE, bool SAT>
 static int pair_clusters_of(int dev) {
     using C = GemmCfg<TOK, MODE, true>;
@@ -858,7 +914,7 @@ static qoq_status launch_gemm_t(const GemmArgs &a, cudaStream_t stream, int unit
     p.grid = (int)std::min<long long>(units_max, blocks);
     // The partial-sum slots are indexed by CTA: the workspace must hold one
     // per CTA of this grid.
-    if (scratch_bytes_for_grid(TOK, PAIR ? 2 * p.grid : p.grid) > a.ws_capacity) return QOQ_ERR_WORKSPACE;
+    if (scratch_bytes_for_grid(TOK, PAIR ? 2 * p.grid : p.grid, 2) > a.ws_capacity) return QOQ_ERR_WORKSPACE;
     // Whole tiles in data-parallel waves while at least one to two waves of
     // tiles remain for the stream-K tail, which evens out the last wave.
     const long long tiles = (long long)p.MT * p.NTw;
@@ -901,6 +957,7 @@ static qoq_status launch_gemm_t(const GemmArgs &a, cudaStream_t stream, int unit
 struct GemmPlan {
     int tok;
     bool pair;
+    bool decode;    // runs on the decode kernel (token tiles up to 64, not saturating)
     int units_max;
 };
 
@@ -911,6 +968,7 @@ static bool plan_gemm(int64_t M, int64_t N, int64_t K, int mode, bool saturating
     if (sms <= 0) return false;
     pl->tok = token_tile_for(M, N, K);
     pl->pair = false;
+    pl->decode = pl->tok <= kDecodeMaxTok && !saturating;
     pl->units_max = std::min(sms, kMaxGrid);
     if (pl->tok == 256 && (N / kTileN) % 2 == 0) {
         // 256-token tiles run on CTA pairs when the n-tiles pair up.
@@ -934,14 +992,14 @@ size_t gemm_scratch_bytes(int64_t M, int64_t N, int64_t K, int group, bool satur
     const int64_t NTw = pl.pair ? N / kTileN / 2 : N / kTileN;
     const int64_t blocks = ((M + pl.tok - 1) / pl.tok) * NTw * (K / kTileK);
     const int64_t units = std::min<int64_t>(pl.units_max, blocks);
-    return scratch_bytes_for_grid(pl.tok, pl.pair ? 2 * units : units);
+    return scratch_bytes_for_grid(pl.tok, pl.pair ? 2 * units : units, pl.decode ? 1 : 2);
 }
 
 template <int MODE>
 static qoq_status launch_gemm_mode(const GemmArgs &a, cudaStream_t stream) {
     GemmPlan pl;
     if (!plan_gemm(a.M, a.N, a.K, MODE, false, &pl)) return QOQ_ERR_CUDA;
-    if (pl.tok <= kDecodeMaxTok) return launch_decode_gemm(a, stream, pl.tok, pl.units_max);
+    if (pl.decode) return launch_decode_gemm(a, stream, pl.tok, pl.units_max);
     if (pl.tok == 128) return launch_gemm_t<128, MODE, false>(a, stream, pl.units_max);
     return pl.pair ? launch_gemm_t<256, MODE, true>(a, stream, pl.units_max)
                    : launch_gemm_t<256, MODE, false>(a, stream, pl.units_max);

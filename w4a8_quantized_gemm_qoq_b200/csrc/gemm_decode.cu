@@ -767,7 +767,7 @@ static qoq_status launch_decode_t(const GemmArgs &a, cudaStream_t stream, int un
     p.grid = (int)std::min<long long>(units_max, blocks);
     // The split tiles' sum buffers, one per CTA (the owner's index), must be
     // zero when the launch starts; every launch that completes leaves them so.
-    if (scratch_bytes_for_grid(TOK, p.grid) > a.ws_capacity) return QOQ_ERR_WORKSPACE;
+    if (scratch_bytes_for_grid(TOK, p.grid, 1) > a.ws_capacity) return QOQ_ERR_WORKSPACE;
     const long long tiles = (long long)p.MT * p.NT;
     const long long dp_tiles = tiles >= 2ll * p.grid ? (tiles / p.grid - 1) * p.grid : 0;
     p.dp_tiles = (uint32_t)dp_tiles;
@@ -780,7 +780,7 @@ static qoq_status launch_decode_t(const GemmArgs &a, cudaStream_t stream, int un
     if (FUSED) {
         // Codes, scales and row sums of the fused quantisation live in the
         // workspace after the partial sums.
-        const FusedLayout F = fused_layout(a.M, a.K, scratch_bytes_for_grid(TOK, kMaxGrid));
+        const FusedLayout F = fused_layout(a.M, a.K, workspace_bytes_for(a.M, a.N, a.K));
         if (F.total > a.ws_capacity) return QOQ_ERR_WORKSPACE;
         p.X = static_cast<const __half *>(a.X);
         p.X8q = reinterpret_cast<int8_t *>(ws + F.off_x8);

@@ -67,7 +67,7 @@ enum WaitSite : int {
     kSiteMmaOperands = 3,     // MMA warp waiting for a token tile / dequantised weights
     kSiteDequantFull = 4,     // dequant warp waiting for a stage's copies
     kSiteEpilogueAcc = 5,     // epilogue waiting for an accumulator
-    kSiteOwnerFlag = 6,       // tile owner waiting for a contributor's partial sums
+    kSiteOwnerFlag = 6,       // a global flag wait (the watchdog self-test)
     kSiteLastOwner = 7,       // last arriver of a split tile waiting for the owner's partial sums
     kSiteRowsDone = 8,        // fused activation quantisation: waiting for every token row
     kSiteXEmpty = 9,          // token-tile producer / dequantiser waiting for a free A/X stage

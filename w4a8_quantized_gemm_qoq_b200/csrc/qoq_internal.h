@@ -100,8 +100,11 @@ static_assert(256 + 4 * kMaxGrid == QOQ_WORKSPACE_CONTROL_BYTES, "workspace cont
 // tiles up to 64) as the sum buffers of its split tiles, which must be zero
 // when a launch starts and which every launch that completes leaves zero.
 constexpr int kDecodeMaxTok = 64;
-inline size_t scratch_bytes_for_grid(int tok, int64_t grid_ctas) {
-    return QOQ_WORKSPACE_CONTROL_BYTES + sizeof(int32_t) * (size_t)grid_ctas * tok * kTileN;
+// slots: partial-sum tiles per CTA (the decode kernel 1; the general kernel 2,
+// one for the tile it contributes to and one for the tile it owns, which a
+// CTA can hold at the same time when it is not the last to arrive at either).
+inline size_t scratch_bytes_for_grid(int tok, int64_t grid_ctas, int slots) {
+    return QOQ_WORKSPACE_CONTROL_BYTES + sizeof(int32_t) * (size_t)slots * grid_ctas * tok * kTileN;
 }
 
 // CTAs per SM of the decode kernel for a problem: one (the whole SM, deepest
@@ -110,7 +113,7 @@ int decode_ctas_per_sm(int64_t M, int64_t N, int64_t K);
 
 // Workspace size the size query reports: enough for any grid (kMaxGrid CTAs).
 inline size_t workspace_bytes_for(int64_t M, int64_t N, int64_t K) {
-    return scratch_bytes_for_grid(token_tile_for(M, N, K), kMaxGrid);
+    return scratch_bytes_for_grid(token_tile_for(M, N, K), kMaxGrid, 2);
 }
 
 // qoq_w4a8_linear keeps the quantised activations in the workspace, after
