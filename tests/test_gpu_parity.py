@@ -482,3 +482,18 @@ def test_linear_both_launch_configurations(fuse):
     r = subprocess.run([sys.executable, os.path.join(here, "linear_check.py"), str(2 - fuse)], env=env,
                        capture_output=True, text=True, timeout=900)
     assert r.returncode == 0 and "linear_check ok" in r.stdout, r.stdout[-2000:] + r.stderr[-4000:]
+
+
+def test_split_tiles_finished_by_a_late_contributor():
+    """Every contributor to a split tile arrives 300 us late (in a process of
+    its own: tests/gemm_late_check.py), so every split tile is finished by a
+    contributor from the owner's stored partial sums: bit-exact INT32 and FP16
+    within 1 ulp of the oracle, status 0, control words clear."""
+    import os
+    import subprocess
+    import sys
+    here = os.path.dirname(os.path.abspath(__file__))
+    env = dict(os.environ, QOQ_FORCE_CONFIG="lateck=300")
+    r = subprocess.run([sys.executable, os.path.join(here, "gemm_late_check.py")], env=env, capture_output=True,
+                       text=True, timeout=900)
+    assert r.returncode == 0 and "gemm_late_check ok" in r.stdout, r.stdout[-2000:] + r.stderr[-4000:]

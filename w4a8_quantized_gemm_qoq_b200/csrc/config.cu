@@ -14,6 +14,10 @@
 //     aqt=128|256|512        activation quantiser: threads per CTA
 //     aq2=1|2                activation quantiser: the two-pass form (1) or the
 //                            row in registers where it fits (2) at every shape
+//     lateck=1..10000        general GEMM kernel: every contributor to a split
+//                            tile arrives this many microseconds late (a
+//                            sleep), so that owners arrive first and the last
+//                            contributor finishes each tile (a test of that path)
 // Unknown keys and values are ignored.
 #include <cstdlib>
 #include <cstring>
@@ -40,6 +44,9 @@ const ForcedConfig &forced_config() {
             } else if (len > 4 && std::strncmp(p, "cps=", 4) == 0) {
                 v = std::atoi(p + 4);
                 if (v == 1 || v == 2) cfg.cps = v;
+            } else if (len > 7 && std::strncmp(p, "lateck=", 7) == 0) {
+                v = std::atoi(p + 7);
+                if (v >= 1 && v <= 10000) cfg.lateck = v;
             } else if (len > 4 && std::strncmp(p, "aq2=", 4) == 0) {
                 v = std::atoi(p + 4);
                 if (v == 1 || v == 2) cfg.aq2 = v;

@@ -137,6 +137,7 @@ struct GemmParams {
     int32_t *status;
     int32_t *flags;         // [grid]: arrival counter of the split tile owned by schedule unit c (bit 16: owner's sums stored)
     int32_t *partials;      // [grid][2][TOK][128]: CTA c's partial sums as a contributor (0) and as an owner (1)
+    long long late_arrival_ns;   // test override: contributors' arrivals delayed by this long (0)
     int M, N, K, group;
     int NT, KT, MT;
     int NTw;                // n-tiles of the schedule: NT, or NT / 2 CTA pairs' 256-row tiles
@@ -760,6 +761,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     } else {
                         // A contributor arrives; the last one finishes the tile.
+                        // (QOQ_FORCE_CONFIG=lateck=us delays the arrival, so
+                        // that owners arrive first and contributors finish.)
+                        if (leader && p.late_arrival_ns) {
+                            const uint64_t t_end = globaltimer_ns() + (uint64_t)p.late_arrival_ns;
+                            while (globaltimer_ns() < t_end) __nanosleep(1000);
+                        }
                         if (leader) ctl->fix_old = atom_add_acq_rel_gpu(cnt, 1);
                         named_bar_sync(kBarAll, NEPI);
                         if ((ctl->fix_old & 0xFFFF) == nparts - 1) {
@@ -897,6 +904,7 @@ static qoq_status launch_gemm_t(const GemmArgs &a, cudaStream_t stream, int unit
     uint8_t *ws = static_cast<uint8_t *>(a.ws);
     p.status = reinterpret_cast<int32_t *>(ws);
     p.flags = reinterpret_cast<int32_t *>(ws + 256);
+    p.late_arrival_ns = 1000ll * forced_config().lateck;
     p.partials = reinterpret_cast<int32_t *>(ws + 256 + sizeof(int32_t) * kMaxGrid);
     p.M = (int)a.M;
     p.N = (int)a.N;
