@@ -486,9 +486,10 @@ def test_linear_both_launch_configurations(fuse):
 
 def test_split_tiles_finished_by_a_late_contributor():
     """Every contributor to a split tile arrives 300 us late (in a process of
-    its own: tests/gemm_late_check.py), so every split tile is finished by a
-    contributor from the owner's stored partial sums: bit-exact INT32 and FP16
-    within 1 ulp of the oracle, status 0, control words clear."""
+    its own: tests/gemm_late_check.py), so every split tile of both GEMM
+    kernels is finished by a contributor from the owner's stored partial
+    sums: bit-exact INT32 and FP16 within 1 ulp of the oracle, status 0,
+    control words clear."""
     import os
     import subprocess
     import sys

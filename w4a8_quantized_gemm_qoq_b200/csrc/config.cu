@@ -14,7 +14,7 @@
 //     aqt=128|256|512        activation quantiser: threads per CTA
 //     aq2=1|2                activation quantiser: the two-pass form (1) or the
 //                            row in registers where it fits (2) at every shape
-//     lateck=1..10000        general GEMM kernel: every contributor to a split
+//     lateck=1..10000        GEMM kernels: every contributor to a split
 //                            tile arrives this many microseconds late (a
 //                            sleep), so that owners arrive first and the last
 //                            contributor finishes each tile (a test of that path)

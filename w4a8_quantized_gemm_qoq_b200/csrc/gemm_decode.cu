@@ -145,6 +145,7 @@ struct DecParams {
     uint32_t total_blocks, dp_tiles, sk_base;
     long long off_codes, off_scale, off_zero;
     int fp16_out;
+    long long late_arrival_ns;   // test override: contributors' arrivals delayed by this long (0)
 };
 
 struct DecCtl {
@@ -659,6 +660,12 @@ __global__ void __launch_bounds__(dec::kThreads, CPS)
                             if (leader) red_or_release_gpu(cnt, 0x10000);
                         } else {
                             // A contributor: arrive now, read the result later.
+                            // (QOQ_FORCE_CONFIG=lateck=us delays the arrival, so
+                            // that owners arrive first and contributors finish.)
+                            if (leader && p.late_arrival_ns) {
+                                const uint64_t t_end = globaltimer_ns() + (uint64_t)p.late_arrival_ns;
+                                while (globaltimer_ns() < t_end) __nanosleep(1000);
+                            }
                             if (leader) pend_old = atom_add_acq_rel_gpu(cnt, 1);
                             pend = true;
                             pend_first = (int)first;
@@ -776,6 +783,7 @@ static qoq_status launch_decode_t(const GemmArgs &a, cudaStream_t stream, int un
     p.off_scale = L.off_scale;
     p.off_zero = L.off_zero;
     p.fp16_out = a.fp16_out ? 1 : 0;
+    p.late_arrival_ns = 1000ll * forced_config().lateck;
     const int8_t *x8 = a.X8;
     if (FUSED) {
         // Codes, scales and row sums of the fused quantisation live in the

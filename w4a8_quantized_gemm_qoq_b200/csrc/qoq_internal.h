@@ -63,7 +63,7 @@ struct ForcedConfig {
     int kvt = 0;   // KV4 attention: 64-token tiles per warp
     int aqt = 0;   // activation quantiser: threads per CTA (one row per CTA)
     int aq2 = 0;   // activation quantiser: 1 = the two-pass form, 2 = the register form
-    int lateck = 0;   // general GEMM kernel: contributors' arrivals delayed by this many us (tests)
+    int lateck = 0;   // GEMM kernels: contributors' arrivals delayed by this many us (tests)
 };
 
 // Whether qoq_w4a8_linear quantises the activations inside the decode GEMM's
