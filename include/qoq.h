@@ -44,7 +44,7 @@
 extern "C" {
 #endif
 
-/* Leading workspace bytes that hold control words (status + flags). */
+/* Leading workspace bytes that hold control words (status + arrival counters). */
 #define QOQ_WORKSPACE_CONTROL_BYTES 1280
 
 typedef enum {
@@ -155,7 +155,7 @@ qoq_status qoq_quantize_weights(const void *W_fp16, int64_t N, int64_t K, int gr
  * Workspace: device memory of *workspace_bytes bytes, ZERO-FILLED by the caller
  * before its first use. Its first QOQ_WORKSPACE_CONTROL_BYTES bytes are
  * control words that every call which completes leaves zero again (an int32
- * status word at offset 0, then cross-CTA flags); the rest is scratch for the
+ * status word at offset 0, then per-tile arrival counters); the rest is scratch for the
  * stream-K partial sums. So one workspace serves any number of calls on one
  * stream; calls that may overlap on the device need separate workspaces. The
  * status word is 0, or a qoq_status code (QOQ_ERR_BAD_BLOB, QOQ_ERR_TIMEOUT)

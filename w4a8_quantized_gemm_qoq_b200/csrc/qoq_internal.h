@@ -90,13 +90,13 @@ inline int token_tile_for(int64_t M, int64_t N, int64_t K) {
     return 256;
 }
 
-// Workspace: [0, 256) status word + reserved; then int32 flags [kMaxGrid]
-// (together QOQ_WORKSPACE_CONTROL_BYTES, left zero by every call); then int32
-// partial tiles [kMaxGrid][tok][128] (scratch).
+// Workspace: [0, 256) status word + reserved; then int32 arrival counters
+// [kMaxGrid], one per split tile (together QOQ_WORKSPACE_CONTROL_BYTES, left
+// zero by every call); then int32 partial tiles (scratch, `slots` per CTA).
 static_assert(256 + 4 * kMaxGrid == QOQ_WORKSPACE_CONTROL_BYTES, "workspace control layout");
 
 // Workspace bytes a launch of `grid_ctas` CTAs with token tile `tok` uses:
-// the control words, then one INT32 partial tile per CTA. The general kernel
+// the control words, then `slots` INT32 partial tiles per CTA. The general kernel
 // (token tiles of 128 and 256) uses them as scratch; the decode kernel (token
 // tiles up to 64) as the sum buffers of its split tiles, which must be zero
 // when a launch starts and which every launch that completes leaves zero.

@@ -3,8 +3,8 @@
 // inside a pre-planned memory arena, a host thread that must not call into
 // the allocator while a CUDA graph or another library owns the device heap,
 // or an embedding runtime that forbids cudaMalloc after start-up. Instead of
-// a caller-supplied workspace, the stream-K scratch (status word, cross-CTA
-// flags and partial tiles) lives in one file-scope device array of a fixed
+// a caller-supplied workspace, the stream-K scratch (status word, arrival
+// counters and partial tiles) lives in one file-scope device array of a fixed
 // size that every GPU which loads the library keeps until the process exits.
 #include <cuda_runtime.h>
 #include <mutex>

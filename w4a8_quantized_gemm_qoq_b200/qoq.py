@@ -19,7 +19,7 @@ STATUS = {0: "QOQ_OK", 1: "QOQ_ERR_INVALID_ARG", 2: "QOQ_ERR_UNSUPPORTED", 3: "Q
           4: "QOQ_ERR_WORKSPACE", 5: "QOQ_ERR_BAD_BLOB", 6: "QOQ_ERR_CUDA", 7: "QOQ_ERR_TIMEOUT"}
 TILE = 128
 GROUP = 128
-WORKSPACE_CONTROL_BYTES = 1280   # status word + cross-CTA flags (include/qoq.h)
+WORKSPACE_CONTROL_BYTES = 1280   # status word + per-tile arrival counters (include/qoq.h)
 
 _lib = None
 
@@ -184,7 +184,7 @@ def quantize_weights(W, group_size: int = GROUP, blob=None, stream=None):
 
 class Workspace:
     """Zero-filled device workspace for the GEMM calls. Its leading control
-    bytes (the device status word, then cross-CTA flags) are left zero by
+    bytes (the device status word, then per-tile arrival counters) are left zero by
     every call that completes; the rest is scratch."""
 
     def __init__(self, nbytes: int, device="cuda"):
