@@ -22,7 +22,8 @@ def _same(got, want, what):
 
 
 @pytest.mark.parametrize("M,K,eps", [(1, 4096, 1e-5), (7, 4096, 1e-6), (33, 14336, 1e-5), (130, 8192, 1e-5),
-                                     (3, 32768, 1e-6), (5, 8, 1e-5), (260, 1024, 0.25), (17, 11008, 1e-5)])
+                                     (3, 32768, 1e-6), (5, 8, 1e-5), (260, 1024, 0.25), (17, 11008, 1e-5),
+                                     (5, 2048, 1e-5), (9, 512, 1e-5), (6, 6144, 1e-5)])
 def test_rmsnorm_quant_parity(M, K, eps):
     X = inputs.make_activations(M, K, seed=M + K, token_scale_span=(-3, 1))
     g = inputs.make_norm_weight(K, seed=K)
@@ -46,7 +47,8 @@ def test_rmsnorm_quant_degenerate_rows():
         _same(qoq.rmsnorm_quant(dev(X), dev(g), eps), P.rmsnorm_quant(X, g, eps), "degenerate eps=%g" % eps)
 
 
-@pytest.mark.parametrize("M,I", [(1, 14336), (9, 4096), (65, 11008), (3, 32768), (4, 8), (130, 1024)])
+@pytest.mark.parametrize("M,I", [(1, 14336), (9, 4096), (65, 11008), (3, 32768), (4, 8), (130, 1024),
+                                 (6, 8192), (5, 512), (11, 2048), (2, 20480)])
 def test_silu_mul_quant_parity(M, I):
     GU = inputs.make_gate_up(M, I, seed=M * 7 + I)
     _same(qoq.silu_mul_quant(dev(GU)), P.silu_mul_quant(GU), "silu %dx%d" % (M, I))

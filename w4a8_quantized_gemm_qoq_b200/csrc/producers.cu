@@ -12,29 +12,53 @@
 //   SiLU-gated:     h_k = (g_k / (1 + e^-g_k)) * u_k   (gate | up halves of a row)
 // then s = FP16(max_k |h| / 127), X8 = clamp(RNE(h / FP32(s)), -127, 127)
 // (0 where s == 0) and rowsum = sum_k X8. Every floating-point step is one
-// correctly rounded binary32 operation (__fdiv_rn, __fsqrt_rn, ...; the
-// quantising division takes the exact reciprocal shortcut of quant_math.cuh;
-// no contraction), the sum of squares is exact (128-bit integer accumulation,
-// then one rounding), and e^x is computed here from Cody and Waite's argument
-// reduction and the degree-7 Taylor polynomial, so that the codes these
-// floating-point values decide are reproducible bit for bit.
+// correctly rounded binary32 operation (no contraction), the sum of squares is
+// exact (integer accumulation, then one rounding), and e^x is computed here
+// from Cody and Waite's argument reduction and the degree-7 Taylor polynomial,
+// so that the codes these floating-point values decide are reproducible bit
+// for bit.
 //
-// B200 layout: one 256-thread CTA per token row (memory-bound: each row is
-// read once from HBM and written once as INT8). Thread t owns the 8-element
-// chunks t, t+256, ...; the FP32 row h lives in shared memory between the
-// passes, element i of chunk c at h[i * K/8 + c] so that a warp's accesses
-// fall in distinct banks (each thread reads back only its own chunks).
+// The two divisions whose divisor is fixed for the whole row, x / r and
+// h / s, are formed without a division instruction: with y = RN(1/b) (one
+// correctly rounded reciprocal per row), q0 = RN(a * y), the residual
+// a - b * q0 (exact in one FMA) and q = RN(q0 + residual * y) (one FMA).
+// Markstein's theorem (P. Markstein, IBM J. Res. Dev. 34(1), 1990; also
+// Muller et al., Handbook of Floating-Point Arithmetic, the section on
+// division with an FMA) states that q is then the correctly rounded quotient
+// whenever y is the correctly rounded reciprocal, q0 lies within one ulp of
+// a / b and nothing overflows or underflows; both hold for every operand
+// these kernels form (FP16 or bounded FP32 numerators, divisors in the normal
+// range). The quotient's integer code is taken with the 1.5 * 2^23 addition,
+// which rounds to nearest even exactly for |q| <= 2^22, after the clamp to
+// [-127, 127]; the low byte of the sum's bit pattern is then the code.
+//
+// B200 layout: the row stays in registers from its load to its codes. Rows of
+// up to 4096 elements (RMSNorm) or 2048 (SiLU-gated) belong to one warp each,
+// four rows per CTA, and every reduction is a warp shuffle; wider rows belong
+// to a CTA of 256 or 512 threads, with one shared-memory step per reduction.
+// Thread t of a row owns the 8-element chunks t, t + T, t + 2T, ... (T the
+// row's threads), so that every load of a chunk (16 bytes per thread) and
+// every store of its codes (8 bytes) is coalesced across the warp.
 #include <cuda_fp16.h>
 
 #include "qoq_device.cuh"
 #include "qoq_internal.h"
-#include "quant_math.cuh"
 
 namespace qoq {
 
 namespace {
 
-constexpr int kProdThreads = 256;
+constexpr int kWarpRows = 4;   // rows per CTA when a warp owns a row
+
+// Threads per row (TPR), and rows and threads per CTA.
+template <int TPR>
+struct RowCta {
+    static_assert(TPR == 32 || TPR == 256 || TPR == 512 || TPR == 1024, "row shapes");
+    static constexpr int kRows = TPR == 32 ? kWarpRows : 1;
+    static constexpr int kThreads = TPR * kRows;
+    static constexpr int kWarps = TPR / 32;   // warps of one row
+    static_assert(kWarps * 32 == TPR, "whole warps");
+};
 
 // ------------------------------------------------------------------ e^x
 
@@ -82,16 +106,6 @@ __device__ __forceinline__ void add128(U128 &a, const U128 &b) {
     a.lo = lo;
 }
 
-// |x| * 2^24 of an FP16 x (an integer below 2^40).
-__device__ __forceinline__ unsigned long long fp16_scaled(uint32_t bits) {
-    const uint32_t e = (bits >> 10) & 0x1Fu, f = bits & 0x3FFu;
-    return e ? (unsigned long long)(0x400u | f) << (e - 1) : (unsigned long long)f;
-}
-
-__device__ __forceinline__ void add_square(U128 &acc, uint32_t bits16) {
-    const unsigned long long v = fp16_scaled(bits16);
-    add128(acc, U128{v * v, __umul64hi(v, v)});
-}
 
 // S * 2^-48 rounded to binary32, ties to even. Every S formed here is 0 or at
 // least 1, so the result is 0 or normal.
@@ -132,79 +146,187 @@ __device__ __forceinline__ float rn32_scaled(U128 S) {
     return __fmul_rn(__uint2float_rn((unsigned)m), pow2_f32(drop - 48));
 }
 
-// ------------------------------------------------------ block reductions
 
-__device__ __forceinline__ U128 block_sum128(U128 v, U128 *red) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+// The exact squares of both FP16 halves of w, added to two 64-bit
+// accumulators. |x| * 2^24 = m << s with m the 11-bit significand (hidden bit
+// included for normal numbers) and s = max(e - 1, 0) for the exponent field e;
+// a square with s < 15 is added to a0 as (m << s)^2 = x^2 * 2^48, the others to
+// a1 as (m << (s - 15))^2 = x^2 * 2^48 / 2^30. Every such square is below 2^50
+// (2^52 for the infinity and NaN patterns), so a thread's 128 elements at
+// most, and a warp's 32 threads' sums, stay below 2^64 for finite inputs.
+__device__ __forceinline__ void add_squares(uint32_t w, unsigned long long &a0, unsigned long long &a1) {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        U128 w;
-        w.lo = __shfl_xor_sync(0xffffffffu, v.lo, o);
-        w.hi = __shfl_xor_sync(0xffffffffu, v.hi, o);
-        add128(v, w);
+    for (int k = 0; k < 2; ++k) {
+        const uint32_t h = k ? w >> 16 : w & 0xFFFFu;
+        const uint32_t e = (h >> 10) & 31u;
+        const uint32_t f = h & 0x3FFu;
+        const uint32_t m = e ? (f | 0x400u) : f;
+        const uint32_t s = e ? e - 1u : 0u;
+        const bool up = s >= 15u;
+        const uint32_t v = m << (up ? s - 15u : s);
+        const unsigned long long sq = (unsigned long long)v * v;
+        if (up)
+            a1 += sq;
+        else
+            a0 += sq;
     }
-    if (lane == 0) red[warp] = v;
-    __syncthreads();
-    U128 t = red[0];
-    for (int w = 1; w < kProdThreads / 32; ++w) add128(t, red[w]);
-    return t;   // every thread gets the same exact sum
 }
 
-__device__ __forceinline__ float block_max(float v, float *red) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    if (lane == 0) red[warp] = v;
-    __syncthreads();
-    float t = red[0];
-    for (int w = 1; w < kProdThreads / 32; ++w) t = fmaxf(t, red[w]);
-    return t;
-}
-
-__device__ __forceinline__ int block_sum(int v, int *red) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (lane == 0) red[warp] = v;
-    __syncthreads();
-    int t = 0;
-    for (int w = 0; w < kProdThreads / 32; ++w) t += red[w];
-    return t;
+// a / b correctly rounded, given y = RN(1/b) (Markstein's correction; the
+// conditions are stated at the top of this file).
+__device__ __forceinline__ float div_by_recip(float a, float b, float y) {
+    const float q0 = __fmul_rn(a, y);
+    const float res = __fmaf_rn(-q0, b, a);
+    return __fmaf_rn(res, y, q0);
 }
 
 __device__ __forceinline__ float half_lo(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w & 0xFFFFu))); }
 __device__ __forceinline__ float half_hi(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w >> 16))); }
+__device__ __forceinline__ uint32_t word_at(const uint4 &u, int i) {   // i = 0..3
+    return i < 2 ? (i == 0 ? u.x : u.y) : (i == 2 ? u.z : u.w);
+}
 
-// Quantise the FP32 row h (shared memory, element i of chunk c at
-// h[i * K/8 + c]; this thread's chunks) and write the codes, the scale and the
-// row sum of token m.
-__device__ __forceinline__ void quantize_row(const float *h, int K, float amax_row, int64_t m, int8_t *X8,
-                                             __half *s_x, int32_t *rowsum, int *red_i) {
-    __shared__ float s_shared, inv_shared;
-    if (threadIdx.x == 0) {
-        const __half sh = __float2half_rn(__fdiv_rn(amax_row, 127.0f));
-        s_x[m] = sh;
-        s_shared = __half2float(sh);
-        inv_shared = __frcp_rn(__half2float(sh));
-    }
-    __syncthreads();
-    const float s = s_shared, inv = inv_shared;
-    const int nc = K / 8;
-    int8_t *out = X8 + m * K;
-    int sum = 0;
-    for (int c = threadIdx.x; c * 8 < K; c += kProdThreads) {
-        uint32_t packed[2] = {0u, 0u};
+// ------------------------------------------------------ row reductions
+//
+// Over the TPR threads of one row; every thread receives the result. A warp
+// row reduces with shuffles alone; a CTA row adds one shared-memory exchange
+// (each reduction has its own array, so no barrier guards a reuse).
+
+struct RowRed {
+    U128 sq[32];
+    float mx[32];
+    int sum[32];
+};
+
+template <int TPR>
+__device__ __forceinline__ U128 row_sum_squares(unsigned long long a0, unsigned long long a1, RowRed &red) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int q = quant_code_recip(h[i * nc + c], s, inv, 127);
-            sum += q;
-            packed[i >> 2] |= (uint32_t)(q & 0xFF) << (8 * (i & 3));
-        }
-        *reinterpret_cast<uint2 *>(out + c * 8) = make_uint2(packed[0], packed[1]);
+    for (int o = 16; o > 0; o >>= 1) {
+        a0 += __shfl_xor_sync(0xffffffffu, a0, o);
+        a1 += __shfl_xor_sync(0xffffffffu, a1, o);
     }
-    if (rowsum != nullptr) {
-        const int t = block_sum(sum, red_i);
-        if (threadIdx.x == 0) rowsum[m] = t;
+    // S = a0 + a1 * 2^30
+    U128 S{a0, 0ull};
+    add128(S, U128{a1 << 30, a1 >> 34});
+    if constexpr (TPR > 32) {
+        const int warp = threadIdx.x >> 5;
+        if ((threadIdx.x & 31) == 0) red.sq[warp] = S;
+        __syncthreads();
+        S = red.sq[0];
+#pragma unroll
+        for (int w = 1; w < RowCta<TPR>::kWarps; ++w) add128(S, red.sq[w]);
+    }
+    return S;
+}
+
+template <int TPR>
+__device__ __forceinline__ float row_max(float v, RowRed &red) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    if constexpr (TPR > 32) {
+        const int warp = threadIdx.x >> 5;
+        if ((threadIdx.x & 31) == 0) red.mx[warp] = v;
+        __syncthreads();
+        v = red.mx[0];
+#pragma unroll
+        for (int w = 1; w < RowCta<TPR>::kWarps; ++w) v = fmaxf(v, red.mx[w]);
+    }
+    return v;
+}
+
+template <int TPR>
+__device__ __forceinline__ int row_sum(int v, RowRed &red) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if constexpr (TPR > 32) {
+        const int warp = threadIdx.x >> 5;
+        if ((threadIdx.x & 31) == 0) red.sum[warp] = v;
+        __syncthreads();
+        v = 0;
+#pragma unroll
+        for (int w = 0; w < RowCta<TPR>::kWarps; ++w) v += red.sum[w];
+    }
+    return v;
+}
+
+// ------------------------------------------------------ quantisation
+
+// Code byte of the quotient q, rounded to nearest even through the 1.5 * 2^23
+// addition: the low byte of the sum's pattern is the code. kClamp first
+// clamps q to [-127, 127]. Without it q must already lie below 127.5 in
+// magnitude, which holds whenever the row's scale is a normal FP16 number: s is
+// max|h| / 127 rounded to FP32 and then to FP16, with relative errors of at most
+// 2^-24 and 2^-11, so |h / s| <= 127 / ((1 - 2^-24)(1 - 2^-11)) < 127.1.
+template <bool kClamp>
+__device__ __forceinline__ uint32_t code_bits(float q) {
+    if constexpr (kClamp) q = fminf(fmaxf(q, -127.0f), 127.0f);
+    return __float_as_uint(__fadd_rn(q, 12582912.0f));
+}
+
+// Bytes 0 of a, b, c, d as one word (a in the lowest byte).
+__device__ __forceinline__ uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    return __byte_perm(__byte_perm(a, b, 0x0040u), __byte_perm(c, d, 0x0040u), 0x5410u);
+}
+
+// Codes of this thread's chunks: chunk j is the row's chunk c = t + TPR * j,
+// valid when below nc, and row_chunk(j, c, h) yields its 8 FP32 values.
+// Returns this thread's sum of the codes.
+template <int TPR, int CPT, bool kClamp, typename RowChunk>
+__device__ __forceinline__ int store_codes(RowChunk &row_chunk, int t, int nc, float s, float y, uint2 *out) {
+    int sum = 0;
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) {
+        const int c = t + TPR * j;
+        if (c < nc) {
+            float h[8];
+            row_chunk(j, c, h);
+            uint32_t b[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) b[i] = code_bits<kClamp>(div_by_recip(h[i], s, y));
+            const uint32_t lo = pack_low_bytes(b[0], b[1], b[2], b[3]);
+            const uint32_t hi = pack_low_bytes(b[4], b[5], b[6], b[7]);
+            out[c] = make_uint2(lo, hi);
+            sum = __dp4a((int)lo, 0x01010101, sum);
+            sum = __dp4a((int)hi, 0x01010101, sum);
+        }
+    }
+    return sum;
+}
+
+// Quantise the FP32 row h (this thread's max |h| in amax; row_chunk as in
+// store_codes) and write its codes, scale and code sum.
+template <int TPR, int CPT, typename RowChunk>
+__device__ __forceinline__ void quantize_row(RowChunk row_chunk, float amax, int t, int nc, int64_t m,
+                                             int64_t width, int8_t *__restrict__ X8, __half *__restrict__ s_x,
+                                             int32_t *__restrict__ rowsum, RowRed &red) {
+    amax = row_max<TPR>(amax, red);
+    const __half sh = __float2half_rn(__fdiv_rn(amax, 127.0f));
+    float s = __half2float(sh);
+    float y = __frcp_rn(s);
+    if (!(s > 0.0f) || isinf(s)) {
+        // s == 0: every code is 0 by definition; s == inf: every h / s is
+        // 0. The substitute divisor 1 with reciprocal 0 gives q = 0 below.
+        s = 1.0f;
+        y = 0.0f;
+    }
+    uint2 *out = reinterpret_cast<uint2 *>(X8 + m * width);
+    int sum = s >= 6.103515625e-05f   // 2^-14, the smallest normal FP16
+                  ? store_codes<TPR, CPT, false>(row_chunk, t, nc, s, y, out)
+                  : store_codes<TPR, CPT, true>(row_chunk, t, nc, s, y, out);
+    if (rowsum != nullptr) sum = row_sum<TPR>(sum, red);
+    if (t == 0) {
+        s_x[m] = sh;
+        if (rowsum != nullptr) rowsum[m] = sum;
+    }
+}
+
+// h = (x / r) * gamma for the 8 elements of one chunk (yr = RN(1/r)).
+__device__ __forceinline__ void rms_chunk(const uint4 &xv, const uint4 &gv, float r, float yr, float (&h)[8]) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t xw = word_at(xv, i), gw = word_at(gv, i);
+        h[2 * i] = __fmul_rn(div_by_recip(half_lo(xw), r, yr), half_lo(gw));
+        h[2 * i + 1] = __fmul_rn(div_by_recip(half_hi(xw), r, yr), half_hi(gw));
     }
 }
 
@@ -212,137 +334,176 @@ __device__ __forceinline__ void quantize_row(const float *h, int K, float amax_r
 
 // --------------------------------------------------------------- kernels
 
-__global__ void __launch_bounds__(kProdThreads) rmsnorm_quant_kernel(const __half *__restrict__ X,
-                                                                     const __half *__restrict__ gamma, int K,
-                                                                     float eps, int8_t *__restrict__ X8,
-                                                                     __half *__restrict__ s_x,
-                                                                     int32_t *__restrict__ rowsum) {
-    extern __shared__ float h[];   // [K]
-    __shared__ U128 red128[kProdThreads / 32];
-    __shared__ float red_f[kProdThreads / 32];
-    __shared__ int red_i[kProdThreads / 32];
-    __shared__ float r_shared;
-    griddep_wait();
-    griddep_launch_dependents();
-    const int64_t m = blockIdx.x;
-    const __half *row = X + m * K;
-    const int nc = K / 8;   // chunks per row; element i of chunk c sits at h[i * nc + c] (no bank conflicts)
-
-    // Pass 1: the row's exact sum of squares; keep x (FP32) in shared memory.
-    U128 acc{0ull, 0ull};
-    for (int c = threadIdx.x; c * 8 < K; c += kProdThreads) {
-        const uint4 u = *reinterpret_cast<const uint4 *>(row + c * 8);
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            add_square(acc, w[i] & 0xFFFFu);
-            add_square(acc, w[i] >> 16);
-            h[(2 * i) * nc + c] = half_lo(w[i]);
-            h[(2 * i + 1) * nc + c] = half_hi(w[i]);
-        }
-    }
-    const U128 S = block_sum128(acc, red128);
-    if (threadIdx.x == 0) {
-        const float ss = rn32_scaled(S);
-        const float ms = __fdiv_rn(ss, (float)K);
-        r_shared = __fsqrt_rn(__fadd_rn(ms, eps));
-    }
-    __syncthreads();
-    const float r = r_shared;
-
-    // Pass 2: h = (x / r) * gamma in place, and the row's max |h|.
-    float amax = 0.0f;
-    for (int c = threadIdx.x; c * 8 < K; c += kProdThreads) {
-        const uint4 gu = *reinterpret_cast<const uint4 *>(gamma + c * 8);
-        const uint32_t g[4] = {gu.x, gu.y, gu.z, gu.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float h0 = __fmul_rn(__fdiv_rn(h[(2 * i) * nc + c], r), half_lo(g[i]));
-            const float h1 = __fmul_rn(__fdiv_rn(h[(2 * i + 1) * nc + c], r), half_hi(g[i]));
-            h[(2 * i) * nc + c] = h0;
-            h[(2 * i + 1) * nc + c] = h1;
-            amax = fmaxf(amax, fmaxf(fabsf(h0), fabsf(h1)));
-        }
-    }
-    amax = block_max(amax, red_f);
-    quantize_row(h, K, amax, m, X8, s_x, rowsum, red_i);
+// Launch bounds: CTAs per SM the register budget must allow.
+template <int TPR, int CPT, bool kWide>
+constexpr int row_min_blocks() {
+    if constexpr (TPR == 32) return kWide ? 3 : (CPT >= 16 ? 5 : 4);   // kWide: 128 FP32 values kept per thread
+    return TPR == 256 ? 2 : 1;
 }
 
-__global__ void __launch_bounds__(kProdThreads) silu_mul_quant_kernel(const __half *__restrict__ GU, int I,
-                                                                      int8_t *__restrict__ X8,
-                                                                      __half *__restrict__ s_x,
-                                                                      int32_t *__restrict__ rowsum) {
-    extern __shared__ float h[];   // [I]
-    __shared__ float red_f[kProdThreads / 32];
-    __shared__ int red_i[kProdThreads / 32];
+// kKeepH: the normalised row stays in registers between its max and its
+// codes; otherwise it is formed a second time for the codes (fewer registers,
+// more CTAs per SM).
+template <int TPR, int CPT, bool kKeepH>
+__global__ void __launch_bounds__(RowCta<TPR>::kThreads, (row_min_blocks<TPR, CPT, kKeepH && CPT >= 16>()))
+    rmsnorm_quant_kernel(const __half *__restrict__ X, const __half *__restrict__ gamma, int64_t M, int K,
+                         float eps, int8_t *__restrict__ X8, __half *__restrict__ s_x,
+                         int32_t *__restrict__ rowsum) {
+    __shared__ RowRed red;
     griddep_wait();
     griddep_launch_dependents();
-    const int64_t m = blockIdx.x;
-    const int nc = I / 8;   // chunks per row; element i of chunk c sits at h[i * nc + c]
-    const __half *gate = GU + m * 2 * (int64_t)I;
-    const __half *up = gate + I;
+    const int t = threadIdx.x % TPR;
+    const int64_t m = (int64_t)blockIdx.x * RowCta<TPR>::kRows + threadIdx.x / TPR;
+    if (m >= M) return;   // warp rows only: a CTA row always exists
+    const int nc = K >> 3;
+    const uint4 *row = reinterpret_cast<const uint4 *>(X + m * K);
+    const uint4 *g4 = reinterpret_cast<const uint4 *>(gamma);
+
+    uint4 xv[CPT];
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) {
+        const int c = t + TPR * j;
+        xv[j] = c < nc ? row[c] : make_uint4(0u, 0u, 0u, 0u);
+    }
+    // The row's exact sum of squares (zero chunks add nothing).
+    unsigned long long a0 = 0ull, a1 = 0ull;
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) add_squares(word_at(xv[j], i), a0, a1);
+    }
+    const U128 S = row_sum_squares<TPR>(a0, a1, red);
+    const float r = __fsqrt_rn(__fadd_rn(__fdiv_rn(rn32_scaled(S), (float)K), eps));
+    const float yr = __frcp_rn(r);
+
+    // h = (x / r) * gamma and the row's max |h|.
+    float hk[kKeepH ? CPT : 1][8];
     float amax = 0.0f;
-    for (int c = threadIdx.x; c * 8 < I; c += kProdThreads) {
-        const uint4 gv = *reinterpret_cast<const uint4 *>(gate + c * 8);
-        const uint4 uv = *reinterpret_cast<const uint4 *>(up + c * 8);
-        const uint32_t g[4] = {gv.x, gv.y, gv.z, gv.w};
-        const uint32_t u[4] = {uv.x, uv.y, uv.z, uv.w};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+    for (int j = 0; j < CPT; ++j) {
+        const int c = t + TPR * j;
+        if (c < nc) {
+            float h[8];
+            rms_chunk(xv[j], __ldg(g4 + c), r, yr, h);
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const float gf = j ? half_hi(g[i]) : half_lo(g[i]);
-                const float uf = j ? half_hi(u[i]) : half_lo(u[i]);
-                const float e = exp_cw(-gf);
-                const float sg = __fdiv_rn(gf, __fadd_rn(1.0f, e));
-                const float hv = __fmul_rn(sg, uf);
-                h[(2 * i + j) * nc + c] = hv;
-                amax = fmaxf(amax, fabsf(hv));
+            for (int i = 0; i < 8; ++i) {
+                amax = fmaxf(amax, fabsf(h[i]));
+                if constexpr (kKeepH) hk[j][i] = h[i];
             }
         }
     }
-    amax = block_max(amax, red_f);
-    quantize_row(h, I, amax, m, X8, s_x, rowsum, red_i);
+    auto row_chunk = [&](int j, int c, float (&h)[8]) {
+        if constexpr (kKeepH) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) h[i] = hk[j][i];
+        } else {
+            rms_chunk(xv[j], __ldg(g4 + c), r, yr, h);
+        }
+    };
+    quantize_row<TPR, CPT>(row_chunk, amax, t, nc, m, K, X8, s_x, rowsum, red);
+}
+
+template <int TPR, int CPT>
+__global__ void __launch_bounds__(RowCta<TPR>::kThreads, (row_min_blocks<TPR, CPT, false>()))
+    silu_mul_quant_kernel(const __half *__restrict__ GU, int64_t M, int I, int8_t *__restrict__ X8,
+                          __half *__restrict__ s_x, int32_t *__restrict__ rowsum) {
+    __shared__ RowRed red;
+    griddep_wait();
+    griddep_launch_dependents();
+    const int t = threadIdx.x % TPR;
+    const int64_t m = (int64_t)blockIdx.x * RowCta<TPR>::kRows + threadIdx.x / TPR;
+    if (m >= M) return;   // warp rows only: a CTA row always exists
+    const int nc = I >> 3;
+    const uint4 *gate = reinterpret_cast<const uint4 *>(GU + m * 2 * (int64_t)I);
+    const uint4 *up = gate + nc;
+
+    uint4 gv[CPT], uv[CPT];
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) {
+        const int c = t + TPR * j;
+        gv[j] = c < nc ? gate[c] : make_uint4(0u, 0u, 0u, 0u);
+        uv[j] = c < nc ? up[c] : make_uint4(0u, 0u, 0u, 0u);
+    }
+    // h = (g / (1 + e^-g)) * u and the row's max |h| (zero chunks give 0).
+    float hk[CPT][8];
+    float amax = 0.0f;
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t gw = word_at(gv[j], i >> 1), uw = word_at(uv[j], i >> 1);
+            const float gf = (i & 1) ? half_hi(gw) : half_lo(gw);
+            const float uf = (i & 1) ? half_hi(uw) : half_lo(uw);
+            const float sg = __fdiv_rn(gf, __fadd_rn(1.0f, exp_cw(-gf)));
+            hk[j][i] = __fmul_rn(sg, uf);
+            amax = fmaxf(amax, fabsf(hk[j][i]));
+        }
+    }
+    auto row_chunk = [&](int j, int, float (&h)[8]) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) h[i] = hk[j][i];
+    };
+    quantize_row<TPR, CPT>(row_chunk, amax, t, nc, m, I, X8, s_x, rowsum, red);
 }
 
 namespace {
 
-template <typename Kernel, typename... Args>
-cudaError_t launch_row_kernel(Kernel kernel, int64_t M, int width, cudaStream_t stream, Args... args) {
-    const size_t smem = (size_t)width * sizeof(float);
-    int dev = 0;
-    cudaError_t err = cudaGetDevice(&dev);
-    if (err != cudaSuccess) return err;
-    if (smem > 48 * 1024) {
-        err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (err != cudaSuccess) return err;
-    }
+template <typename... KArgs, typename... Args>
+cudaError_t launch_rows(void (*kernel)(KArgs...), int tpr, int64_t M, cudaStream_t stream, Args... args) {
+    const int rows = tpr == 32 ? kWarpRows : 1;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)M);
-    cfg.blockDim = dim3(kProdThreads);
-    cfg.dynamicSmemBytes = smem;
+    cfg.gridDim = dim3((unsigned)((M + rows - 1) / rows));
+    cfg.blockDim = dim3((unsigned)(tpr * rows));
+    cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = kProgrammaticLaunch ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, kernel, args...);
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
 }  // namespace
 
+// Row shapes by the number of 8-element chunks nc: a warp per row up to 512
+// chunks (RMSNorm) or 256 (SiLU-gated, which holds gate and up), then CTA rows
+// of 256 to 1024 threads with at most 8 chunks per thread (4096 chunks =
+// kMaxProducerWidth at most).
 cudaError_t launch_rmsnorm_quant(const void *X, const void *gamma, int64_t M, int64_t K, float eps, int8_t *X8,
                                  void *s_x, int32_t *rowsum, cudaStream_t stream) {
-    return launch_row_kernel(rmsnorm_quant_kernel, M, (int)K, stream, static_cast<const __half *>(X),
-                             static_cast<const __half *>(gamma), (int)K, eps, X8, static_cast<__half *>(s_x),
-                             rowsum);
+    const int nc = (int)(K / 8);
+    const auto *x = static_cast<const __half *>(X);
+    const auto *g = static_cast<const __half *>(gamma);
+    auto *s = static_cast<__half *>(s_x);
+    const bool keep = forced_config().prs != 2;
+#define QOQ_RMS(TPR, CPT, KEEP) \
+    launch_rows(rmsnorm_quant_kernel<TPR, CPT, KEEP>, TPR, M, stream, x, g, M, (int)K, eps, X8, s, rowsum)
+    if (nc <= 64) return keep ? QOQ_RMS(32, 2, true) : QOQ_RMS(32, 2, false);
+    if (nc <= 128) return keep ? QOQ_RMS(32, 4, true) : QOQ_RMS(32, 4, false);
+    if (nc <= 256) return keep ? QOQ_RMS(32, 8, true) : QOQ_RMS(32, 8, false);
+    if (nc <= 512) return keep ? QOQ_RMS(32, 16, true) : QOQ_RMS(32, 16, false);
+    if (nc <= 1024) return QOQ_RMS(256, 4, true);
+    if (nc <= 2048) return QOQ_RMS(256, 8, true);
+    return QOQ_RMS(512, 8, true);
+#undef QOQ_RMS
 }
 
 cudaError_t launch_silu_mul_quant(const void *GU, int64_t M, int64_t I, int8_t *X8, void *s_x, int32_t *rowsum,
                                   cudaStream_t stream) {
-    return launch_row_kernel(silu_mul_quant_kernel, M, (int)I, stream, static_cast<const __half *>(GU), (int)I, X8,
-                             static_cast<__half *>(s_x), rowsum);
+    const int nc = (int)(I / 8);
+    const auto *gu = static_cast<const __half *>(GU);
+    auto *s = static_cast<__half *>(s_x);
+    const bool wide = forced_config().pst == 2;
+#define QOQ_SILU(TPR, CPT) launch_rows(silu_mul_quant_kernel<TPR, CPT>, TPR, M, stream, gu, M, (int)I, X8, s, rowsum)
+    if (nc <= 64) return QOQ_SILU(32, 2);
+    if (nc <= 128) return QOQ_SILU(32, 4);
+    if (nc <= 256) return QOQ_SILU(32, 8);
+    if (nc <= 512) return QOQ_SILU(256, 2);
+    if (nc <= 1024) return QOQ_SILU(256, 4);
+    if (nc <= 2048) return wide ? QOQ_SILU(512, 4) : QOQ_SILU(256, 8);
+    return wide ? QOQ_SILU(1024, 4) : QOQ_SILU(512, 8);
+#undef QOQ_SILU
 }
 
 }  // namespace qoq

@@ -64,6 +64,8 @@ struct ForcedConfig {
     int aqt = 0;   // activation quantiser: threads per CTA (one row per CTA)
     int aq2 = 0;   // activation quantiser: 1 = the two-pass form, 2 = the register form
     int lateck = 0;   // GEMM kernels: contributors' arrivals delayed by this many us (tests)
+    int prs = 0;   // RMSNorm producer, warp rows: 1 = normalised row kept in registers, 2 = formed twice
+    int pst = 0;   // SiLU-gated producer, rows above 8192: 1 = narrower CTA shape, 2 = wider
 };
 
 // Whether qoq_w4a8_linear quantises the activations inside the decode GEMM's
@@ -152,7 +154,8 @@ cudaError_t launch_kv4_attention(const void *q, const uint8_t *kc, const void *k
                                  const void *vs, const void *vz, const int32_t *seq_lens, int64_t B, int64_t Hq,
                                  int64_t Hkv, int64_t Tmax, int64_t D, void *out, void *ws, cudaStream_t stream);
 
-// Row width limit of the fused producers (the FP32 row lives in shared memory).
+// Row width limit of the fused producers (the row lives in registers: at most
+// 8 chunks of 8 elements per thread of a 512-thread row, or 4 of a 1024-thread row).
 constexpr int kMaxProducerWidth = 32768;
 
 struct GemmArgs {
