@@ -1,5 +1,5 @@
-// Exact per-token quantisation arithmetic shared by the activation quantiser
-// and the fused producers.
+// Exact per-token quantisation arithmetic of the activation quantiser (the
+// stand-alone kernel and its form inside the decode GEMM's launch).
 #pragma once
 
 #include <cuda_runtime.h>
