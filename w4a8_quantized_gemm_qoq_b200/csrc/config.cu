@@ -18,9 +18,10 @@
 //                            tile arrives this many microseconds late (a
 //                            sleep), so that owners arrive first and the last
 //                            contributor finishes each tile (a test of that path)
-//     prs=1|2                RMSNorm producer, rows of up to 4096: keep the
-//                            normalised row in registers (1) or form it again
-//                            for the codes (2)
+//     prs=1|2|3              RMSNorm producer, rows of up to 4096: keep the
+//                            normalised row in registers (1), form it again
+//                            for the codes (2), or stage the input row in
+//                            shared memory and loop over it (3)
 //     pst=1|2                SiLU-gated producer, rows above 8192: the narrower
 //                            (1) or the wider (2) of its two CTA shapes
 // Unknown keys and values are ignored.
@@ -57,7 +58,7 @@ const ForcedConfig &forced_config() {
                 if (v == 1 || v == 2) cfg.aq2 = v;
             } else if (len > 4 && std::strncmp(p, "prs=", 4) == 0) {
                 v = std::atoi(p + 4);
-                if (v == 1 || v == 2) cfg.prs = v;
+                if (v >= 1 && v <= 3) cfg.prs = v;
             } else if (len > 4 && std::strncmp(p, "pst=", 4) == 0) {
                 v = std::atoi(p + 4);
                 if (v == 1 || v == 2) cfg.pst = v;

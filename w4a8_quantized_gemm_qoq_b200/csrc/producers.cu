@@ -268,26 +268,42 @@ __device__ __forceinline__ uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint3
     return __byte_perm(__byte_perm(a, b, 0x0040u), __byte_perm(c, d, 0x0040u), 0x5410u);
 }
 
+// Codes of one chunk c (8 FP32 values h) to out[c]; returns their sum.
+template <bool kClamp>
+__device__ __forceinline__ int code_chunk(const float (&h)[8], float s, float y, uint2 *out, int c) {
+    uint32_t b[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) b[i] = code_bits<kClamp>(div_by_recip(h[i], s, y));
+    const uint32_t lo = pack_low_bytes(b[0], b[1], b[2], b[3]);
+    const uint32_t hi = pack_low_bytes(b[4], b[5], b[6], b[7]);
+    out[c] = make_uint2(lo, hi);
+    return __dp4a((int)hi, 0x01010101, __dp4a((int)lo, 0x01010101, 0));
+}
+
 // Codes of this thread's chunks: chunk j is the row's chunk c = t + TPR * j,
 // valid when below nc, and row_chunk(j, c, h) yields its 8 FP32 values.
+// CPT == 0: a loop over c unrolled twice, and row_chunk gets j = -1 (the
+// row's values come from memory, not from per-thread arrays).
 // Returns this thread's sum of the codes.
 template <int TPR, int CPT, bool kClamp, typename RowChunk>
 __device__ __forceinline__ int store_codes(RowChunk &row_chunk, int t, int nc, float s, float y, uint2 *out) {
     int sum = 0;
-#pragma unroll
-    for (int j = 0; j < CPT; ++j) {
-        const int c = t + TPR * j;
-        if (c < nc) {
+    if constexpr (CPT == 0) {
+#pragma unroll 2
+        for (int c = t; c < nc; c += TPR) {
             float h[8];
-            row_chunk(j, c, h);
-            uint32_t b[8];
+            row_chunk(-1, c, h);
+            sum += code_chunk<kClamp>(h, s, y, out, c);
+        }
+    } else {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) b[i] = code_bits<kClamp>(div_by_recip(h[i], s, y));
-            const uint32_t lo = pack_low_bytes(b[0], b[1], b[2], b[3]);
-            const uint32_t hi = pack_low_bytes(b[4], b[5], b[6], b[7]);
-            out[c] = make_uint2(lo, hi);
-            sum = __dp4a((int)lo, 0x01010101, sum);
-            sum = __dp4a((int)hi, 0x01010101, sum);
+        for (int j = 0; j < CPT; ++j) {
+            const int c = t + TPR * j;
+            if (c < nc) {
+                float h[8];
+                row_chunk(j, c, h);
+                sum += code_chunk<kClamp>(h, s, y, out, c);
+            }
         }
     }
     return sum;
@@ -319,6 +335,13 @@ __device__ __forceinline__ void quantize_row(RowChunk row_chunk, float amax, int
         if (rowsum != nullptr) rowsum[m] = sum;
     }
 }
+
+// 16-byte asynchronous copy global -> shared (both 16-byte aligned), and the
+// wait for all of this thread's copies (a hardware wait, no polling).
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // h = (x / r) * gamma for the 8 elements of one chunk (yr = RN(1/r)).
 __device__ __forceinline__ void rms_chunk(const uint4 &xv, const uint4 &gv, float r, float yr, float (&h)[8]) {
@@ -403,6 +426,53 @@ __global__ void __launch_bounds__(RowCta<TPR>::kThreads, (row_min_blocks<TPR, CP
     quantize_row<TPR, CPT>(row_chunk, amax, t, nc, m, K, X8, s_x, rowsum, red);
 }
 
+// RMSNorm rows of up to 4096 elements staged in shared memory (K * 2 bytes
+// per warp): one warp per row, four rows per CTA. Each lane copies its own
+// chunks in and reads back only those, so no barrier is needed; the three
+// passes over the row (squares, max, codes) are loops unrolled twice, which
+// keeps the kernel's body small, and the normalised row is formed again for
+// its codes instead of being kept.
+__global__ void __launch_bounds__(kWarpRows * 32, 7)
+    rmsnorm_quant_srow_kernel(const __half *__restrict__ X, const __half *__restrict__ gamma, int64_t M, int K,
+                              float eps, int8_t *__restrict__ X8, __half *__restrict__ s_x,
+                              int32_t *__restrict__ rowsum) {
+    extern __shared__ uint4 srow[];   // [kWarpRows][K / 8]
+    __shared__ RowRed red;            // unused by warp rows
+    griddep_wait();
+    griddep_launch_dependents();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t m = (int64_t)blockIdx.x * kWarpRows + warp;
+    if (m >= M) return;
+    const int nc = K >> 3;
+    uint4 *xs = srow + (size_t)warp * nc;
+    const uint4 *row = reinterpret_cast<const uint4 *>(X + m * K);
+    const uint4 *g4 = reinterpret_cast<const uint4 *>(gamma);
+    for (int c = lane; c < nc; c += 32) cp_async16(xs + c, row + c);
+    cp_async_wait_all();
+
+    unsigned long long a0 = 0ull, a1 = 0ull;
+#pragma unroll 2
+    for (int c = lane; c < nc; c += 32) {
+        const uint4 v = xs[c];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) add_squares(word_at(v, i), a0, a1);
+    }
+    const U128 S = row_sum_squares<32>(a0, a1, red);
+    const float r = __fsqrt_rn(__fadd_rn(__fdiv_rn(rn32_scaled(S), (float)K), eps));
+    const float yr = __frcp_rn(r);
+
+    float amax = 0.0f;
+#pragma unroll 2
+    for (int c = lane; c < nc; c += 32) {
+        float h[8];
+        rms_chunk(xs[c], __ldg(g4 + c), r, yr, h);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(h[i]));
+    }
+    auto row_chunk = [&](int, int c, float (&h)[8]) { rms_chunk(xs[c], __ldg(g4 + c), r, yr, h); };
+    quantize_row<32, 0>(row_chunk, amax, lane, nc, m, K, X8, s_x, rowsum, red);
+}
+
 template <int TPR, int CPT>
 __global__ void __launch_bounds__(RowCta<TPR>::kThreads, (row_min_blocks<TPR, CPT, false>()))
     silu_mul_quant_kernel(const __half *__restrict__ GU, int64_t M, int I, int8_t *__restrict__ X8,
@@ -449,12 +519,13 @@ __global__ void __launch_bounds__(RowCta<TPR>::kThreads, (row_min_blocks<TPR, CP
 namespace {
 
 template <typename... KArgs, typename... Args>
-cudaError_t launch_rows(void (*kernel)(KArgs...), int tpr, int64_t M, cudaStream_t stream, Args... args) {
+cudaError_t launch_rows_smem(void (*kernel)(KArgs...), int tpr, int64_t M, size_t smem, cudaStream_t stream,
+                             Args... args) {
     const int rows = tpr == 32 ? kWarpRows : 1;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)((M + rows - 1) / rows));
     cfg.blockDim = dim3((unsigned)(tpr * rows));
-    cfg.dynamicSmemBytes = 0;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -462,6 +533,11 @@ cudaError_t launch_rows(void (*kernel)(KArgs...), int tpr, int64_t M, cudaStream
     cfg.attrs = attr;
     cfg.numAttrs = kProgrammaticLaunch ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_rows(void (*kernel)(KArgs...), int tpr, int64_t M, cudaStream_t stream, Args... args) {
+    return launch_rows_smem(kernel, tpr, M, 0, stream, args...);
 }
 
 }  // namespace
@@ -476,7 +552,11 @@ cudaError_t launch_rmsnorm_quant(const void *X, const void *gamma, int64_t M, in
     const auto *x = static_cast<const __half *>(X);
     const auto *g = static_cast<const __half *>(gamma);
     auto *s = static_cast<__half *>(s_x);
-    const bool keep = forced_config().prs != 2;
+    const int prs = forced_config().prs;
+    const bool keep = prs != 2;
+    if (prs == 3 && nc <= 512)   // at most 32 KB of shared memory per CTA
+        return launch_rows_smem(rmsnorm_quant_srow_kernel, 32, M, (size_t)kWarpRows * K * 2, stream, x, g, M,
+                                (int)K, eps, X8, s, rowsum);
 #define QOQ_RMS(TPR, CPT, KEEP) \
     launch_rows(rmsnorm_quant_kernel<TPR, CPT, KEEP>, TPR, M, stream, x, g, M, (int)K, eps, X8, s, rowsum)
     if (nc <= 64) return keep ? QOQ_RMS(32, 2, true) : QOQ_RMS(32, 2, false);

@@ -64,7 +64,7 @@ struct ForcedConfig {
     int aqt = 0;   // activation quantiser: threads per CTA (one row per CTA)
     int aq2 = 0;   // activation quantiser: 1 = the two-pass form, 2 = the register form
     int lateck = 0;   // GEMM kernels: contributors' arrivals delayed by this many us (tests)
-    int prs = 0;   // RMSNorm producer, warp rows: 1 = normalised row kept in registers, 2 = formed twice
+    int prs = 0;   // RMSNorm producer, warp rows: 1 = row kept in registers, 2 = formed twice, 3 = staged in smem
     int pst = 0;   // SiLU-gated producer, rows above 8192: 1 = narrower CTA shape, 2 = wider
 };
 
