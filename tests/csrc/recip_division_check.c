@@ -16,7 +16,9 @@
  *   2. b = every positive finite FP16 value, a = n_num numerators per b with
  *      quotients in [-256, 256], half of them within 4 ulp of a half-integer
  *      quotient (the quantisation h / s).
- * Prints "mismatches <count> of <checked>" and exits 1 on any mismatch. */
+ * Prints "mismatches <count> of <checked>" and exits 1 on any mismatch.
+ * Built with -DPLANT_NO_CORRECTION it returns q0 itself, which the sweeps
+ * must catch. */
 #include <math.h>
 #include <stdint.h>
 #include <stdio.h>
@@ -43,7 +45,12 @@ static uint32_t next32(void) {   /* xorshift64 */
 static float quotient(float a, float b, float y) {
     const float q0 = a * y;
     const float r = fmaf(-q0, b, a);
+#ifdef PLANT_NO_CORRECTION   /* a planted mistake: the uncorrected product */
+    (void)r;
+    return q0;
+#else
     return fmaf(r, y, q0);
+#endif
 }
 
 static long bad = 0, checked = 0;

@@ -13,11 +13,26 @@ import pytest
 HERE = os.path.dirname(os.path.abspath(__file__))
 
 
+def _build(tmp_path, *defines):
+    exe = str(tmp_path / ("recip_division_check" + "".join(defines)))
+    subprocess.check_call(["gcc", "-O2", "-std=c99", "-ffp-contract=off", *defines, "-o", exe,
+                           os.path.join(HERE, "csrc", "recip_division_check.c"), "-lm"])
+    return exe
+
+
 @pytest.mark.skipif(shutil.which("gcc") is None, reason="gcc not found")
 def test_markstein_quotient_is_correctly_rounded(tmp_path):
-    exe = str(tmp_path / "recip_division_check")
-    subprocess.check_call(["gcc", "-O2", "-std=c99", "-ffp-contract=off", "-o", exe,
-                           os.path.join(HERE, "csrc", "recip_division_check.c"), "-lm"])
-    out = subprocess.run([exe, "2000", "200"], capture_output=True, text=True, timeout=300)
+    out = subprocess.run([_build(tmp_path), "2000", "200"], capture_output=True, text=True, timeout=300)
     assert out.returncode == 0, out.stdout
     assert out.stdout.strip().startswith("mismatches 0 of")
+
+
+@pytest.mark.skipif(shutil.which("gcc") is None, reason="gcc not found")
+def test_the_sweeps_catch_a_missing_correction(tmp_path):
+    """Planted on the CPU: without the FMA correction the product q0 = a * y is
+    often one ulp off, and the sweeps must say so."""
+    out = subprocess.run([_build(tmp_path, "-DPLANT_NO_CORRECTION"), "200", "20"], capture_output=True, text=True,
+                         timeout=300)
+    assert out.returncode == 1
+    bad = int(out.stdout.strip().splitlines()[-1].split()[1])
+    assert bad > 1000

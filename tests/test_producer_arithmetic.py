@@ -20,25 +20,24 @@ from oracle import producers as P
 F32 = np.float32
 
 
-def _bucketed_sum_of_squares(x16: np.ndarray) -> list:
+def _bucketed_sum_of_squares(x16: np.ndarray, split: int = 15, shift: int = 30, hidden: bool = True) -> list:
     b = np.asarray(x16, dtype=np.float16).view(np.uint16).astype(np.int64)
     e = (b >> 10) & 31
     f = b & 1023
-    m = np.where(e > 0, f | 1024, f)
+    m = np.where(e > 0, f | 1024, f) if hidden else f
     s = np.where(e > 0, e - 1, 0)
-    up = s >= 15
-    v = m << np.where(up, s - 15, s)
+    up = s >= split
+    v = m << np.where(up, s - split, s)
     sq = v * v
-    assert int(sq[np.isfinite(np.asarray(x16, dtype=np.float16))].max(initial=0)) < 2 ** 50
     out = []
     for r in range(sq.shape[0]):
         a0 = int(sq[r][~up[r]].sum())
         a1 = int(sq[r][up[r]].sum())
-        out.append(a0 + (a1 << 30))
+        out.append(a0 + (a1 << shift))
     return out
 
 
-def test_two_bucket_sum_of_squares_equals_the_exact_sum():
+def _test_rows() -> np.ndarray:
     rng = np.random.default_rng(7)
     every = np.arange(0, 0x7C00, dtype=np.uint16)          # every non-negative finite FP16
     every = np.concatenate([every, every | 0x8000]).view(np.float16)
@@ -47,8 +46,28 @@ def test_two_bucket_sum_of_squares_equals_the_exact_sum():
     rows.append(np.full(4096, 6e-8, np.float16))             # the smallest subnormal everywhere
     wide = rng.standard_normal(4096) * np.exp(rng.uniform(-20, 11, 4096))
     rows.append(np.clip(wide, -65504, 65504).astype(np.float16))
-    X = np.stack(rows)
-    assert _bucketed_sum_of_squares(X) == [int(v) for v in P.exact_sum_of_squares(X)]
+    return np.stack(rows)
+
+
+def test_two_bucket_sum_of_squares_equals_the_exact_sum():
+    X = _test_rows()
+    b = np.asarray(X).view(np.uint16).astype(np.int64)
+    e = (b >> 10) & 31
+    v = np.where(e > 0, (b & 1023) | 1024, b & 1023) << np.where(e > 0, e - 1, 0)
+    largest = int(v.max())
+    # the largest square of the upper bucket, (v >> 15)^2, and of the lower, (2047 << 14)^2, are below 2^50
+    assert (largest >> 15) ** 2 < 2 ** 50 and ((2 ** 11 - 1) << 14) ** 2 < 2 ** 50
+    assert _bucketed_sum_of_squares(X) == [int(t) for t in P.exact_sum_of_squares(X)]
+
+
+def test_planted_bucket_mistakes_are_caught():
+    """Planted on the CPU: a wrong bucket boundary, a wrong scale of the
+    upper bucket, or a dropped hidden bit each changes some row's sum."""
+    X = _test_rows()
+    want = [int(t) for t in P.exact_sum_of_squares(X)]
+    assert _bucketed_sum_of_squares(X, split=14) != want
+    assert _bucketed_sum_of_squares(X, shift=28) != want
+    assert _bucketed_sum_of_squares(X, hidden=False) != want
 
 
 def test_accumulators_cannot_wrap():
